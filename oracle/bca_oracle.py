@@ -1,0 +1,304 @@
+"""fp64 CPU oracle for block-causal grouped-query attention with QK-RMSNorm.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this module.  It shares no code with the CUDA path and imports nothing from
+it.
+
+It is the plain definition of the operation, written out step by step in
+float64 with an explicit per-token mask (no tiling, no online softmax, no
+folding of scales):
+
+1. QK-normalisation (MAGI-1 §2.2.2, "QK normalization"; MAGI-1 notes §3.2.2,
+   "QK-Norm + GQA").  The norm is per-head RMSNorm with a learnable gain:
+   ``rmsnorm(x) = x / sqrt(mean_d x^2 + eps) * gamma``.  The notes' DiT block
+   sketch writes ``l2_normalize``; this oracle takes the RMS reading (the two
+   differ by sqrt(D) in the logit scale), and ``eps`` is a parameter with
+   default 1e-6.
+2. Grouped-query attention (MAGI-1 §2.2.2; notes §3.2.2 model table,
+   "128 heads (8 groups)"): query head ``h`` reads key/value head
+   ``h // (Hq // Hkv)`` (contiguous groups).
+3. Block-causal mask (MAGI-1 §2, Fig. 1; notes §2 and Fig. 1: full attention
+   inside a chunk, causal attention between chunks).  Query token i of
+   query chunk c may see key token j iff j's kv chunk index is at most
+   ``n_kv - n_q + c``: the query chunks are the last ``n_q`` chunks of the
+   key/value sequence (streaming layout: active chunks after the cached clean
+   chunks, MAGI-1 §2 and §2.4.4; identity when n_q == n_kv).
+4. Softmax attention with scale ``1/sqrt(D)`` (a reading: the pages give no
+   scale), ``O = softmax(scale * q~ k~^T + mask) v``; the log-sum-exp
+   ``lse = ln sum_j exp(scale * q~_i . k~_j)`` over unmasked j, natural log, in
+   units of the scaled logits.
+5. Backward (training layout; FLOP convention of MAGI-1 App. B.2.1: the
+   backward recomputes the forward), analytic in float64: dV = P^T dO,
+   dP = dO V^T, Delta = rowsum(dO * O), dS = P * (dP - Delta),
+   dq~ = scale dS k~, dk~ = scale dS^T q~, summed over each query-head group
+   for k and v, then the RMSNorm Jacobian back to the raw q and k, and the
+   gain gradients dgamma = sum over (batch, token, head) of dx~ * x_hat.
+
+Every function below is pinned by ``tests/test_oracle_pins.py`` against
+brute force, a library routine or an invariant; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["rms_norm", "rms_norm_backward", "chunk_of", "matched_kv_chunk",
+           "block_causal_mask", "forward", "forward_rows", "backward", "backward_rows",
+           "DEFAULT_EPS"]
+
+DEFAULT_EPS = 1e-6
+
+
+def _f64(x):
+    """Any array-like (numpy or torch, any float dtype) -> float64 ndarray."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu()
+        if str(x.dtype) == "torch.bfloat16":
+            x = x.float()
+        x = x.numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def rms_norm(x, gamma, eps=DEFAULT_EPS):
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gamma."""
+    x = _f64(x)
+    g = _f64(gamma)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * g
+
+
+def rms_norm_backward(x, gamma, dy, eps=DEFAULT_EPS):
+    """Gradients of y = rms_norm(x, gamma) given dy.
+
+    With r = 1/sqrt(mean(x^2) + eps), x_hat = x r and g = gamma * dy:
+    dx = r * (g - x_hat * mean(g * x_hat)), dgamma = sum over leading axes
+    of dy * x_hat.  Returns (dx, dgamma)."""
+    x = _f64(x)
+    gm = _f64(gamma)
+    dy = _f64(dy)
+    d = x.shape[-1]
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    xh = x * r
+    g = gm * dy
+    dx = r * (g - xh * np.sum(g * xh, axis=-1, keepdims=True) / d)
+    dgamma = np.sum((dy * xh).reshape(-1, d), axis=0)
+    return dx, dgamma
+
+
+def chunk_of(offsets, n_tokens):
+    """Chunk index of every token, from cumulative offsets [0, ..., n]."""
+    offs = np.asarray(offsets, dtype=np.int64)
+    idx = np.empty(n_tokens, dtype=np.int64)
+    for c in range(len(offs) - 1):
+        idx[offs[c]:offs[c + 1]] = c
+    return idx
+
+
+def matched_kv_chunk(q_chunk, n_q_chunks, n_kv_chunks):
+    """The kv chunk that holds query chunk ``q_chunk`` (tail-aligned)."""
+    return n_kv_chunks - n_q_chunks + np.asarray(q_chunk)
+
+
+def block_causal_mask(q_offsets, kv_offsets, rows=None):
+    """Boolean mask M[i, j]: query token i may attend key token j.
+
+    Built token by token from chunk ids, not from tile arithmetic."""
+    q_offsets = np.asarray(q_offsets)
+    kv_offsets = np.asarray(kv_offsets)
+    nq, nkv = len(q_offsets) - 1, len(kv_offsets) - 1
+    cq = chunk_of(q_offsets, int(q_offsets[-1]))
+    ck = chunk_of(kv_offsets, int(kv_offsets[-1]))
+    if rows is not None:
+        cq = cq[np.asarray(rows)]
+    return ck[None, :] <= matched_kv_chunk(cq, nq, nkv)[:, None]
+
+
+def _check(q, k, v, q_offsets, kv_offsets):
+    B, Sq, Hq, D = q.shape
+    Bk, Skv, Hkv, Dk = k.shape
+    assert v.shape == k.shape and Bk == B and Dk == D
+    assert Hq % Hkv == 0
+    assert q_offsets[0] == 0 and q_offsets[-1] == Sq
+    assert kv_offsets[0] == 0 and kv_offsets[-1] == Skv
+    assert len(q_offsets) <= len(kv_offsets)
+    return B, Sq, Hq, D, Skv, Hkv
+
+
+def _attend_rows(qn_rows, kn, vv, mask_rows, scale):
+    """Softmax attention of a block of normalised query rows [R, D] against
+    all normalised keys [S, D]; returns (O [R, D], lse [R], P [R, S])."""
+    s = scale * (qn_rows @ kn.T)
+    s = np.where(mask_rows, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = np.sum(p, axis=1, keepdims=True)
+    p = p / l
+    return p @ vv, (m + np.log(l))[:, 0], p
+
+
+def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=None,
+                 batches=None, scale=None, eps=DEFAULT_EPS, block=512):
+    """Forward on a subset of query rows.
+
+    ``rows`` is an int array of query-token indices; ``heads`` / ``batches``
+    restrict the query heads and batch elements (default all).  Returns
+    (out [nb, R, nh, D], lse [nb, nh, R]) in float64 for those rows only."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    q_offsets = np.asarray(q_offsets)
+    kv_offsets = np.asarray(kv_offsets)
+    B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
+    scale = 1.0 / np.sqrt(D) if not scale else float(scale)
+    rows = np.asarray(rows, dtype=np.int64)
+    heads = list(range(Hq)) if heads is None else list(heads)
+    batches = list(range(B)) if batches is None else list(batches)
+    group = Hq // Hkv
+    out = np.zeros((len(batches), len(rows), len(heads), D))
+    lse = np.zeros((len(batches), len(heads), len(rows)))
+    for bi, b in enumerate(batches):
+        kn_all = rms_norm(k[b], gamma_k, eps)            # [Skv, Hkv, D]
+        for hi, h in enumerate(heads):
+            hk = h // group
+            kn = kn_all[:, hk, :]
+            vv = v[b, :, hk, :]
+            for r0 in range(0, len(rows), block):
+                rr = rows[r0:r0 + block]
+                qn = rms_norm(q[b, rr, h, :], gamma_q, eps)
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                o, ls, _ = _attend_rows(qn, kn, vv, mask, scale)
+                out[bi, r0:r0 + len(rr), hi, :] = o
+                lse[bi, hi, r0:r0 + len(rr)] = ls
+    return out, lse
+
+
+def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS):
+    """Full forward.  Returns (out [B, Sq, Hq, D], lse [B, Hq, Sq]), float64."""
+    Sq = q.shape[1]
+    return forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k,
+                        rows=np.arange(Sq), scale=scale, eps=eps)
+
+
+def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
+             eps=DEFAULT_EPS):
+    """Full analytic backward in float64.
+
+    Returns dict(dq, dk, dv, dgamma_q, dgamma_k, out, lse); dq/dk are the
+    gradients with respect to the raw (pre-norm) q and k."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(dout)
+    gq = _f64(gamma_q)
+    gk = _f64(gamma_k)
+    q_offsets = np.asarray(q_offsets)
+    kv_offsets = np.asarray(kv_offsets)
+    B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
+    scale = 1.0 / np.sqrt(D) if not scale else float(scale)
+    group = Hq // Hkv
+    mask = block_causal_mask(q_offsets, kv_offsets)
+    dqn = np.zeros_like(q)
+    dkn = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    out = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Sq))
+    qn_all = rms_norm(q, gq, eps)
+    kn_all = rms_norm(k, gk, eps)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // group
+            qn = qn_all[b, :, h, :]
+            kn = kn_all[b, :, hk, :]
+            vv = v[b, :, hk, :]
+            o, ls, p = _attend_rows(qn, kn, vv, mask, scale)
+            out[b, :, h, :] = o
+            lse[b, h, :] = ls
+            g = do[b, :, h, :]
+            dv[b, :, hk, :] += p.T @ g
+            dp = g @ vv.T
+            delta = np.sum(g * o, axis=1, keepdims=True)
+            ds = p * (dp - delta)
+            dqn[b, :, h, :] = scale * (ds @ kn)
+            dkn[b, :, hk, :] += scale * (ds.T @ qn)
+    dq, dgq = rms_norm_backward(q, gq, dqn, eps)
+    dk, dgk = rms_norm_backward(k, gk, dkn, eps)
+    return dict(dq=dq, dk=dk, dv=dv, dgamma_q=dgq, dgamma_k=dgk, out=out, lse=lse)
+
+
+def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows=None,
+                  kv_rows=None, kv_heads=None, batches=None, scale=None, eps=DEFAULT_EPS,
+                  block=256):
+    """Exact backward on chosen rows, without a full backward.
+
+    * dq of query rows ``q_rows`` (all heads): needs only those rows' P, dP
+      and Delta.
+    * dk, dv of key rows ``kv_rows`` for kv heads ``kv_heads``: needs every
+      query row that sees those keys (rows are located from the mask) and
+      each such row's full softmax; cheap when the keys sit in the last chunk.
+
+    Returns dict(dq [nb, R, Hq, D], dk [nb, Rk, nkh, D], dv [nb, Rk, nkh, D]),
+    keys present only for the parts requested."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    do = _f64(dout)
+    gq = _f64(gamma_q)
+    gk = _f64(gamma_k)
+    q_offsets = np.asarray(q_offsets)
+    kv_offsets = np.asarray(kv_offsets)
+    B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
+    scale = 1.0 / np.sqrt(D) if not scale else float(scale)
+    group = Hq // Hkv
+    batches = list(range(B)) if batches is None else list(batches)
+    res = {}
+    if q_rows is not None:
+        q_rows = np.asarray(q_rows, dtype=np.int64)
+        dq = np.zeros((len(batches), len(q_rows), Hq, D))
+        for bi, b in enumerate(batches):
+            kn_all = rms_norm(k[b], gk, eps)
+            for r0 in range(0, len(q_rows), block):
+                rr = q_rows[r0:r0 + block]
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                dqn = np.zeros((len(rr), Hq, D))
+                for h in range(Hq):
+                    hk = h // group
+                    qn = rms_norm(q[b, rr, h, :], gq, eps)
+                    o, _, p = _attend_rows(qn, kn_all[:, hk, :], v[b, :, hk, :], mask, scale)
+                    g = do[b, rr, h, :]
+                    dp = g @ v[b, :, hk, :].T
+                    delta = np.sum(g * o, axis=1, keepdims=True)
+                    ds = p * (dp - delta)
+                    dqn[:, h, :] = scale * (ds @ kn_all[:, hk, :])
+                dq[bi, r0:r0 + len(rr)], _ = rms_norm_backward(q[b, rr], gq, dqn, eps)
+        res["dq"] = dq
+    if kv_rows is not None:
+        kv_rows = np.asarray(kv_rows, dtype=np.int64)
+        kv_heads = list(range(Hkv)) if kv_heads is None else list(kv_heads)
+        dk = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
+        dv = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
+        # every query row that sees at least one of the requested keys
+        cols_mask = block_causal_mask(q_offsets, kv_offsets)[:, kv_rows]
+        seeing = np.nonzero(cols_mask.any(axis=1))[0]
+        for bi, b in enumerate(batches):
+            kn_all = rms_norm(k[b], gk, eps)
+            for khi, hk in enumerate(kv_heads):
+                kn = kn_all[:, hk, :]
+                vv = v[b, :, hk, :]
+                dkn = np.zeros((len(kv_rows), D))
+                for h in range(hk * group, (hk + 1) * group):
+                    for r0 in range(0, len(seeing), block):
+                        rr = seeing[r0:r0 + block]
+                        qn = rms_norm(q[b, rr, h, :], gq, eps)
+                        mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                        o, _, p = _attend_rows(qn, kn, vv, mask, scale)
+                        g = do[b, rr, h, :]
+                        delta = np.sum(g * o, axis=1, keepdims=True)
+                        pc = p[:, kv_rows]
+                        dpc = g @ vv[kv_rows].T
+                        dsc = pc * (dpc - delta)
+                        dv[bi, :, khi, :] += pc.T @ g
+                        dkn += scale * (dsc.T @ qn)
+                dk[bi, :, khi, :], _ = rms_norm_backward(k[b, kv_rows, hk, :], gk, dkn, eps)
+        res["dk"] = dk
+        res["dv"] = dv
+    return res

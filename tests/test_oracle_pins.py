@@ -1,0 +1,364 @@
+"""Pins for the fp64 oracle: each test checks it against something other than
+itself (a hand-written fixture, brute force, a library routine, a closed
+form or an invariant that the method fixes), so that a dropped term, a wrong
+sign or index, or a transposed operand fails at least one of them."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import bca_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def offs(lens):
+    return np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+
+
+def rand_case(rng, B, q_lens, kv_lens, Hq, Hkv, D, gamma=True):
+    Sq, Skv = sum(q_lens), sum(kv_lens)
+    q = rng.standard_normal((B, Sq, Hq, D))
+    k = rng.standard_normal((B, Skv, Hkv, D))
+    v = rng.standard_normal((B, Skv, Hkv, D))
+    gq = 1 + 0.1 * rng.standard_normal(D) if gamma else np.ones(D)
+    gk = 1 + 0.1 * rng.standard_normal(D) if gamma else np.ones(D)
+    return q, k, v, gq, gk, offs(q_lens), offs(kv_lens)
+
+
+def read_mask_fixture(name):
+    rows, meta = [], {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line[0].isalpha():
+                key, *vals = line.split()
+                meta[key] = [int(x) for x in vals]
+            else:
+                rows.append([c == "1" for c in line])
+    return meta, np.array(rows)
+
+
+# ---------------------------------------------------------------- the mask
+
+@pytest.mark.parametrize("name", ["mask_train_2_1_3.txt", "mask_stream_2of3.txt"])
+def test_mask_matches_hand_written_fixture(name):
+    meta, want = read_mask_fixture(name)
+    got = orc.block_causal_mask(offs(meta["q_chunks"]), offs(meta["kv_chunks"]))
+    assert got.shape == want.shape
+    assert np.array_equal(got, want)
+
+
+# ------------------------------------------------------- brute force (loops)
+
+def brute_force(q, k, v, qo, ko, gq, gk, eps=1e-6):
+    """Pure-Python loops straight from the definition (tiny inputs only)."""
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    nq, nkv = len(qo) - 1, len(ko) - 1
+    scale = 1.0 / math.sqrt(D)
+
+    def chunk(o, t):
+        for c in range(len(o) - 1):
+            if o[c] <= t < o[c + 1]:
+                return c
+        raise AssertionError
+
+    def norm(x, g):
+        ms = sum(xx * xx for xx in x) / len(x)
+        r = 1.0 / math.sqrt(ms + eps)
+        return [xx * r * gg for xx, gg in zip(x, g)]
+
+    out = np.zeros((B, Sq, Hq, D))
+    lse = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            for i in range(Sq):
+                qi = norm(list(q[b, i, h]), list(gq))
+                ci = chunk(qo, i) + (nkv - nq)
+                logits = []
+                for j in range(Skv):
+                    if chunk(ko, j) <= ci:
+                        kj = norm(list(k[b, j, hk]), list(gk))
+                        logits.append((j, scale * sum(a * c for a, c in zip(qi, kj))))
+                mx = max(s for _, s in logits)
+                den = sum(math.exp(s - mx) for _, s in logits)
+                lse[b, h, i] = mx + math.log(den)
+                for d in range(D):
+                    out[b, i, h, d] = sum(math.exp(s - mx) / den * v[b, j, hk, d] for j, s in logits)
+    return out, lse
+
+
+@pytest.mark.parametrize("q_lens,kv_lens", [([2, 3, 1], [2, 3, 1]), ([3, 2], [2, 3, 2]),
+                                            ([1, 1, 1, 1], [1, 1, 1, 1])])
+def test_forward_matches_brute_force(q_lens, kv_lens):
+    rng = np.random.default_rng(11)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, q_lens, kv_lens, 4, 2, 4)
+    o, l = orc.forward(q, k, v, qo, ko, gq, gk)
+    ob, lb = brute_force(q, k, v, qo, ko, gq, gk)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, lb, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------- library special cases
+
+def torch_reference(q, k, v, qo, ko, gq, gk, eps=1e-6, mask=None):
+    """fp64 torch: F.rms_norm + repeat_interleave (GQA) + SDPA with a boolean
+    mask built here from per-token chunk ids."""
+    Q = torch.tensor(q)
+    K = torch.tensor(k)
+    V = torch.tensor(v)
+    D = Q.shape[-1]
+    Qn = F.rms_norm(Q, (D,), weight=torch.tensor(gq), eps=eps)
+    Kn = F.rms_norm(K, (D,), weight=torch.tensor(gk), eps=eps)
+    g = Q.shape[2] // K.shape[2]
+    Kn = Kn.repeat_interleave(g, dim=2)
+    Vr = V.repeat_interleave(g, dim=2)
+    if mask is None:
+        cq = torch.bucketize(torch.arange(Q.shape[1]), torch.tensor(qo[1:]), right=True)
+        ck = torch.bucketize(torch.arange(K.shape[1]), torch.tensor(ko[1:]), right=True)
+        shift = (len(ko) - 1) - (len(qo) - 1)
+        mask = ck[None, :] <= (cq[:, None] + shift)
+    o = F.scaled_dot_product_attention(Qn.transpose(1, 2), Kn.transpose(1, 2), Vr.transpose(1, 2),
+                                       attn_mask=mask)
+    return o.transpose(1, 2).numpy()
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,Hq,Hkv,D", [
+    ([7, 13, 5, 9], [7, 13, 5, 9], 6, 2, 16),
+    ([11, 4], [3, 8, 11, 4], 4, 4, 8),
+    ([33], [33], 3, 1, 32),
+])
+def test_forward_matches_torch_sdpa_fp64(q_lens, kv_lens, Hq, Hkv, D):
+    rng = np.random.default_rng(5)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, q_lens, kv_lens, Hq, Hkv, D)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    np.testing.assert_allclose(o, torch_reference(q, k, v, qo, ko, gq, gk), rtol=0, atol=1e-12)
+
+
+def test_single_chunk_is_full_bidirectional_attention():
+    rng = np.random.default_rng(6)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [40], [40], 4, 2, 16)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    full = torch_reference(q, k, v, qo, ko, gq, gk, mask=torch.ones(40, 40, dtype=torch.bool))
+    np.testing.assert_allclose(o, full, rtol=0, atol=1e-12)
+
+
+def test_unit_chunks_are_token_causal_attention():
+    rng = np.random.default_rng(7)
+    n = 17
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [1] * n, [1] * n, 2, 1, 8)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    causal = torch_reference(q, k, v, qo, ko, gq, gk,
+                             mask=torch.ones(n, n, dtype=torch.bool).tril())
+    np.testing.assert_allclose(o, causal, rtol=0, atol=1e-12)
+
+
+def test_lse_is_log_sum_exp_of_scaled_logits():
+    rng = np.random.default_rng(8)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [3, 5], [4, 3, 5], 2, 1, 8)
+    _, l = orc.forward(q, k, v, qo, ko, gq, gk)
+    Qn = F.rms_norm(torch.tensor(q), (8,), weight=torch.tensor(gq), eps=1e-6)[0]
+    Kn = F.rms_norm(torch.tensor(k), (8,), weight=torch.tensor(gk), eps=1e-6)[0, :, 0]
+    mask = torch.tensor(read_mask_like(qo, ko))
+    for h in range(2):
+        s = (Qn[:, h] @ Kn.T) / math.sqrt(8)
+        s = s.masked_fill(~mask, -math.inf)
+        np.testing.assert_allclose(l[0, h], torch.logsumexp(s, dim=1).numpy(), rtol=0, atol=1e-12)
+
+
+def read_mask_like(qo, ko):
+    # q chunk c sees kv chunks <= c + (n_kv - n_q), built from token loops
+    nq, nkv = len(qo) - 1, len(ko) - 1
+    m = np.zeros((qo[-1], ko[-1]), dtype=bool)
+    for c in range(nq):
+        m[qo[c]:qo[c + 1], :ko[c + nkv - nq + 1]] = True
+    return m
+
+
+# ------------------------------------------------------------- invariants
+
+def test_later_chunk_kv_does_not_change_earlier_outputs():
+    rng = np.random.default_rng(9)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [5, 6, 7], [5, 6, 7], 4, 2, 8)
+    o1, l1 = orc.forward(q, k, v, qo, ko, gq, gk)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, 11:] = rng.standard_normal(k2[:, 11:].shape) * 5
+    v2[:, 11:] = rng.standard_normal(v2[:, 11:].shape) * 5
+    o2, l2 = orc.forward(q, k2, v2, qo, ko, gq, gk)
+    assert np.array_equal(o1[:, :11], o2[:, :11])
+    assert np.array_equal(l1[:, :, :11], l2[:, :, :11])
+    assert not np.allclose(o1[:, 11:], o2[:, 11:])
+
+
+def test_constant_v_gives_v():
+    rng = np.random.default_rng(10)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [4, 4, 4], [4, 4, 4], 4, 2, 8)
+    c = rng.standard_normal((1, 1, 2, 8))
+    v = np.broadcast_to(c, v.shape).copy()
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    want = np.broadcast_to(np.repeat(c, 2, axis=2), o.shape)
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-13)
+
+
+def test_softmax_rows_sum_to_one_and_vanish_outside_the_mask():
+    # with v_j = e_j (one-hot, Skv <= D) the output row IS the softmax row
+    rng = np.random.default_rng(12)
+    lens = [3, 2, 4]
+    S = sum(lens)
+    q, k, _, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 2, 1, 16)
+    v = np.zeros((1, S, 1, 16))
+    v[0, np.arange(S), 0, np.arange(S)] = 1.0
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    p = o[0, :, :, :S]                      # [Sq, Hq, Skv]
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=0, atol=1e-14)
+    assert (p >= 0).all()
+    mask = read_mask_like(qo, ko)
+    assert (p[~np.broadcast_to(mask[:, None, :], p.shape)] == 0).all()
+    assert (p[np.broadcast_to(mask[:, None, :], p.shape)] > 0).all()
+
+
+def test_permutation_within_a_chunk_permutes_outputs():
+    rng = np.random.default_rng(13)
+    lens = [4, 6, 5]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 2, 2, 8)
+    perm = np.arange(15)
+    perm[4:10] = rng.permutation(np.arange(4, 10))
+    o1, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    o2, _ = orc.forward(q[:, perm], k[:, perm], v[:, perm], qo, ko, gq, gk)
+    np.testing.assert_allclose(o2, o1[:, perm], rtol=0, atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    rng = np.random.default_rng(14)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [3, 5], [3, 5], 6, 2, 8)
+    o1, l1 = orc.forward(q, k, v, qo, ko, gq, gk)
+    o2, l2 = orc.forward(q, np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2), qo, ko, gq, gk)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-14)
+
+
+def test_rms_norm_closed_forms_and_library():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((7, 32)) * rng.uniform(0.01, 10, (7, 1))
+    y = orc.rms_norm(x, np.ones(32), eps=1e-6)
+    ms = np.mean(x * x, axis=1)
+    np.testing.assert_allclose(np.mean(y * y, axis=1), ms / (ms + 1e-6), rtol=1e-13)
+    g = rng.standard_normal(32)
+    want = F.rms_norm(torch.tensor(x), (32,), weight=torch.tensor(g), eps=1e-6).numpy()
+    np.testing.assert_allclose(orc.rms_norm(x, g, 1e-6), want, rtol=0, atol=1e-13)
+
+
+def test_positive_token_rescaling_of_q_and_k_leaves_output_unchanged():
+    rng = np.random.default_rng(16)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [6, 6], [6, 6], 2, 1, 8)
+    sq = np.exp(rng.standard_normal((1, 12, 1, 1)))
+    sk = np.exp(rng.standard_normal((1, 12, 1, 1)))
+    o1, _ = orc.forward(q, k, v, qo, ko, gq, gk, eps=0.0)
+    o2, _ = orc.forward(q * sq, k * sk, v, qo, ko, gq, gk, eps=0.0)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    o3, _ = orc.forward(q * sq, k * sk, v, qo, ko, gq, gk, eps=1e-6)
+    np.testing.assert_allclose(o1, o3, rtol=0, atol=1e-4)
+
+
+def test_forward_rows_subset_matches_full():
+    rng = np.random.default_rng(17)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [5, 4], [6, 5, 4], 4, 2, 8)
+    o, l = orc.forward(q, k, v, qo, ko, gq, gk)
+    rows = np.array([0, 3, 5, 8])
+    o2, l2 = orc.forward_rows(q, k, v, qo, ko, gq, gk, rows, heads=[1, 3], batches=[1])
+    np.testing.assert_array_equal(o2, o[1:2][:, rows][:, :, [1, 3]])
+    np.testing.assert_array_equal(l2, l[1:2][:, [1, 3]][:, :, rows])
+
+
+# -------------------------------------------------------------- backward
+
+def oracle_loss(params, dout, qo, ko):
+    q, k, v, gq, gk = params
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    return float(np.sum(o * dout))
+
+
+def test_backward_matches_central_finite_differences():
+    rng = np.random.default_rng(18)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [2, 3], [2, 3], 4, 2, 4)
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk)
+    params = [q, k, v, gq, gk]
+    names = ["dq", "dk", "dv", "dgamma_q", "dgamma_k"]
+    h = 1e-6
+    for pi, name in enumerate(names):
+        base = params[pi]
+        num = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            pp = [p.copy() for p in params]
+            pp[pi][idx] += h
+            lp = oracle_loss(pp, do, qo, ko)
+            pp[pi][idx] -= 2 * h
+            lm = oracle_loss(pp, do, qo, ko)
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_matches_torch_autograd_fp64():
+    rng = np.random.default_rng(19)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [5, 7, 4], [5, 7, 4], 6, 2, 16)
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk)
+    T = [torch.tensor(x, requires_grad=True) for x in (q, k, v, gq, gk)]
+    D = 16
+    Qn = F.rms_norm(T[0], (D,), weight=T[3], eps=1e-6)
+    Kn = F.rms_norm(T[1], (D,), weight=T[4], eps=1e-6).repeat_interleave(3, dim=2)
+    Vr = T[2].repeat_interleave(3, dim=2)
+    mask = torch.tensor(read_mask_like(qo, ko))
+    o = F.scaled_dot_product_attention(Qn.transpose(1, 2), Kn.transpose(1, 2), Vr.transpose(1, 2),
+                                       attn_mask=mask).transpose(1, 2)
+    (o * torch.tensor(do)).sum().backward()
+    for t, name in zip(T, ["dq", "dk", "dv", "dgamma_q", "dgamma_k"]):
+        np.testing.assert_allclose(g[name], t.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
+    np.testing.assert_allclose(g["out"], o.detach().numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_rows_match_full_backward():
+    rng = np.random.default_rng(20)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [4, 5, 6], [3, 4, 5, 6], 4, 2, 8)
+    do = rng.standard_normal(q.shape)
+    full = orc.backward(q, k, v, do, qo, ko, gq, gk)
+    qr = np.array([0, 4, 9, 14])
+    kr = np.array([12, 13, 17])           # last chunk keys
+    part = orc.backward_rows(q, k, v, do, qo, ko, gq, gk, q_rows=qr, kv_rows=kr, kv_heads=[1])
+    np.testing.assert_allclose(part["dq"], full["dq"][:, qr], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dk"], full["dk"][:, kr][:, :, [1]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dv"], full["dv"][:, kr][:, :, [1]], rtol=0, atol=1e-12)
+
+
+def test_backward_structure_and_identities():
+    rng = np.random.default_rng(21)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [4, 5, 6], [4, 5, 6], 4, 2, 8)
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk, eps=0.0)
+    # dV summed over keys = dO summed over queries of the group (rows of P sum to 1)
+    for hk in range(2):
+        np.testing.assert_allclose(g["dv"][0, :, hk].sum(0), do[0, :, 2 * hk:2 * hk + 2].sum((0, 1)),
+                                   rtol=0, atol=1e-12)
+    # RMSNorm (eps = 0) is scale invariant, so raw gradients are orthogonal to the input
+    np.testing.assert_allclose(np.sum(g["dq"] * q, -1), 0, atol=1e-12)
+    np.testing.assert_allclose(np.sum(g["dk"] * k, -1), 0, atol=1e-12)
+    # keys of chunk c receive no gradient from queries of earlier chunks:
+    # changing q and dO of chunk 0 leaves dk, dv of chunks 1-2 unchanged
+    q2, do2 = q.copy(), do.copy()
+    q2[:, :4] = rng.standard_normal(q2[:, :4].shape)
+    do2[:, :4] = rng.standard_normal(do2[:, :4].shape)
+    g2 = orc.backward(q2, k, v, do2, qo, ko, gq, gk, eps=0.0)
+    np.testing.assert_allclose(g2["dk"][:, 4:], g["dk"][:, 4:], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(g2["dv"][:, 4:], g["dv"][:, 4:], rtol=0, atol=1e-13)
+    assert not np.allclose(g2["dk"][:, :4], g["dk"][:, :4])

@@ -1,0 +1,223 @@
+"""Block-causal grouped-query attention with QK-RMSNorm on B200 (sm_100a).
+
+Thin ctypes binding over ``libmagi_bca.so`` (C ABI in ``include/magi_bca.h``).
+This module only marshals arguments: PyTorch provides device memory and the
+current stream; every step of the computation runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback: if the library is missing or
+the device is not an sm_100 GPU, the calls raise.
+
+The operation (MAGI-1: Autoregressive Video Generation at Scale, §2 and
+Figure 1; §2.2.2): every query token attends to all tokens of its own chunk
+and of every earlier chunk; q and k are RMS-normalised per head with gains
+gamma_q / gamma_k; query head h reads kv head h // (Hq // Hkv).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
+           "magi_bca_status_string", "magi_bca_last_device_status", "MagiBcaError", "Dims", "library",
+           "library_path", "EXPORTED_SYMBOLS"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libmagi_bca.so")
+
+EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
+                    "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version"]
+
+
+class MagiBcaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: status {status} ({magi_bca_status_string(status)})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seqlen_q", ctypes.c_int32), ("seqlen_kv", ctypes.c_int32),
+                ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("n_q_chunks", ctypes.c_int32), ("n_kv_chunks", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Loads libmagi_bca.so (built in-tree by ``build.py``); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"{library_path} is missing: build it with "
+                           "`python -m block_causal_attention_gqa_b200.build` (no fallback exists)")
+    lib = ctypes.CDLL(library_path)
+    vp, i32p, f32p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p
+    dp = ctypes.POINTER(Dims)
+    lib.magi_bca_fwd.argtypes = [vp, vp, vp, i32p, i32p, f32p, f32p, vp, f32p, dp, vp]
+    lib.magi_bca_fwd.restype = ctypes.c_int
+    lib.magi_bca_bwd.argtypes = [vp, vp, vp, vp, vp, f32p, i32p, i32p, f32p, f32p, vp, vp, vp, f32p, f32p, vp,
+                                 ctypes.c_size_t, dp, vp]
+    lib.magi_bca_bwd.restype = ctypes.c_int
+    lib.magi_bca_bwd_workspace_size.argtypes = [dp]
+    lib.magi_bca_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.magi_bca_status_string.argtypes = [ctypes.c_int]
+    lib.magi_bca_status_string.restype = ctypes.c_char_p
+    lib.magi_bca_last_device_status.argtypes = []
+    lib.magi_bca_last_device_status.restype = ctypes.c_int
+    lib.magi_bca_fwd_schedule.argtypes = [i32p, i32p, dp, i32p, ctypes.c_int64]
+    lib.magi_bca_fwd_schedule.restype = ctypes.c_int64
+    lib.magi_bca_version.argtypes = []
+    lib.magi_bca_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def magi_bca_status_string(status: int) -> str:
+    return library().magi_bca_status_string(int(status)).decode()
+
+
+def magi_bca_last_device_status() -> int:
+    return int(library().magi_bca_last_device_status())
+
+
+def _offsets(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().numpy()
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+    if a.ndim != 1:
+        raise ValueError("chunk offsets must be a 1-D array")
+    return a
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def make_dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
+              softmax_scale=0.0, rms_eps=1e-6) -> Dims:
+    return Dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
+                float(softmax_scale), float(rms_eps))
+
+
+def _check_bf16(name, t, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16 (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _check_f32(name, t, shape):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous float32 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _stream_handle(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out=None, lse=None,
+                 softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True):
+    """Forward.  q [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] bf16; gammas fp32 [D];
+    offsets: host int arrays of chunk boundaries.  Returns (out, lse)."""
+    import torch
+    _check_bf16("q", q)
+    B, Sq, Hq, D = q.shape
+    _check_bf16("k", k)
+    Skv, Hkv = k.shape[1], k.shape[2]
+    _check_bf16("k", k, (B, Skv, Hkv, D))
+    _check_bf16("v", v, (B, Skv, Hkv, D))
+    _check_f32("gamma_q", gamma_q, (D,))
+    _check_f32("gamma_k", gamma_k, (D,))
+    qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_bf16("out", out, q.shape)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, Sq, device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _check_f32("lse", lse, (B, Hq, Sq))
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    with torch.cuda.device(q.device):
+        st = library().magi_bca_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _i32p(qo), _i32p(ko),
+                                    gamma_q.data_ptr(), gamma_k.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr() if lse is not None else None, ctypes.byref(dims),
+                                    _stream_handle(stream, q.device))
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_fwd")
+    return out, lse
+
+
+def magi_bca_bwd_workspace_size(dims: Dims) -> int:
+    return int(library().magi_bca_bwd_workspace_size(ctypes.byref(dims)))
+
+
+def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
+                 dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
+                 workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None):
+    """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
+    respect to the raw (pre-norm) q and k."""
+    import torch
+    _check_bf16("q", q)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    _check_bf16("k", k, (B, Skv, Hkv, D))
+    _check_bf16("v", v, (B, Skv, Hkv, D))
+    _check_bf16("out", out, q.shape)
+    _check_bf16("dout", dout, q.shape)
+    _check_f32("lse", lse, (B, Hq, Sq))
+    _check_f32("gamma_q", gamma_q, (D,))
+    _check_f32("gamma_k", gamma_k, (D,))
+    qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_bf16("dq", dq, q.shape)
+    _check_bf16("dk", dk, k.shape)
+    _check_bf16("dv", dv, v.shape)
+    if want_dgamma:
+        dgamma_q = torch.empty(D, device=q.device, dtype=torch.float32) if dgamma_q is None else dgamma_q
+        dgamma_k = torch.empty(D, device=q.device, dtype=torch.float32) if dgamma_k is None else dgamma_k
+    ws_bytes = magi_bca_bwd_workspace_size(dims)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), device=q.device, dtype=torch.uint8)
+    with torch.cuda.device(q.device):
+        st = library().magi_bca_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                                    lse.data_ptr(), _i32p(qo), _i32p(ko), gamma_q.data_ptr(), gamma_k.data_ptr(),
+                                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                    dgamma_q.data_ptr() if dgamma_q is not None else None,
+                                    dgamma_k.data_ptr() if dgamma_k is not None else None,
+                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(dims), _stream_handle(stream, q.device))
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_bwd")
+    return dq, dk, dv, dgamma_q, dgamma_k
+
+
+def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim) -> np.ndarray:
+    """Host-only: the forward's work units as an int32 array [n_units, 8]."""
+    qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
+    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1)
+    lib = library()
+    n = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), None, 0)
+    if n < 0:
+        raise MagiBcaError(int(n), "magi_bca_fwd_schedule")
+    buf = np.zeros((max(n, 1), 8), dtype=np.int32)
+    n2 = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), _i32p(buf), n)
+    assert n2 == n
+    return buf[:n]

@@ -1,0 +1,236 @@
+// C ABI of libmagi_bca: argument checks, the schedule cache, TMA descriptors
+// and kernel dispatch.  See include/magi_bca.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <vector>
+
+#include "../../include/magi_bca.h"
+#include "bca_kernels.h"
+#include "bca_sched.h"
+
+namespace magi {
+
+// Device status word written by bounded waits that give up (0 = fine).
+__device__ int g_device_status;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mutex;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+struct DeviceState {
+  int* status = nullptr;
+  bool checked = false;
+  bool supported = false;
+};
+
+struct ScheduleEntry {
+  int32_t* dev = nullptr;  // units, then q offsets, then kv offsets
+  int n_units = 0;
+};
+
+std::map<int, DeviceState> g_devices;
+std::map<std::vector<int32_t>, ScheduleEntry> g_schedules;
+
+// Checks the current device once (sm_100 family) and resolves the status word.
+int device_state(int* device_out, DeviceState** st_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_devices[dev];
+  if (!st.checked) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+    st.supported = (prop.major == 10 && prop.minor == 0);
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+    st.status = static_cast<int*>(addr);
+    st.checked = true;
+  }
+  if (!st.supported) return MAGI_BCA_UNSUPPORTED;
+  *device_out = dev;
+  *st_out = &st;
+  return MAGI_BCA_OK;
+}
+
+std::vector<int32_t> schedule_key(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko) {
+  std::vector<int32_t> key = {dev, kind, d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim,
+                              d.n_q_chunks, d.n_kv_chunks};
+  key.insert(key.end(), qo, qo + d.n_q_chunks + 1);
+  key.insert(key.end(), ko, ko + d.n_kv_chunks + 1);
+  return key;
+}
+
+// Returns the cached device schedule, building and uploading it on first use.
+int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko,
+                 ScheduleEntry* out) {
+  std::vector<int32_t> key = schedule_key(dev, kind, d, qo, ko);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto it = g_schedules.find(key);
+  if (it != g_schedules.end()) {
+    *out = it->second;
+    return MAGI_BCA_OK;
+  }
+  std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d);
+  ScheduleEntry e;
+  e.n_units = static_cast<int>(units.size() / kUnitInts);
+  std::vector<int32_t> blob = units;
+  blob.insert(blob.end(), qo, qo + d.n_q_chunks + 1);
+  blob.insert(blob.end(), ko, ko + d.n_kv_chunks + 1);
+  if (cudaMalloc(&e.dev, blob.size() * sizeof(int32_t)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+  if (cudaMemcpy(e.dev, blob.data(), blob.size() * sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(e.dev);
+    return MAGI_BCA_CUDA_ERROR;
+  }
+  g_schedules[key] = e;
+  *out = e;
+  return MAGI_BCA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D map over a [B, S, H, D] bf16 tensor with a {64, 1, 128, 1} box and the
+// 128-byte swizzle, so one load brings 128 tokens x 64 features of one head.
+int make_map(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MAGI_BCA_CUDA_ERROR;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
+}
+
+float resolve_scale(const magi_bca_dims& d) {
+  return d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / std::sqrt((float)d.head_dim);
+}
+
+}  // namespace
+}  // namespace magi
+
+using namespace magi;
+
+extern "C" {
+
+const char* magi_bca_version(void) { return "magi_bca 0.1 (sm_100a)"; }
+
+const char* magi_bca_status_string(int status) {
+  switch (status) {
+    case MAGI_BCA_OK: return "ok";
+    case MAGI_BCA_INVALID_ARG: return "invalid argument";
+    case MAGI_BCA_UNSUPPORTED: return "unsupported configuration or device";
+    case MAGI_BCA_BAD_OFFSETS: return "bad chunk offsets";
+    case MAGI_BCA_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MAGI_BCA_CUDA_ERROR: return "CUDA runtime error";
+    case MAGI_BCA_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                              const magi_bca_dims* dims, int32_t* units, int64_t capacity) {
+  int st = validate_dims(dims);
+  if (st != MAGI_BCA_OK) return st;
+  st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, *dims);
+  if (st != MAGI_BCA_OK) return st;
+  if (capacity > 0 && units == nullptr) return MAGI_BCA_INVALID_ARG;
+  std::vector<int32_t> s = build_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, *dims);
+  const int64_t n = (int64_t)(s.size() / kUnitInts);
+  const int64_t w = n < capacity ? n : capacity;
+  if (w > 0) std::memcpy(units, s.data(), (size_t)w * kUnitInts * sizeof(int32_t));
+  return n;
+}
+
+int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                 const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets, const float* gamma_q,
+                 const float* gamma_k, magi_bca_bf16* out, float* lse, const magi_bca_dims* dims, void* stream) {
+  int st = validate_dims(dims);
+  if (st != MAGI_BCA_OK) return st;
+  const magi_bca_dims& d = *dims;
+  if (!q || !k || !v || !gamma_q || !gamma_k || !out) return MAGI_BCA_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MAGI_BCA_INVALID_ARG;
+  st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, d);
+  if (st != MAGI_BCA_OK) return st;
+  int dev;
+  DeviceState* ds;
+  st = device_state(&dev, &ds);
+  if (st != MAGI_BCA_OK) return st;
+  ScheduleEntry sched;
+  st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, &sched);
+  if (st != MAGI_BCA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&tk, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&tv, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK)
+    return MAGI_BCA_CUDA_ERROR;
+  FwdParams p;
+  p.units = sched.dev;
+  p.q_offsets = sched.dev + (size_t)sched.n_units * kUnitInts;
+  p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
+  p.n_q_chunks = d.n_q_chunks;
+  p.n_kv_chunks = d.n_kv_chunks;
+  p.gamma_q = gamma_q;
+  p.gamma_k = gamma_k;
+  p.out = out;
+  p.lse = lse;
+  p.seqlen_q = d.seqlen_q;
+  p.seqlen_kv = d.seqlen_kv;
+  p.heads_q = d.heads_q;
+  p.scale_log2 = resolve_scale(d) * 1.4426950408889634f;
+  p.eps = d.rms_eps;
+  p.status = ds->status;
+  cudaError_t e = launch_fwd(tq, tk, tv, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
+}
+
+size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims) {
+  if (validate_dims(dims) != MAGI_BCA_OK) return 0;
+  return 0;
+}
+
+int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v, const magi_bca_bf16* out,
+                 const magi_bca_bf16* dout, const float* lse, const int32_t* q_chunk_offsets,
+                 const int32_t* kv_chunk_offsets, const float* gamma_q, const float* gamma_k, magi_bca_bf16* dq,
+                 magi_bca_bf16* dk, magi_bca_bf16* dv, float* dgamma_q, float* dgamma_k, void* workspace,
+                 size_t workspace_bytes, const magi_bca_dims* dims, void* stream) {
+  (void)q; (void)k; (void)v; (void)out; (void)dout; (void)lse; (void)q_chunk_offsets; (void)kv_chunk_offsets;
+  (void)gamma_q; (void)gamma_k; (void)dq; (void)dk; (void)dv; (void)dgamma_q; (void)dgamma_k; (void)workspace;
+  (void)workspace_bytes; (void)dims; (void)stream;
+  return MAGI_BCA_UNSUPPORTED;
+}
+
+int magi_bca_last_device_status(void) {
+  int host = 0;
+  if (cudaMemcpyFromSymbol(&host, g_device_status, sizeof(int)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+  return host == 0 ? MAGI_BCA_OK : MAGI_BCA_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"

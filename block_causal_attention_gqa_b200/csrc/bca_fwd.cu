@@ -1,0 +1,442 @@
+// Forward kernel: block-causal GQA attention with fused QK-RMSNorm, sm_100a.
+//
+// One CTA runs one work unit: up to two 128-row query tiles ("sub-tiles")
+// that share a key/value head and a kv extent (bca_sched.h).  Roles:
+//   warps 0-3  softmax warpgroup for sub-tile 0 (thread i owns query row i,
+//              which is TMEM lane i)
+//   warps 4-7  softmax warpgroup for sub-tile 1
+//   warp  8    tcgen05 MMA issue (one elected thread)
+//   warp  9    TMA producer (one elected thread)
+// TMEM (512 columns): S_s at 256*s, O_s at 256*s + 128.  P_s (bf16 pairs)
+// overwrites the first 64 columns of S_s once S_s has been read.
+//
+// Per kv tile j the MMA thread issues, for each sub-tile s,
+//   O_s += P_s(j) V_j      (A from TMEM, V as an MN-major B operand)
+//   S_s  = Q_s K_{j+1}^T   (both K-major)
+// and commits s_full[s]; a commit completes only when every earlier tcgen05
+// operation of the thread has, so s_full also says "O_s is up to date".
+//
+// QK-RMSNorm fold.  With r_q = rsqrt(mean q^2 + eps), r_k likewise,
+//   scale * q~.k~ = r_q r_k sum_d (q_d gamma_q[d] gamma_k[d] scale) k_d.
+// The softmax warps scale each Q row once by r_q * gamma_q*gamma_k*scale*log2(e)
+// in shared memory (the MMA then produces logits in log2 units up to the
+// per-key factor), and apply r_k of key j as a column factor on S.  r_k is
+// computed from the K tile in shared memory while it is resident.
+//
+// Online softmax with a lazy maximum: a row's reference maximum moves only
+// when a tile's maximum exceeds it by more than 8 (log2 units), so P <= 256
+// and the O rescale (TMEM load, multiply, store) is rare after the first
+// tiles.  The result is exact: O and l are always scaled by the same factor.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "bca_kernels.h"
+#include "sm100.cuh"
+
+namespace magi {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;
+
+enum : int {
+  kErrQ = 1001, kErrKFull = 1002, kErrVFull = 1003, kErrKEmpty = 1004, kErrVEmpty = 1005,
+  kErrSFull = 1006, kErrPReady = 1007, kErrQReady = 1008, kErrKSoft = 1009
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;  // one [128][D] bf16 tile
+  static constexpr int kQ = 0;                     // 2 sub-tiles
+  static constexpr int kK = kQ + 2 * kTileBytes;   // kStages
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kRk = kV + kStages * kTileBytes;  // float [2 wg][2 buf][128]
+  static constexpr int kQScale = kRk + 2 * 2 * 128 * 4;   // float [D]
+  static constexpr int kBars = kQScale + D * 4;
+  static constexpr int kNumBars = 16;
+  static constexpr int kTmemSlot = kBars + kNumBars * 8;
+  static constexpr int kTotal = kTmemSlot + 16;
+  static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
+};
+
+struct Bars {
+  uint64_t q_full[2], q_ready[2], s_full[2], p_ready[2];
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+};
+
+// Bounded wait whose outcome every lane of the warp agrees on, so warp-wide
+// tcgen05 instructions are executed by all lanes or by none.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool ok, int* status, int code) {
+  if (ok) ok = mbar_wait(bar, parity, status, code);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
+  int lo = 0, hi = n;  // offs[lo] <= row < offs[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(offs + mid) <= row) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// Sum of squares of one [D] bf16 row stored 128B-swizzled across D/64 boxes.
+template <int D>
+__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
+  float acc = 0.f;
+#pragma unroll
+  for (int box = 0; box < D / 64; ++box) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + box * 16384 + sw128_offset(row, c * 8));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
+        acc = fmaf(lo, lo, acc);
+        acc = fmaf(hi, hi, acc);
+      }
+    }
+  }
+  return acc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  float* qscale = reinterpret_cast<float*>(smem + L::kQScale);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int32_t* u = p.units + (size_t)blockIdx.x * 8;
+  const int b = __ldg(u + 0), hk = __ldg(u + 1);
+  const int head[2] = {__ldg(u + 2), __ldg(u + 4)};
+  const int m0[2] = {__ldg(u + 3), __ldg(u + 5)};
+  const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
+  const int n_sub = head[1] >= 0 ? 2 : 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_ready[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_ready[s], 1);
+    }
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&bars->k_full[st], 1);
+      mbar_init(&bars->k_empty[st], 1 + n_sub);  // MMA commit + each softmax warpgroup's r_k pass
+      mbar_init(&bars->v_full[st], 1);
+      mbar_init(&bars->v_empty[st], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  for (int d = threadIdx.x; d < D; d += kThreads)
+    qscale[d] = __ldg(p.gamma_q + d) * __ldg(p.gamma_k + d) * p.scale_log2;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      for (int s = 0; s < n_sub; ++s) {
+        mbar_arrive_expect_tx(&bars->q_full[s], L::kTileBytes);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_4d(smem + L::kQ + s * L::kTileBytes + box * 16384, &tm_q, &bars->q_full[s], box * 64,
+                      head[s], m0[s], b);
+      }
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % kStages;
+        const uint32_t par = ((j / kStages) & 1) ^ 1;
+        if (!mbar_wait(&bars->k_empty[st], par, p.status, kErrKEmpty)) break;
+        mbar_arrive_expect_tx(&bars->k_full[st], L::kTileBytes);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_4d(smem + L::kK + st * L::kTileBytes + box * 16384, &tm_k, &bars->k_full[st], box * 64, hk,
+                      j * 128, b);
+        if (!mbar_wait(&bars->v_empty[st], par, p.status, kErrVEmpty)) break;
+        mbar_arrive_expect_tx(&bars->v_full[st], L::kTileBytes);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_4d(smem + L::kV + st * L::kTileBytes + box * 16384, &tm_v, &bars->v_full[st], box * 64, hk,
+                      j * 128, b);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, D, false, true);
+      const uint32_t q_base = smem_u32(smem + L::kQ);
+      const uint32_t k_base = smem_u32(smem + L::kK);
+      const uint32_t v_base = smem_u32(smem + L::kV);
+      bool ok = true;
+      auto issue_s = [&](int s, int st) {
+        const uint32_t qa = q_base + s * L::kTileBytes, ka = k_base + st * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + 256 * s, make_sw128_desc(qa + off, 16, 1024), make_sw128_desc(ka + off, 16, 1024),
+                      idesc_s, kk > 0);
+        }
+      };
+      for (int s = 0; s < n_sub && ok; ++s) ok = mbar_wait(&bars->q_ready[s], 0, p.status, kErrQReady);
+      ok = ok && mbar_wait(&bars->k_full[0], 0, p.status, kErrKFull);
+      if (ok) {
+        tc_fence_after();
+        for (int s = 0; s < n_sub; ++s) {
+          issue_s(s, 0);
+          mma_commit(&bars->s_full[s]);
+        }
+        mma_commit(&bars->k_empty[0]);
+      }
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, p.status, kErrVFull)) break;
+        const bool has_next = j + 1 < n_tiles;
+        const int st1 = (j + 1) % kStages;
+        for (int s = 0; s < n_sub; ++s) {
+          if (!mbar_wait(&bars->p_ready[s], j & 1, p.status, kErrPReady)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t va = v_base + st * L::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + 256 * s + 128, tmem + 256 * s + kk * 8,
+                        make_sw128_desc(va + kk * 2048, 16384, 1024), idesc_o, j > 0 || kk > 0);
+          if (has_next) {
+            if (s == 0 && !mbar_wait(&bars->k_full[st1], ((j + 1) / kStages) & 1, p.status, kErrKFull)) {
+              ok = false;
+              break;
+            }
+            issue_s(s, st1);
+          }
+          mma_commit(&bars->s_full[s]);
+        }
+        if (!ok) break;
+        mma_commit(&bars->v_empty[st]);
+        if (has_next) mma_commit(&bars->k_empty[st1]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int s = warp >> 2;           // sub-tile
+    const int r = threadIdx.x & 127;   // row within the tile == TMEM lane
+    if (s < n_sub) {
+      const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t t_s = tmem + lane_base + 256 * s;        // S_s / P_s
+      const uint32_t t_o = tmem + lane_base + 256 * s + 128;  // O_s
+      uint8_t* q_tile = smem + L::kQ + s * L::kTileBytes;
+      float* rk_buf = reinterpret_cast<float*>(smem + L::kRk) + s * 256;
+      const int bar_id = 1 + s;
+      bool ok = true;
+
+      // Q prologue: RMSNorm the row and fold gains, scale and log2(e) into it.
+      ok = warp_wait(&bars->q_full[s], 0, ok, p.status, kErrQ);
+      if (ok) {
+        const float rq = rsqrtf(row_sumsq<D>(q_tile, r) * (1.0f / D) + p.eps);
+#pragma unroll
+        for (int box = 0; box < D / 64; ++box) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4* ptr = reinterpret_cast<uint4*>(q_tile + box * 16384 + sw128_offset(r, c * 8));
+            uint4 v = *ptr;
+            uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const int d0 = box * 64 + c * 8;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float lo = __uint_as_float(w[i] << 16) * rq * qscale[d0 + 2 * i];
+              const float hi = __uint_as_float(w[i] & 0xffff0000u) * rq * qscale[d0 + 2 * i + 1];
+              w[i] = pack_bf16x2(lo, hi);
+            }
+            *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(bar_id, 128);
+      if (r == 0 && ok) mbar_arrive(&bars->q_ready[s]);
+
+      // Visible-key end of this row.
+      const int row = m0[s] + r;
+      int limit = p.seqlen_kv;
+      if (row < p.seqlen_q) {
+        const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
+        limit = __ldg(p.kv_offsets + p.n_kv_chunks - p.n_q_chunks + c + 1);
+      }
+
+      float m_ref = -INFINITY, l_sum = 0.f;
+      // Every thread runs all n_tiles iterations and reaches every named
+      // barrier even after a failed wait; only the work is skipped.
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j % kStages;
+        // r_k of this kv tile, from the resident K tile.
+        ok = warp_wait(&bars->k_full[st], (j / kStages) & 1, ok, p.status, kErrKSoft);
+        float* rk = rk_buf + (j & 1) * 128;
+        if (ok) rk[r] = rsqrtf(row_sumsq<D>(smem + L::kK + st * L::kTileBytes, r) * (1.0f / D) + p.eps);
+        named_bar_sync(bar_id, 128);
+        if (r == 0 && ok) mbar_arrive(&bars->k_empty[st]);
+
+        ok = warp_wait(&bars->s_full[s], j & 1, ok, p.status, kErrSFull);
+        if (ok) {
+        tc_fence_after();
+        float x[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(t_s + c * 32, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(raw[i]);
+        }
+        float m_tile = -INFINITY;
+        const float4* rk4 = reinterpret_cast<const float4*>(rk);
+        if (j >= n_full) {
+          const int lim = limit - j * 128;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float4 f = rk4[c];
+            x[4 * c + 0] = (4 * c + 0 < lim) ? x[4 * c + 0] * f.x : -INFINITY;
+            x[4 * c + 1] = (4 * c + 1 < lim) ? x[4 * c + 1] * f.y : -INFINITY;
+            x[4 * c + 2] = (4 * c + 2 < lim) ? x[4 * c + 2] * f.z : -INFINITY;
+            x[4 * c + 3] = (4 * c + 3 < lim) ? x[4 * c + 3] * f.w : -INFINITY;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float4 f = rk4[c];
+            x[4 * c + 0] *= f.x;
+            x[4 * c + 1] *= f.y;
+            x[4 * c + 2] *= f.z;
+            x[4 * c + 3] *= f.w;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 128; ++c) m_tile = fmaxf(m_tile, x[c]);
+        // Lazy maximum: move the reference only when P could exceed 2^8.
+        float alpha = 1.f;
+        if (m_tile > m_ref + kRescaleThreshold) {
+          alpha = fast_exp2(m_ref - m_tile);  // 0 on the first tile (m_ref = -inf)
+          m_ref = m_tile;
+          l_sum *= alpha;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // PV(j-1) is complete (s_full of tile j is committed after it).
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(t_o + c * 32, o);
+          }
+        }
+        float l_tile = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = fast_exp2(x[c * 32 + 2 * i] - m_ref);
+            const float p1 = fast_exp2(x[c * 32 + 2 * i + 1] - m_ref);
+            l_tile += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(t_s + c * 16, pk);
+        }
+        l_sum += l_tile;
+        tmem_wait_st();
+        tc_fence_before();
+        }
+        named_bar_sync(bar_id, 128);
+        if (r == 0 && ok) mbar_arrive(&bars->p_ready[s]);
+      }
+
+      // Epilogue: wait for the last PV, then O / l -> bf16, and the LSE.
+      ok = warp_wait(&bars->s_full[s], n_tiles & 1, ok, p.status, kErrSFull);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_sum;
+        const bool live = row < p.seqlen_q;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.seqlen_q + row) * p.heads_q + head[s]) * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_o + c * 32, o);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv_l, __uint_as_float(o[8 * i + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv_l, __uint_as_float(o[8 * i + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv_l, __uint_as_float(o[8 * i + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv_l, __uint_as_float(o[8 * i + 7]) * inv_l);
+              dst[c * 4 + i] = w;
+            }
+          }
+        }
+        if (live && p.lse != nullptr)
+          p.lse[((size_t)b * p.heads_q + head[s]) * p.seqlen_q + row] = (m_ref + log2f(l_sum)) * kLn2;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+template <int D>
+static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const FwdParams& p, int n_units, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  static uint64_t configured = 0;  // one bit per device ordinal that has the attribute set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !((configured >> dev) & 1u)) {
+    e = cudaFuncSetAttribute(bca_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= uint64_t(1) << dev;
+  }
+  bca_fwd_kernel<D><<<n_units, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                       int head_dim, int n_units, cudaStream_t stream) {
+  if (n_units <= 0) return cudaSuccess;
+  if (head_dim == 128) return launch_fwd_d<128>(tq, tk, tv, p, n_units, stream);
+  return launch_fwd_d<64>(tq, tk, tv, p, n_units, stream);
+}
+
+size_t fwd_smem_bytes(int head_dim) {
+  return head_dim == 128 ? FwdLayout<128>::kAlloc : FwdLayout<64>::kAlloc;
+}
+
+}  // namespace magi

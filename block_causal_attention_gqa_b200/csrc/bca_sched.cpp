@@ -1,0 +1,157 @@
+// Host-side argument checks and the chunk-aware tile scheduler (see bca_sched.h).
+#include "bca_sched.h"
+
+#include <algorithm>
+#include <cmath>
+#include <tuple>
+
+namespace magi {
+
+int validate_dims(const magi_bca_dims* dims) {
+  if (dims == nullptr) return MAGI_BCA_INVALID_ARG;
+  const magi_bca_dims& d = *dims;
+  if (d.batch <= 0 || d.seqlen_q <= 0 || d.seqlen_kv <= 0 || d.heads_q <= 0 || d.heads_kv <= 0 ||
+      d.head_dim <= 0 || d.n_q_chunks <= 0 || d.n_kv_chunks <= 0)
+    return MAGI_BCA_INVALID_ARG;
+  if (!(d.rms_eps >= 0.f) || !std::isfinite(d.rms_eps)) return MAGI_BCA_INVALID_ARG;
+  if (!(d.softmax_scale >= 0.f) || !std::isfinite(d.softmax_scale)) return MAGI_BCA_INVALID_ARG;
+  if (d.head_dim != 64 && d.head_dim != 128) return MAGI_BCA_UNSUPPORTED;
+  if (d.heads_q % d.heads_kv != 0) return MAGI_BCA_UNSUPPORTED;
+  if (d.n_q_chunks > d.n_kv_chunks) return MAGI_BCA_BAD_OFFSETS;
+  // TMA coordinates and the flattened index arithmetic are 32-bit.
+  const int64_t rows_q = (int64_t)d.batch * d.seqlen_q * d.heads_q;
+  const int64_t rows_kv = (int64_t)d.batch * d.seqlen_kv * d.heads_kv;
+  if (rows_q >= (int64_t(1) << 31) || rows_kv >= (int64_t(1) << 31)) return MAGI_BCA_UNSUPPORTED;
+  return MAGI_BCA_OK;
+}
+
+int validate_offsets(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d) {
+  if (qo == nullptr || ko == nullptr) return MAGI_BCA_INVALID_ARG;
+  if (qo[0] != 0 || ko[0] != 0) return MAGI_BCA_BAD_OFFSETS;
+  if (qo[d.n_q_chunks] != d.seqlen_q || ko[d.n_kv_chunks] != d.seqlen_kv) return MAGI_BCA_BAD_OFFSETS;
+  for (int c = 0; c < d.n_q_chunks; ++c)
+    if (qo[c + 1] <= qo[c]) return MAGI_BCA_BAD_OFFSETS;
+  for (int c = 0; c < d.n_kv_chunks; ++c)
+    if (ko[c + 1] <= ko[c]) return MAGI_BCA_BAD_OFFSETS;
+  const int shift = d.n_kv_chunks - d.n_q_chunks;
+  for (int c = 0; c < d.n_q_chunks; ++c)
+    if (qo[c + 1] - qo[c] != ko[shift + c + 1] - ko[shift + c]) return MAGI_BCA_BAD_OFFSETS;
+  return MAGI_BCA_OK;
+}
+
+int row_kv_end(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d, int row) {
+  // chunk c with qo[c] <= row < qo[c+1]
+  const int32_t* it = std::upper_bound(qo, qo + d.n_q_chunks + 1, row);
+  const int c = static_cast<int>(it - qo) - 1;
+  return ko[d.n_kv_chunks - d.n_q_chunks + c + 1];
+}
+
+QTileExtent qtile_extent(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d, int m0) {
+  const int last = std::min(m0 + kBlockM, d.seqlen_q) - 1;
+  // visible ends are non-decreasing in the row index
+  const int lo = row_kv_end(qo, ko, d, m0);
+  const int hi = row_kv_end(qo, ko, d, last);
+  QTileExtent e;
+  e.n_full = lo / kBlockN;
+  e.n_tiles = (hi + kBlockN - 1) / kBlockN;
+  return e;
+}
+
+std::vector<int32_t> build_fwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d) {
+  const int n_qt = (d.seqlen_q + kBlockM - 1) / kBlockM;
+  const int group = d.heads_q / d.heads_kv;
+  std::vector<QTileExtent> ext(n_qt);
+  for (int t = 0; t < n_qt; ++t) ext[t] = qtile_extent(qo, ko, d, t * kBlockM);
+
+  struct Unit {
+    int b, hk, h0, m00, h1, m01, n_full, n_tiles, first_tile;
+  };
+  std::vector<Unit> units;
+  units.reserve((size_t)d.batch * d.heads_kv * n_qt * ((group + 1) / 2));
+  for (int b = 0; b < d.batch; ++b) {
+    for (int hk = 0; hk < d.heads_kv; ++hk) {
+      // Walk the (tile, head) sub-tiles of this kv head in tile-major order
+      // and pair neighbours that share an extent.
+      int pend_h = -1, pend_t = -1;
+      for (int t = 0; t < n_qt; ++t) {
+        for (int h = hk * group; h < (hk + 1) * group; ++h) {
+          if (pend_h >= 0 && ext[pend_t].n_full == ext[t].n_full && ext[pend_t].n_tiles == ext[t].n_tiles) {
+            units.push_back({b, hk, pend_h, pend_t * kBlockM, h, t * kBlockM, ext[t].n_full,
+                             ext[t].n_tiles, pend_t});
+            pend_h = -1;
+            pend_t = -1;
+          } else {
+            if (pend_h >= 0)
+              units.push_back({b, hk, pend_h, pend_t * kBlockM, -1, 0, ext[pend_t].n_full,
+                               ext[pend_t].n_tiles, pend_t});
+            pend_h = h;
+            pend_t = t;
+          }
+        }
+      }
+      if (pend_h >= 0)
+        units.push_back({b, hk, pend_h, pend_t * kBlockM, -1, 0, ext[pend_t].n_full,
+                         ext[pend_t].n_tiles, pend_t});
+    }
+  }
+  // Longest first (list scheduling in launch order approximates LPT); among
+  // equal costs keep one (batch, kv head) together so the CTAs that run at
+  // the same time stream the same K/V through L2.
+  std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
+    const int ca = a.n_tiles * (a.h1 >= 0 ? 2 : 1), cb = b.n_tiles * (b.h1 >= 0 ? 2 : 1);
+    if (ca != cb) return ca > cb;
+    return std::tie(a.b, a.hk, a.first_tile, a.h0) < std::tie(b.b, b.hk, b.first_tile, b.h0);
+  });
+  std::vector<int32_t> out;
+  out.reserve(units.size() * kUnitInts);
+  for (const Unit& u : units) {
+    const int32_t v[kUnitInts] = {u.b, u.hk, u.h0, u.m00, u.h1, u.m01, u.n_full, u.n_tiles};
+    out.insert(out.end(), v, v + kUnitInts);
+  }
+  return out;
+}
+
+std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d) {
+  const int n_qt = (d.seqlen_q + kBlockM - 1) / kBlockM;
+  const int n_kt = (d.seqlen_kv + kBlockN - 1) / kBlockN;
+  std::vector<int> tile_lo(n_qt);  // smallest visible end among the tile's rows
+  for (int t = 0; t < n_qt; ++t) tile_lo[t] = row_kv_end(qo, ko, d, t * kBlockM);
+  struct Unit {
+    int b, hk, n0, qb, qe, nd;
+  };
+  std::vector<Unit> units;
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int n0 = kt * kBlockN;
+    const int n_end = std::min(n0 + kBlockN, d.seqlen_kv);
+    // first query row whose visible end exceeds n0
+    int qrow = d.seqlen_q;
+    {
+      int lo = 0, hi = d.seqlen_q;  // binary search on the non-decreasing row ends
+      while (lo < hi) {
+        const int mid = (lo + hi) / 2;
+        if (row_kv_end(qo, ko, d, mid) > n0) hi = mid; else lo = mid + 1;
+      }
+      qrow = lo;
+    }
+    if (qrow >= d.seqlen_q) continue;  // nobody sees this kv tile
+    const int qb = qrow / kBlockM;
+    int nd = 0;
+    for (int t = qb; t < n_qt && tile_lo[t] < n_end; ++t) ++nd;
+    for (int b = 0; b < d.batch; ++b)
+      for (int hk = 0; hk < d.heads_kv; ++hk) units.push_back({b, hk, n0, qb, n_qt, nd});
+  }
+  std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
+    const int ca = a.qe - a.qb, cb = b.qe - b.qb;
+    if (ca != cb) return ca > cb;
+    return std::tie(a.b, a.hk, a.n0) < std::tie(b.b, b.hk, b.n0);
+  });
+  std::vector<int32_t> out;
+  out.reserve(units.size() * kUnitInts);
+  for (const Unit& u : units) {
+    const int32_t v[kUnitInts] = {u.b, u.hk, u.n0, u.qb, u.qe, u.nd, 0, 0};
+    out.insert(out.end(), v, v + kUnitInts);
+  }
+  return out;
+}
+
+}  // namespace magi

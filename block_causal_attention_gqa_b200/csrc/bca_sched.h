@@ -1,0 +1,56 @@
+// Host-side argument checks and the chunk-aware tile scheduler.
+//
+// Block-causal attention (MAGI-1 §2, Figure 1) lets query chunk c see every
+// key of kv chunks 0 .. n_kv - n_q + c.  Over 128 x 128 tiles this means:
+//   * a query tile whose rows all sit in chunks whose visible range ends at
+//     or after column tile j's end needs tile j with no mask ("full" tile);
+//   * tiles between the smallest and the largest visible end of the tile's
+//     rows straddle a chunk boundary and need the per-row mask ("diagonal");
+//   * tiles past the largest end are never visited.
+// Because the visible range always starts at key 0, the full tiles of a
+// query tile are the prefix [0, n_full) and the diagonal ones
+// [n_full, n_tiles).
+#pragma once
+#include <cstdint>
+#include <vector>
+
+#include "../../include/magi_bca.h"
+
+namespace magi {
+
+constexpr int kBlockM = 128;  // query rows per sub-tile (one TMEM lane per row)
+constexpr int kBlockN = 128;  // kv rows per tile
+constexpr int kUnitInts = 8;  // int32 values per work unit
+
+// Checks dims and offsets.  Returns MAGI_BCA_OK or a negative status.
+int validate_dims(const magi_bca_dims* dims);
+int validate_offsets(const int32_t* q_offsets, const int32_t* kv_offsets, const magi_bca_dims& d);
+
+struct QTileExtent {
+  int n_full;   // kv tiles [0, n_full) need no mask for any row of the tile
+  int n_tiles;  // kv tiles [0, n_tiles) are visited
+};
+
+// Visible-key end for query row `row` (row < seqlen_q).
+int row_kv_end(const int32_t* q_offsets, const int32_t* kv_offsets, const magi_bca_dims& d, int row);
+
+// Extent of the query tile starting at row m0.
+QTileExtent qtile_extent(const int32_t* q_offsets, const int32_t* kv_offsets, const magi_bca_dims& d,
+                         int m0);
+
+// Forward schedule: units of up to two sub-tiles with the same (batch,
+// kv head, extent), sorted longest first and, among equals, grouped by
+// (batch, kv head) so concurrently running units share K/V in L2.
+std::vector<int32_t> build_fwd_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
+                                        const magi_bca_dims& d);
+
+// Backward schedule, kv-tile major: for kv tile t (rows [t*128, t*128+128))
+// the query tiles that see any of its keys are the q tiles [q_begin, n_qt):
+// since visibility only grows with the chunk index, every query row at or
+// after the first row whose visible end exceeds t*128 sees some key of it.
+// Emits per unit {batch, kv_head, n0, q_tile_begin, q_tile_end, n_diag_q_tiles, 0, 0}
+// where the first n_diag_q_tiles q tiles of the range need the mask.
+std::vector<int32_t> build_bwd_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
+                                        const magi_bca_dims& d);
+
+}  // namespace magi

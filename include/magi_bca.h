@@ -1,0 +1,145 @@
+/*
+ * magi_bca — block-causal grouped-query attention with QK-RMSNorm for
+ * NVIDIA B200 (sm_100a).  Plain C ABI: device pointers, host arrays, sizes.
+ *
+ * The operation (MAGI-1: Autoregressive Video Generation at Scale):
+ *   - A latent video is a sequence of fixed-length chunks.  A query token
+ *     attends to every token of its own chunk (bidirectional) and of every
+ *     earlier chunk, and never to a later chunk ("block-causal attention",
+ *     MAGI-1 §2 and Figure 1; notes page §2 and Figure 1).
+ *   - Query and key heads are normalised per head before the dot product
+ *     ("QK normalization", MAGI-1 §2.2.2); the norm is RMSNorm with a
+ *     learnable gain gamma of length head_dim:
+ *         x~ = x / sqrt(mean_d x^2 + eps) * gamma.
+ *   - Grouped-query attention (MAGI-1 §2.2.2; notes §3.2.2 model table):
+ *     query head h reads key/value head h / (heads_q / heads_kv).
+ *   - O = softmax(softmax_scale * q~ k~^T + mask) v, and
+ *     lse = ln sum_j exp(softmax_scale * q~_i . k~_j) over unmasked j.
+ *   - Streaming inference (MAGI-1 §2: up to four chunks denoised at once;
+ *     §2.4.4: KV cache of clean chunks): the query sequence holds the LAST
+ *     n_q_chunks chunks of the key/value sequence, so query chunk c is
+ *     key/value chunk n_kv_chunks - n_q_chunks + c.  With n_q == n_kv this
+ *     is the training layout.
+ *   - Backward: FLOP convention of MAGI-1 App. B.2.1 (the backward
+ *     recomputes attention; 2.5x the forward).
+ *
+ * Layouts (all contiguous, row-major):
+ *   q, out, dout, dq : [batch, seqlen_q,  heads_q,  head_dim]  bf16
+ *   k, v, dk, dv     : [batch, seqlen_kv, heads_kv, head_dim]  bf16
+ *   lse              : [batch, heads_q, seqlen_q]              fp32 (natural log)
+ *   gamma_q, gamma_k : [head_dim]                              fp32 (shared by all heads)
+ *   dgamma_q/_k      : [head_dim]                              fp32
+ *   *_chunk_offsets  : host int32 [n_chunks + 1], offsets[0] = 0, strictly
+ *                      increasing, offsets[n] = seqlen; the same chunking
+ *                      applies to every batch element.  Matched chunks
+ *                      (query chunk c and kv chunk n_kv - n_q + c) must have
+ *                      equal lengths.
+ *
+ * Ownership: every tensor pointer is caller-owned device memory; the chunk
+ * offsets are host memory read during the call.  The library keeps one
+ * schedule cache (per device and shape; mutex-guarded) and allocates device
+ * memory only when a new shape is first seen, so the first call for a shape
+ * must come before any CUDA-graph capture of later calls.
+ *
+ * Errors: every entry point returns MAGI_BCA_OK (0) or a negative status.
+ * No exception crosses the ABI and no call synchronises the host with the
+ * device.  Faults that happen on the device surface on the stream; a device
+ * wait that times out is reported by magi_bca_last_device_status().
+ *
+ * Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ * work of a call is enqueued on it.
+ */
+#ifndef MAGI_BCA_H_
+#define MAGI_BCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t magi_bca_bf16; /* raw bfloat16 bits */
+
+enum {
+  MAGI_BCA_OK = 0,
+  MAGI_BCA_INVALID_ARG = -1,        /* null pointer, non-positive size, bad dims struct */
+  MAGI_BCA_UNSUPPORTED = -2,        /* head_dim not 64/128, heads_q % heads_kv != 0, device not sm_100 */
+  MAGI_BCA_BAD_OFFSETS = -3,        /* chunk offsets violate the rules above */
+  MAGI_BCA_WORKSPACE_TOO_SMALL = -4,
+  MAGI_BCA_CUDA_ERROR = -5,         /* a CUDA runtime call failed (launch, copy, ...) */
+  MAGI_BCA_DEVICE_TIMEOUT = -6      /* a bounded device-side wait gave up */
+};
+
+typedef struct {
+  int32_t batch;
+  int32_t seqlen_q;     /* total query tokens per batch element */
+  int32_t seqlen_kv;    /* total key/value tokens per batch element */
+  int32_t heads_q;
+  int32_t heads_kv;     /* heads_q % heads_kv == 0 */
+  int32_t head_dim;     /* 64 or 128 */
+  int32_t n_q_chunks;   /* 1 <= n_q_chunks <= n_kv_chunks */
+  int32_t n_kv_chunks;
+  float softmax_scale;  /* 0 selects 1/sqrt(head_dim) */
+  float rms_eps;        /* RMSNorm epsilon; must be >= 0 (1e-6 is the usual value) */
+} magi_bca_dims;
+
+/* Forward.  Writes out (bf16) and lse (fp32; may be NULL when the caller
+ * does not need it, e.g. inference).  The call is asynchronous on `stream`. */
+int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                 const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                 const float* gamma_q, const float* gamma_k,
+                 magi_bca_bf16* out, float* lse,
+                 const magi_bca_dims* dims, void* stream);
+
+/* Bytes of device workspace magi_bca_bwd needs for `dims` (0 on invalid dims). */
+size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims);
+
+/* Backward of the training layout (any layout the forward accepts works).
+ * Inputs: q, k, v, the forward's out and lse, and dout.  Outputs: dq, dk (the
+ * gradients with respect to the RAW, un-normalised q and k, because the
+ * RMSNorm is part of the operation), dv, and optionally dgamma_q / dgamma_k
+ * (NULL to skip).  `workspace` is caller-owned device memory of at least
+ * magi_bca_bwd_workspace_size(dims) bytes, 256-byte aligned; its contents on
+ * entry do not matter. */
+int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                 const magi_bca_bf16* out, const magi_bca_bf16* dout, const float* lse,
+                 const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                 const float* gamma_q, const float* gamma_k,
+                 magi_bca_bf16* dq, magi_bca_bf16* dk, magi_bca_bf16* dv,
+                 float* dgamma_q, float* dgamma_k,
+                 void* workspace, size_t workspace_bytes,
+                 const magi_bca_dims* dims, void* stream);
+
+/* Static text for a status code. */
+const char* magi_bca_status_string(int status);
+
+/* Reads (and clears) the device status word that bounded waits write when
+ * they give up.  Synchronises with the device; returns MAGI_BCA_OK or
+ * MAGI_BCA_DEVICE_TIMEOUT (or MAGI_BCA_CUDA_ERROR if the read itself fails).
+ * Meant for tests and diagnostics, not for the hot path. */
+int magi_bca_last_device_status(void);
+
+/* Host-only view of the tile schedule the kernels run (no device needed).
+ * A work unit is up to two 128-row query tiles ("sub-tiles") that read the
+ * same key/value head and visit the same kv tiles, so every K/V tile the
+ * unit loads into shared memory serves both.  For every unit the scheduler
+ * emits 8 int32 values:
+ *   {batch, kv_head, head_0, m0_0, head_1, m0_1, n_full, n_tiles}
+ * where (head_s, m0_s) is sub-tile s's query head and first query row
+ * (head_1 = -1 when the unit has one sub-tile), n_tiles is the number of
+ * 128-token kv tiles visited and n_full how many of them (from tile 0) need
+ * no mask.  Units are listed in launch order: longest first.
+ * Returns the number of units (even if larger than `capacity`, in which case
+ * only `capacity` units are written), or a negative status. */
+int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                              const magi_bca_dims* dims, int32_t* units, int64_t capacity);
+
+/* Library version string. */
+const char* magi_bca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAGI_BCA_H_ */

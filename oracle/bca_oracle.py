@@ -113,6 +113,11 @@ def block_causal_mask(q_offsets, kv_offsets, rows=None):
     return ck[None, :] <= matched_kv_chunk(cq, nq, nkv)[:, None]
 
 
+def torch_index(rows):
+    import torch
+    return torch.as_tensor(np.asarray(rows, dtype=np.int64))
+
+
 def _check(q, k, v, q_offsets, kv_offsets):
     B, Sq, Hq, D = q.shape
     Bk, Skv, Hkv, Dk = k.shape
@@ -127,33 +132,38 @@ def _check(q, k, v, q_offsets, kv_offsets):
 def _attend_rows(qn_rows, kn, vv, mask_rows, scale):
     """Softmax attention of a block of normalised query rows [R, D] against
     all normalised keys [S, D]; returns (O [R, D], lse [R], P [R, S])."""
-    s = scale * (qn_rows @ kn.T)
-    s = np.where(mask_rows, s, -np.inf)
+    s = qn_rows @ kn.T
+    s *= scale
+    s[~mask_rows] = -np.inf
     m = np.max(s, axis=1, keepdims=True)
-    p = np.exp(s - m)
+    s -= m
+    p = np.exp(s, out=s)
     l = np.sum(p, axis=1, keepdims=True)
-    p = p / l
+    p /= l
     return p @ vv, (m + np.log(l))[:, 0], p
 
 
 def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=None,
-                 batches=None, scale=None, eps=DEFAULT_EPS, block=512):
+                 batches=None, scale=None, eps=DEFAULT_EPS, block=None):
     """Forward on a subset of query rows.
 
     ``rows`` is an int array of query-token indices; ``heads`` / ``batches``
     restrict the query heads and batch elements (default all).  Returns
     (out [nb, R, nh, D], lse [nb, nh, R]) in float64 for those rows only."""
-    q = _f64(q)
+    rows = np.asarray(rows, dtype=np.int64)
     k = _f64(k)
     v = _f64(v)
     q_offsets = np.asarray(q_offsets)
     kv_offsets = np.asarray(kv_offsets)
     B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
+    # only the requested query rows are converted (row i of qsel is rows[i])
+    qsel = _f64(q[:, rows]) if not hasattr(q, "detach") else _f64(q[:, torch_index(rows)])
     scale = 1.0 / np.sqrt(D) if not scale else float(scale)
-    rows = np.asarray(rows, dtype=np.int64)
     heads = list(range(Hq)) if heads is None else list(heads)
     batches = list(range(B)) if batches is None else list(batches)
     group = Hq // Hkv
+    if block is None:   # rows per step, so one logit block stays near 512 MB
+        block = int(max(16, min(512, (1 << 26) // Skv)))
     out = np.zeros((len(batches), len(rows), len(heads), D))
     lse = np.zeros((len(batches), len(heads), len(rows)))
     for bi, b in enumerate(batches):
@@ -164,7 +174,7 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
             vv = v[b, :, hk, :]
             for r0 in range(0, len(rows), block):
                 rr = rows[r0:r0 + block]
-                qn = rms_norm(q[b, rr, h, :], gamma_q, eps)
+                qn = rms_norm(qsel[b, r0:r0 + block, h, :], gamma_q, eps)
                 mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
                 o, ls, _ = _attend_rows(qn, kn, vv, mask, scale)
                 out[bi, r0:r0 + len(rr), hi, :] = o

@@ -1,0 +1,30 @@
+"""Shared helpers for the parity tests: tolerance checks and case builders."""
+import numpy as np
+import torch
+
+# Tolerances for bf16 inputs with fp32 accumulation against the fp64 oracle.
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+
+
+def rel_l2(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+
+
+def assert_close(name, got, want, max_abs=MAX_ABS, rel=REL_L2):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, f"{name}: shape {got.shape} vs {want.shape}"
+    assert np.isfinite(got).all(), f"{name}: non-finite values"
+    err = float(np.max(np.abs(got - want))) if got.size else 0.0
+    r = rel_l2(got, want)
+    assert err <= max_abs and r <= rel, f"{name}: max abs {err:.3e} (<= {max_abs}), rel L2 {r:.3e} (<= {rel})"
+    return err, r
+
+
+def to_np(t):
+    if t.dtype == torch.bfloat16:
+        t = t.float()
+    return t.detach().cpu().numpy().astype(np.float64)

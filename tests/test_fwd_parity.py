@@ -1,0 +1,103 @@
+"""GPU parity of the forward against the fp64 oracle (through the C ABI).
+
+Small workloads are compared on every row; the model-scale, streaming and
+long-context workloads at full size (the launch bench.py times) on 4096
+stratified query rows per head.  Tolerance: max abs 1e-2 and relative L2
+5e-3 for bf16 inputs with fp32 accumulation."""
+import numpy as np
+import pytest
+import torch
+
+import block_causal_attention_gqa_b200 as bca
+import workloads
+from oracle import bca_oracle as orc
+from tests._helpers import assert_close, to_np, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(inp, w, lse=True):
+    dev = "cuda"
+    q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
+    out, l = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, inp["gamma_q"].to(dev),
+                              inp["gamma_k"].to(dev), want_lse=lse)
+    torch.cuda.synchronize()
+    assert bca.magi_bca_last_device_status() == 0
+    return out, l
+
+
+SMALL = {
+    "tiny": workloads.workload("tiny"),
+    "train4k": workloads.workload("train4k"),
+    "ragged_d128": workloads.custom("ragged_d128", 2, [100, 333, 1000, 67], None, 4, 2, 128, seed=11),
+    "ragged_d64_gqa3": workloads.custom("ragged_d64_gqa3", 1, [70, 130, 200], None, 6, 2, 64, seed=12),
+    "stream_small": workloads.custom("stream_small", 2, [150, 250], [300, 200, 150, 250], 8, 2, 128, seed=13),
+    "single_chunk_mha": workloads.custom("single_chunk_mha", 1, [777], None, 2, 2, 128, seed=14),
+    "token_causal": workloads.custom("token_causal", 1, [1] * 37, None, 2, 1, 64, seed=15),
+    "many_chunks": workloads.custom("many_chunks", 1, [50] * 20, None, 4, 1, 128, seed=16),
+    "gqa8_long_rows": workloads.custom("gqa8_long_rows", 1, [640] * 3, None, 16, 2, 128, seed=17,
+                                       token_scale=True),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_all_rows(name):
+    w = SMALL[name]
+    inp = workloads.make_inputs(w, with_grad_out=False)
+    out, lse = run_gpu(inp, w)
+    o_ref, l_ref = orc.forward(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
+                               inp["gamma_q"], inp["gamma_k"])
+    assert_close(f"{name} out", to_np(out), o_ref)
+    assert_close(f"{name} lse", to_np(lse), l_ref)
+    if "q_f32" in inp:
+        # information only: error against the unrounded fp32 inputs
+        o32, _ = orc.forward(inp["q_f32"], inp["k_f32"], inp["v_f32"], w.q_offsets, w.kv_offsets,
+                             inp["gamma_q"], inp["gamma_k"])
+        print(f"{name}: rel L2 vs unrounded fp32 inputs {rel_l2(to_np(out), o32):.3e}")
+
+
+def test_forward_without_lse_and_canary():
+    w = SMALL["ragged_d128"]
+    inp = workloads.make_inputs(w, with_grad_out=False)
+    dev = "cuda"
+    q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
+    n = q.numel()
+    big = torch.full((n + 4096,), 7.0, device=dev, dtype=torch.bfloat16)
+    out = big[:n].view(q.shape)
+    bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, inp["gamma_q"].to(dev), inp["gamma_k"].to(dev),
+                     out=out, want_lse=False)
+    torch.cuda.synchronize()
+    assert (big[n:] == 7.0).all(), "write past the end of out"
+    o_ref, _ = orc.forward(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
+                           inp["gamma_q"], inp["gamma_k"])
+    assert_close("no-lse out", to_np(out), o_ref)
+
+
+def test_forward_is_deterministic():
+    w = SMALL["train4k"]
+    inp = workloads.make_inputs(w, with_grad_out=False)
+    o1, l1 = run_gpu(inp, w)
+    o2, l2 = run_gpu(inp, w)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+LARGE = ["model46k", "stream4of16", "long262k"]
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_forward_full_size_sampled_rows(name):
+    w = workloads.workload(name)
+    inp = workloads.make_inputs(w, with_grad_out=False)
+    out, lse = run_gpu(inp, w)
+    out_c, lse_c = out.cpu(), lse.cpu()
+    del out, lse
+    torch.cuda.empty_cache()
+    # 4096 rows per head, spread over the batch elements
+    per_batch = 4096 // w.batch
+    for b in range(w.batch):
+        rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, per_batch, seed=100 + b)
+        o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
+                                        inp["gamma_q"], inp["gamma_k"], rows, batches=[b])
+        idx = torch.as_tensor(rows)
+        assert_close(f"{name} out b{b}", to_np(out_c[b:b + 1, idx]), o_ref)
+        assert_close(f"{name} lse b{b}", to_np(lse_c[b:b + 1][:, :, idx]), l_ref)

@@ -1,0 +1,465 @@
+#!/usr/bin/env python3
+"""Benchmark: useful TFLOP/s of block-causal GQA attention with QK-RMSNorm on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--pass fwd|fwdbwd]
+                    [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+the forward (and, for training workloads, the backward) of the workload.
+Useful FLOPs count unmasked (query, key) pairs only: forward = 4*D*B*Hq*pairs
+(two matmuls over the mask area), backward = 2.5x forward (MAGI-1 App. B.2.1,
+the Flash-Attention convention).  Multi-GPU runs are independent replicas
+(the path has no exchange step): value = all ranks' FLOPs / max-over-ranks time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference there is)
+on a bounded sample of the same workload, on the host cores, rank 0 only.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+DATASHEET_BF16_TFLOPS = 2250.0   # NVIDIA HGX B200 dense bf16, for context only
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ work model
+def row_kv_ends(w):
+    """Visible-key end of every query row (query chunk c = kv chunk n_kv - n_q + c)."""
+    qo, ko = w.q_offsets, w.kv_offsets
+    nq, nkv = len(qo) - 1, len(ko) - 1
+    ends = np.empty(w.seqlen_q, np.int64)
+    for c in range(nq):
+        ends[qo[c]:qo[c + 1]] = ko[nkv - nq + c + 1]
+    return ends
+
+
+def fwd_flops(w):
+    return 4.0 * w.head_dim * w.batch * w.heads_q * float(row_kv_ends(w).sum())
+
+
+def bwd_flops(w):
+    return 2.5 * fwd_flops(w)
+
+
+def fwd_bytes(w):
+    """Algorithmic HBM bytes of the forward: read q, k, v once, write out and lse."""
+    q = w.batch * w.seqlen_q * w.heads_q * w.head_dim * 2
+    kv = 2 * w.batch * w.seqlen_kv * w.heads_kv * w.head_dim * 2
+    return q + kv + q + w.batch * w.heads_q * w.seqlen_q * 4
+
+
+# ------------------------------------------------------------------ peaks, clocks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def _query_once(self):
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                  "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+            return [l for l in out.stdout.splitlines() if l.strip()]
+        except Exception:
+            return []
+
+    def start(self):
+        self.lines += self._query_once()
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+                self.lines += [l for l in out.splitlines() if l.strip()]
+            except Exception:
+                self.proc.kill()
+        self.lines += self._query_once()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("bca_fwd.cu", "bca_bwd.cu", "sm100.cuh", "bca_kernels.h"):
+        p = os.path.join(ROOT, "block_causal_attention_gqa_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(kernel, {}).get(workload_name)
+        if e and e.get("kernel_source_sha") == kernel_source_sha():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, w, world, rank, local):
+    import block_causal_attention_gqa_b200 as bca
+    dev = torch.device("cuda", local)
+    do_bwd = args.pass_ == "fwdbwd"
+    inp = workloads.make_inputs(w, device=str(dev), with_grad_out=do_bwd)
+    q, k, v, gq, gk = inp["q"], inp["k"], inp["v"], inp["gamma_q"], inp["gamma_k"]
+    out = torch.empty_like(q)
+    lse = torch.empty(w.batch, w.heads_q, w.seqlen_q, device=dev, dtype=torch.float32)
+    if do_bwd:
+        dout = inp["dout"]
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dgq = torch.empty(w.head_dim, device=dev)
+        dgk = torch.empty(w.head_dim, device=dev)
+        dims = bca.make_dims(w.batch, w.seqlen_q, w.seqlen_kv, w.heads_q, w.heads_kv, w.head_dim,
+                             len(w.q_chunks), len(w.kv_chunks))
+        ws = torch.empty(max(bca.magi_bca_bwd_workspace_size(dims), 1), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    l2_flush = torch.empty(512 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, out=out, lse=lse, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if do_bwd:
+            bca.magi_bca_bwd(q, k, v, out, inp["dout"], lse, w.q_offsets, w.kv_offsets, gq, gk, dq=dq, dk=dk,
+                             dv=dv, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        l2_flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    n_ev = 3 if do_bwd else 2
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid else local)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        l2_flush.zero_()           # inputs of small workloads fit in L2: flush between steps
+        step(evs[i])
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall0
+    sampler.stop()
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs] if do_bwd else [0.0] * len(evs)
+    step_ms_total = sum(f + b for f, b in zip(fwd_ms, bwd_ms))
+    step_ms_total = max_over_ranks(step_ms_total, world)
+    st = bca.magi_bca_last_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the timed region")
+
+    # e2e: through the public API with host buffers (pinned), copies in the timed region
+    hq = inp["q"].cpu().pin_memory()
+    hk = inp["k"].cpu().pin_memory()
+    hv = inp["v"].cpu().pin_memory()
+    hdo = inp["dout"].cpu().pin_memory() if do_bwd else None
+    h_out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    if do_bwd:
+        h_dq = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        h_dk = torch.empty(k.shape, dtype=k.dtype).pin_memory()
+        h_dv = torch.empty(v.shape, dtype=v.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        if do_bwd:
+            inp["dout"].copy_(hdo, non_blocking=True)
+        step()
+        if do_bwd:
+            h_dq.copy_(dq, non_blocking=True)
+            h_dk.copy_(dk, non_blocking=True)
+            h_dv.copy_(dv, non_blocking=True)
+        else:
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = (q.numel() + k.numel() + v.numel() + (q.numel() if do_bwd else 0)) * 2
+    d2h = (q.numel() + 2 * k.numel()) * 2 if do_bwd else q.numel() * 2 + lse.numel() * 4
+
+    flops_step = fwd_flops(w) + (bwd_flops(w) if do_bwd else 0.0)
+    value = world * flops_step * args.steps / (step_ms_total * 1e-3) / 1e12
+    e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    # dominant kernel: the one with the larger share of the step time
+    fwd_avg = float(np.mean(fwd_ms))
+    bwd_avg = float(np.mean(bwd_ms)) if do_bwd else 0.0
+    if do_bwd and bwd_avg > fwd_avg:
+        dom, dom_flops, dom_ms = "bca_bwd", bwd_flops(w), bwd_avg
+    else:
+        dom, dom_flops, dom_ms = "bca_fwd_kernel", fwd_flops(w), fwd_avg
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed alone)", "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
+                "traffic": ncu_traffic(dom, w.name), "avg_launch_ms": round(dom_ms, 4),
+                "algorithmic_bytes_per_launch": fwd_bytes(w) if dom == "bca_fwd_kernel" else None}
+    launches_per_step = 1 + (bca_bwd_launches() if do_bwd else 0)
+    clocks = sampler.summary()
+    res = {
+        "metric": "block-causal attention useful TFLOP/s on 1 B200 and % of dense BF16 peak",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms_total / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, gamma 1+N(0,0.1))",
+        "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
+                   "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
+                   "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (512 MB write) between timed steps, outside the step events",
+                   "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4) if do_bwd else None,
+                   "useful_tflop_per_step": round(flops_step / 1e12, 4)},
+        "pct_of_measured_peak": round(100 * value / world / peak, 2),
+        "pct_of_datasheet_peak": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "roofline": roofline,
+        "clocks": clocks,
+        "wall_s_timed_region": round(t_wall, 3),
+    }
+    return res
+
+
+def bca_bwd_launches():
+    return 3
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+def oracle_sample(w, inp, rows, do_bwd):
+    """Runs the oracle on the given query rows (all heads, batch 0)."""
+    from oracle import bca_oracle as orc
+    orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
+                     inp["gamma_k"], rows, batches=[0])
+    if do_bwd:
+        orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
+                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0])
+
+
+def sample_flops(w, rows, do_bwd):
+    ends = row_kv_ends(w)[rows]
+    f = 4.0 * w.head_dim * w.heads_q * float(ends.sum())
+    return f * (1 + (2.5 if do_bwd else 0.0))
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def time_oracle(w, do_bwd, budget_s):
+    """Times the oracle on growing blocks of rows (evenly spread over the
+    query sequence) until ~budget_s of CPU work; returns (TFLOP/s, rows, s)."""
+    inp = workloads.make_inputs(w, with_grad_out=do_bwd)
+    rng = np.random.default_rng(0)
+    n = 16
+    done_rows, done_t, done_f = 0, 0.0, 0.0
+    while done_t < budget_s:
+        rows = np.sort(rng.choice(w.seqlen_q, size=min(n, w.seqlen_q), replace=False))
+        t0 = time.perf_counter()
+        oracle_sample(w, inp, rows, do_bwd)
+        dt = time.perf_counter() - t0
+        done_rows += len(rows)
+        done_t += dt
+        done_f += sample_flops(w, rows, do_bwd)
+        if dt < budget_s / 8:
+            n *= 2
+    return done_f / done_t / 1e12, done_rows, done_t
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return None
+    do_bwd = args.pass_ == "fwdbwd"
+    per_step = max(0.05, 90.0 / max(1, args.steps + args.warmup))
+    inp = workloads.make_inputs(w, with_grad_out=do_bwd)
+    rows_per_step = 8
+    # calibrate the sample size to the per-step budget
+    t0 = time.perf_counter()
+    oracle_sample(w, inp, np.arange(rows_per_step), do_bwd)
+    dt = time.perf_counter() - t0
+    rows_per_step = int(max(1, min(w.seqlen_q, rows_per_step * per_step / max(dt, 1e-6))))
+    rng = np.random.default_rng(1)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, np.sort(rng.choice(w.seqlen_q, rows_per_step, replace=False)), do_bwd)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        rows = np.sort(rng.choice(w.seqlen_q, rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        oracle_sample(w, inp, rows, do_bwd)
+        tot_t += time.perf_counter() - t0
+        tot_f += sample_flops(w, rows, do_bwd)
+    value = tot_f / tot_t / 1e12
+    sample = (f"{rows_per_step} random query rows x all {w.heads_q} heads of batch 0 per step "
+              f"({'fwd+bwd' if do_bwd else 'fwd'}), fp64 NumPy")
+    return {
+        "impl": "reference",
+        "metric": "block-causal attention useful TFLOP/s on 1 B200 and % of dense BF16 peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
+                   "seqlen_kv": w.seqlen_kv, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+                   "head_dim": w.head_dim},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="train4k", help="workload name (see workloads.WORKLOADS)")
+    ap.add_argument("--pass", dest="pass_", default=None, choices=["fwd", "fwdbwd"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = workloads.workload(args.config)
+    if args.pass_ is None:
+        args.pass_ = "fwdbwd" if (w.backward and BWD_AVAILABLE) else "fwd"
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, w, world, rank)
+        else:
+            res = run_ours(args, w, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                tf, nrows, secs = time_oracle(w, args.pass_ == "fwdbwd", budget_s=12.0)
+                res["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                       "sample": f"{nrows} random query rows x all {w.heads_q} heads of batch 0 "
+                                                 f"({args.pass_}), fp64 NumPy, {secs:.1f} s"}
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+BWD_AVAILABLE = False
+
+if __name__ == "__main__":
+    main()

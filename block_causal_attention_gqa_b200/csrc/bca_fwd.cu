@@ -40,7 +40,6 @@ using namespace sm100;
 
 constexpr int kThreads = 320;
 constexpr int kStages = 2;
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;
 

@@ -211,7 +211,8 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
 
 size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims) {
   if (validate_dims(dims) != MAGI_BCA_OK) return 0;
-  return 0;
+  const magi_bca_dims& d = *dims;
+  return bwd_workspace_layout(d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim).total;
 }
 
 int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v, const magi_bca_bf16* out,
@@ -219,10 +220,65 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
                  const int32_t* kv_chunk_offsets, const float* gamma_q, const float* gamma_k, magi_bca_bf16* dq,
                  magi_bca_bf16* dk, magi_bca_bf16* dv, float* dgamma_q, float* dgamma_k, void* workspace,
                  size_t workspace_bytes, const magi_bca_dims* dims, void* stream) {
-  (void)q; (void)k; (void)v; (void)out; (void)dout; (void)lse; (void)q_chunk_offsets; (void)kv_chunk_offsets;
-  (void)gamma_q; (void)gamma_k; (void)dq; (void)dk; (void)dv; (void)dgamma_q; (void)dgamma_k; (void)workspace;
-  (void)workspace_bytes; (void)dims; (void)stream;
-  return MAGI_BCA_UNSUPPORTED;
+  int st = validate_dims(dims);
+  if (st != MAGI_BCA_OK) return st;
+  const magi_bca_dims& d = *dims;
+  if (!q || !k || !v || !out || !dout || !lse || !gamma_q || !gamma_k || !dq || !dk || !dv || !workspace)
+    return MAGI_BCA_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MAGI_BCA_INVALID_ARG;
+  st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, d);
+  if (st != MAGI_BCA_OK) return st;
+  const BwdWorkspace ws = bwd_workspace_layout(d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim);
+  if (workspace_bytes < ws.total) return MAGI_BCA_WORKSPACE_TOO_SMALL;
+  int dev;
+  DeviceState* ds;
+  st = device_state(&dev, &ds);
+  if (st != MAGI_BCA_OK) return st;
+  ScheduleEntry sched;
+  st = get_schedule(dev, 1, d, q_chunk_offsets, kv_chunk_offsets, &sched);
+  if (st != MAGI_BCA_OK) return st;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  BwdParams p;
+  p.q = q;
+  p.k = k;
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.gamma_q = gamma_q;
+  p.gamma_k = gamma_k;
+  p.units = sched.dev;
+  p.q_offsets = sched.dev + (size_t)sched.n_units * kUnitInts;
+  p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
+  p.n_q_chunks = d.n_q_chunks;
+  p.n_kv_chunks = d.n_kv_chunks;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dgamma_q = dgamma_q;
+  p.dgamma_k = dgamma_k;
+  p.qn = reinterpret_cast<uint16_t*>(w + ws.qn);
+  p.ld = reinterpret_cast<float*>(w + ws.ld);
+  p.dqacc = reinterpret_cast<float*>(w + ws.dqacc);
+  p.batch = d.batch;
+  p.seqlen_q = d.seqlen_q;
+  p.seqlen_kv = d.seqlen_kv;
+  p.heads_q = d.heads_q;
+  p.heads_kv = d.heads_kv;
+  p.seqlen_q_pad = (d.seqlen_q + 127) / 128 * 128;
+  p.scale = resolve_scale(d);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  p.eps = d.rms_eps;
+  p.status = ds->status;
+  CUtensorMap t_k, t_v, t_qn, t_do;
+  if (make_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
+    return MAGI_BCA_CUDA_ERROR;
+  cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
 }
 
 int magi_bca_last_device_status(void) {

@@ -1,0 +1,637 @@
+// Backward of block-causal GQA attention with QK-RMSNorm, sm_100a.
+//
+// The backward recomputes the forward's logits from the forward's own
+// operands: the folded query Q^ = bf16(q r_q gamma_q gamma_k scale log2(e))
+// and the raw keys with the per-key factor r_k, so the recomputed P matches
+// the forward's log-sum-exp up to fp32 accumulation order (the helpers in
+// bca_norm.cuh fix the rounding points for both passes).
+//
+// Three launches on the caller's stream:
+//   1. prep      one thread per query row: Q^ into the workspace; Delta =
+//                rowsum(dO * O); {lse*log2(e), Delta} pairs in a 128-padded
+//                layout; zero the fp32 dq accumulator and dgamma.
+//   2. main      one CTA per (batch, kv head, 128-key tile).  It keeps K and V
+//                of its tile in shared memory and walks every (query tile,
+//                group head) that sees the tile (backward schedule, bca_sched.h):
+//                  S^T  = K Q^^T r_k        dP^T = V dO^T                  (TMEM)
+//                  P^T  = exp2(S^T - lse log2e)   (masked on diagonal steps)
+//                  dS'^T = P^T (dP^T - Delta) r_k   (key-row scaled, bf16 in smem)
+//                  dV  += P^T dO        (P^T from TMEM)
+//                  G_k += dS'^T Q^      -> gamma_k * dk~ = G_k / (r_k log2 e)
+//                  G_q  = dS' K         -> dq~ = scale gamma_k * G_q, drained with
+//                                          vector red.add into the fp32 accumulator
+//                and finally writes dv, and dk through the RMSNorm Jacobian (plus
+//                this tile's share of gamma_k * dgamma_k).
+//   3. finalize  one warp per query row: dq through the RMSNorm Jacobian, dgamma_q,
+//                and dgamma_k = (gamma_k * dgamma_k) / gamma_k.
+// These are the five matrix products of the Flash-Attention backward (2.5x the
+// forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
+// query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.
+//
+// Main-kernel roles: warps 0-3 / 4-7 (warpgroups 0 and 1) split the 128 query
+// columns of S^T and dP^T in halves (thread i of a warpgroup owns key row i =
+// TMEM lane i), then drain half of G_q each; warp 8 issues tcgen05 MMAs; warp 9
+// runs TMA.  TMEM: S^T [0,128) (P^T of query half w overwrites columns
+// [64w, 64w+32) once that half has been read), dP^T [128,256) (G_q overwrites
+// it), dV [256,256+D), G_k [384,384+D).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "bca_kernels.h"
+#include "bca_norm.cuh"
+#include "sm100.cuh"
+
+namespace magi {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum : int {
+  kErrKv = 2001, kErrQFull = 2002, kErrQEmpty = 2003, kErrSFull = 2004, kErrDsReady = 2005,
+  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool ok, int* status, int code) {
+  if (ok) ok = mbar_wait(bar, parity, status, code);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+
+// ------------------------------------------------------------------ prep
+// Lane l holds elements [l*E, l*E+E) of a D = 32*E row.
+template <int D>
+struct RowIO {
+  static constexpr int E = D / 32;
+  __device__ static void load_bf16(const uint16_t* row, int lane, float (&x)[E]) {
+    if constexpr (E == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(row + lane * 4);
+      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(row + lane * 2);
+      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+    }
+  }
+  __device__ static void store_bf16(uint16_t* row, int lane, const float (&x)[E]) {
+    if constexpr (E == 4) {
+      uint2 w;
+      w.x = pack_bf16x2(x[0], x[1]);
+      w.y = pack_bf16x2(x[2], x[3]);
+      *reinterpret_cast<uint2*>(row + lane * 4) = w;
+    } else {
+      *reinterpret_cast<uint32_t*>(row + lane * 2) = pack_bf16x2(x[0], x[1]);
+    }
+  }
+  __device__ static void load_f32(const float* row, int lane, float (&x)[E]) {
+    if constexpr (E == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(row + lane * 4);
+      x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(row + lane * 2);
+      x[0] = v.x; x[1] = v.y;
+    }
+  }
+  __device__ static void store_zero_f32(float* row, int lane) {
+    if constexpr (E == 4) {
+      *reinterpret_cast<float4*>(row + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      *reinterpret_cast<float2*>(row + lane * 2) = make_float2(0.f, 0.f);
+    }
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
+  __shared__ float qscale[D];
+  for (int d = threadIdx.x; d < D; d += blockDim.x) qscale[d] = qscale_of(p.gamma_q, p.gamma_k, p.scale_log2, d);
+  if (blockIdx.x == 0 && threadIdx.x < D) {
+    if (p.dgamma_q) p.dgamma_q[threadIdx.x] = 0.f;
+    if (p.dgamma_k) p.dgamma_k[threadIdx.x] = 0.f;
+  }
+  __syncthreads();
+  const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < n_q; r += (int64_t)gridDim.x * blockDim.x) {
+    // the forward's query operand, bit for bit (same helpers, same order)
+    const uint16_t* qrow = p.q + r * D;
+    const float rq = rms_inv<D>(row_sumsq_linear<D>(qrow), p.eps);
+    uint16_t* qh = p.qn + r * D;
+    float dot = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      *reinterpret_cast<uint4*>(qh + c * 8) = fold_q_chunk(*reinterpret_cast<const uint4*>(qrow + c * 8), rq, qscale, c * 8);
+      const uint4 o = *reinterpret_cast<const uint4*>(p.out + r * D + c * 8);
+      const uint4 g = *reinterpret_cast<const uint4*>(p.dout + r * D + c * 8);
+      const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dot = fmaf(bf16_lo(ow[i]), bf16_lo(gw[i]), dot);
+        dot = fmaf(bf16_hi(ow[i]), bf16_hi(gw[i]), dot);
+      }
+      *reinterpret_cast<float4*>(p.dqacc + r * D + c * 8) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(p.dqacc + r * D + c * 8 + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int h = (int)(r % p.heads_q);
+    const int64_t bs = r / p.heads_q;
+    const int s = (int)(bs % p.seqlen_q);
+    const int b = (int)(bs / p.seqlen_q);
+    const int64_t bh = (int64_t)b * p.heads_q + h;
+    float2 v;
+    v.x = __ldg(p.lse + bh * p.seqlen_q + s) * kLog2e;
+    v.y = dot;
+    *reinterpret_cast<float2*>(p.ld + (bh * p.seqlen_q_pad + s) * 2) = v;
+  }
+}
+
+// ------------------------------------------------------------------ main
+template <int D>
+struct BwdLayout {
+  static constexpr int kTile = 128 * D * 2;      // [128][D] bf16
+  static constexpr int kK = 0;                   // raw K tile
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQn = kV + kTile;         // 2 stages
+  static constexpr int kDo = kQn + 2 * kTile;    // 2 stages
+  static constexpr int kDs = kDo + 2 * kTile;    // dS^T [128 keys][128 queries] bf16, two 64-wide boxes
+  static constexpr int kLd = kDs + 32768;        // 2 stages x 128 x {lse2, Delta}
+  static constexpr int kBars = kLd + 2 * 1024;
+  static constexpr int kTmemSlot = kBars + 16 * 8;
+  static constexpr int kTotal = kTmemSlot + 16;
+};
+
+struct BwdBars {
+  uint64_t kv_full, s_full, ds_ready, dq_full, dq_drained, acc_full;
+  uint64_t q_full[2], q_empty[2];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p, const int smem_alloc) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
+  uint8_t* smem = reinterpret_cast<uint8_t*>(base);
+  // The layout needs 1024-byte alignment for the swizzled tiles; refuse to run
+  // (status, no access) if the allocation cannot hold it at this alignment.
+  if (base - reinterpret_cast<uintptr_t>(smem_raw) + L::kTotal > (uintptr_t)smem_alloc) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kErrSmem);
+    return;
+  }
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int32_t* u = p.units + (size_t)blockIdx.x * 8;
+  const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
+  const int qb = __ldg(u + 3), qe = __ldg(u + 4), n_diag = __ldg(u + 5);
+  const int group = p.heads_q / p.heads_kv;
+  const int n_steps = (qe - qb) * group;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->ds_ready, 2);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_drained, 2);
+    mbar_init(&bars->acc_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_qn);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
+      for (int box = 0; box < D / 64; ++box) {
+        tma_load_4d(smem + L::kK + box * 16384, &tm_k, &bars->kv_full, box * 64, hk, n0, b);
+        tma_load_4d(smem + L::kV + box * 16384, &tm_v, &bars->kv_full, box * 64, hk, n0, b);
+      }
+      for (int t = 0; t < n_steps; ++t) {
+        const int st = t & 1;
+        if (!mbar_wait(&bars->q_empty[st], ((t >> 1) & 1) ^ 1, p.status, kErrQEmpty)) break;
+        const int qt = qb + t / group, h = hk * group + t % group;
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 1024);
+        for (int box = 0; box < D / 64; ++box) {
+          tma_load_4d(smem + L::kQn + st * L::kTile + box * 16384, &tm_qn, &bars->q_full[st], box * 64, h,
+                      qt * 128, b);
+          tma_load_4d(smem + L::kDo + st * L::kTile + box * 16384, &tm_do, &bars->q_full[st], box * 64, h,
+                      qt * 128, b);
+        }
+        const float* ld_src = p.ld + (((size_t)b * p.heads_q + h) * p.seqlen_q_pad + (size_t)qt * 128) * 2;
+        bulk_load(smem + L::kLd + st * 1024, ld_src, 1024, &bars->q_full[st]);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t id_kk = make_idesc_bf16(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t id_ts = make_idesc_bf16(128, D, false, true);     // dV (A from TMEM)
+      constexpr uint32_t id_km = make_idesc_bf16(128, D, false, true);     // dK~: A K-major, B MN-major
+      constexpr uint32_t id_mm = make_idesc_bf16(128, D, true, true);      // dQ~: A MN-major, B MN-major
+      const uint32_t kn_a = smem_u32(smem + L::kK), v_a = smem_u32(smem + L::kV);
+      const uint32_t qn_a = smem_u32(smem + L::kQn), do_a = smem_u32(smem + L::kDo);
+      const uint32_t ds_a = smem_u32(smem + L::kDs);
+      // C[128 x 128] = A[128 x D] B[128 x D]^T with both operands K-major.
+      auto mma_kmajor = [&](uint32_t d, uint32_t a, uint32_t bb) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + d, make_sw128_desc(a + off, 16, 1024), make_sw128_desc(bb + off, 16, 1024), id_kk,
+                      kk > 0);
+        }
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, p.status, kErrKv);
+      for (int t = 0; t < n_steps && ok; ++t) {
+        const int st = t & 1;
+        const uint32_t qn_s = qn_a + st * L::kTile, do_s = do_a + st * L::kTile;
+        if (t == 0) {
+          if (!(ok = mbar_wait(&bars->q_full[0], 0, p.status, kErrQFull))) break;
+          tc_fence_after();
+          mma_kmajor(T_S, kn_a, qn_s);
+        } else {
+          if (!(ok = mbar_wait(&bars->dq_drained, (t - 1) & 1, p.status, kErrDqDrained))) break;
+          tc_fence_after();
+        }
+        mma_kmajor(T_DP, v_a, do_s);
+        mma_commit(&bars->s_full);
+        if (!(ok = mbar_wait(&bars->ds_ready, t & 1, p.status, kErrDsReady))) break;
+        tc_fence_after();
+        // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                      make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts, t > 0 || kk > 0);
+        // G_k += dS'^T Q^ : A = dS'^T [keys][queries] (K-major), B = Q^ [queries][D] (MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + T_DK, make_sw128_desc(ds_a + off, 16, 1024),
+                      make_sw128_desc(qn_s + kk * 2048, 16384, 1024), id_km, t > 0 || kk > 0);
+        }
+        // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
+                      make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
+        mma_commit(&bars->dq_full);
+        mma_commit(&bars->q_empty[st]);
+        if (t + 1 < n_steps) {
+          const int st1 = (t + 1) & 1;
+          if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
+          tc_fence_after();
+          mma_kmajor(T_S, kn_a, qn_a + st1 * L::kTile);
+        }
+      }
+      if (ok) mma_commit(&bars->acc_full);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warpgroups
+    const int wg = warp >> 2;               // query-column half
+    const int j = threadIdx.x & 127;        // key row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int bar_id = 1 + wg;
+    // First query row that sees key n0 + j: query chunk c sees keys below
+    // kv_offsets[n_kv - n_q + c + 1], so it is the first chunk whose end exceeds the key.
+    int row_min = p.seqlen_q;
+    {
+      const int key = n0 + j;
+      if (key < p.seqlen_kv) {
+        const int shift = p.n_kv_chunks - p.n_q_chunks;
+        int lo = 0, hi = p.n_q_chunks;  // first c in [0, n_q) with kv_offsets[shift + c + 1] > key
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (__ldg(p.kv_offsets + shift + mid + 1) > key) hi = mid; else lo = mid + 1;
+        }
+        row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
+      }
+    }
+    bool ok = warp_wait(&bars->kv_full, 0, true, p.status, kErrKv);
+    // r_k of this thread's key, exactly as the forward computes it
+    const float rk = ok ? rms_inv<D>(row_sumsq_swizzled<D>(smem + L::kK, j), p.eps) : 0.f;
+    for (int t = 0; t < n_steps; ++t) {
+      const int st = t & 1;
+      const int qt = qb + t / group, h = hk * group + t % group;
+      const int q0 = qt * 128;
+      const bool diag = (qt - qb) < n_diag;
+      ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
+      if (ok) {
+        tc_fence_after();
+        uint32_t sr[64], dpr[64];
+        {
+          uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+          uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
+          uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
+          tmem_ld32(tmem + lane_base + T_S + wg * 64, a0);
+          tmem_ld32(tmem + lane_base + T_S + wg * 64 + 32, a1);
+          tmem_ld32(tmem + lane_base + T_DP + wg * 64, c0);
+          tmem_ld32(tmem + lane_base + T_DP + wg * 64 + 32, c1);
+          tmem_wait_ld();
+        }
+        const float2* ld = reinterpret_cast<const float2*>(smem + L::kLd + st * 1024) + wg * 64;
+        const int lim = row_min - (q0 + wg * 64);   // columns c < lim are masked on diagonal steps
+        uint32_t pk[32], dk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float2 l0 = ld[c], l1 = ld[c + 1];
+          float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), rk, -l0.x));
+          float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), rk, -l1.x));
+          if (diag) {
+            p0 = c < lim ? 0.f : p0;
+            p1 = c + 1 < lim ? 0.f : p1;
+          }
+          const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y) * rk;
+          const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y) * rk;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+          dk[c >> 1] = pack_bf16x2(d0, d1);
+        }
+        // P^T of this half goes to the first 32 columns of the half's own S^T
+        // columns (already read), so the two warpgroups never touch each other's.
+        tmem_st32(tmem + lane_base + T_S + wg * 64, pk);
+        uint8_t* ds_box = smem + L::kDs + wg * 16384;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8)
+          *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, c8 * 8)) =
+              make_uint4(dk[4 * c8], dk[4 * c8 + 1], dk[4 * c8 + 2], dk[4 * c8 + 3]);
+        tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(bar_id, 128);
+      if (j == 0 && ok) mbar_arrive(&bars->ds_ready);
+
+      // drain G_q (rows = queries of this step) into the fp32 accumulator
+      ok = warp_wait(&bars->dq_full, t & 1, ok, p.status, kErrDqFull);
+      if (ok) {
+        tc_fence_after();
+        const int row = q0 + j;
+        float* dst = p.dqacc + (((size_t)b * p.seqlen_q + row) * p.heads_q + h) * D + wg * (D / 2);
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + T_DP + wg * (D / 2) + c, r);
+          tmem_wait_ld();
+          if (row < p.seqlen_q) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              red_add_v4(dst + c + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                         __uint_as_float(r[i + 3]));
+          }
+        }
+        tc_fence_before();
+      }
+      named_bar_sync(bar_id, 128);
+      if (j == 0 && ok) mbar_arrive(&bars->dq_drained);
+    }
+
+    // ---------------------------------------------------------- epilogue
+    ok = warp_wait(&bars->acc_full, 0, ok && n_steps > 0, p.status, kErrAcc);
+    const int key = n0 + j;
+    if (ok) {
+      tc_fence_after();
+      if (wg == 0) {
+        // dV -> bf16
+        uint16_t* dst = p.dv + (((size_t)b * p.seqlen_kv + key) * p.heads_kv + hk) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + T_DV + c, r);
+          tmem_wait_ld();
+          if (key < p.seqlen_kv) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+              w.y = pack_bf16x2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+              w.z = pack_bf16x2(__uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
+              w.w = pack_bf16x2(__uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
+              *reinterpret_cast<uint4*>(dst + c + i) = w;
+            }
+          }
+        }
+      } else {
+        // dk through the RMSNorm Jacobian: with k^ = k r_k and g = gamma_k * dk~
+        // (= G_k / (r_k log2 e)):  dk = r_k (g - k^ mean(g k^)).
+        // This tile's share of gamma_k * dgamma_k is sum_keys g * k^.
+        float* red = reinterpret_cast<float*>(smem + L::kQn);  // [128][D + 1]; stage buffers are idle now
+        const bool live = key < p.seqlen_kv;
+        const uint8_t* ktile = smem + L::kK;
+        const float gscale = 1.0f / (rk * kLog2e);
+        float dot = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + T_DK + c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const uint4 w = *reinterpret_cast<const uint4*>(ktile + ((c + i) >> 6) * 16384 + sw128_offset(j, (c + i) & 63));
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float k0 = bf16_lo(ww[e]) * rk, k1 = bf16_hi(ww[e]) * rk;
+              const float g0 = __uint_as_float(r[i + 2 * e]) * gscale;
+              const float g1 = __uint_as_float(r[i + 2 * e + 1]) * gscale;
+              dot = fmaf(g0, k0, dot);
+              dot = fmaf(g1, k1, dot);
+              red[j * (D + 1) + c + i + 2 * e] = live ? g0 * k0 : 0.f;
+              red[j * (D + 1) + c + i + 2 * e + 1] = live ? g1 * k1 : 0.f;
+            }
+          }
+        }
+        const float mean_dot = dot * (1.0f / D);
+        uint16_t* dst = p.dk + (((size_t)b * p.seqlen_kv + key) * p.heads_kv + hk) * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + T_DK + c, r);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              const uint4 w =
+                  *reinterpret_cast<const uint4*>(ktile + ((c + i) >> 6) * 16384 + sw128_offset(j, (c + i) & 63));
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float k0 = bf16_lo(ww[e]) * rk, k1 = bf16_hi(ww[e]) * rk;
+                o[2 * e] = rk * (__uint_as_float(r[i + 2 * e]) * gscale - k0 * mean_dot);
+                o[2 * e + 1] = rk * (__uint_as_float(r[i + 2 * e + 1]) * gscale - k1 * mean_dot);
+              }
+              uint4 ov;
+              ov.x = pack_bf16x2(o[0], o[1]);
+              ov.y = pack_bf16x2(o[2], o[3]);
+              ov.z = pack_bf16x2(o[4], o[5]);
+              ov.w = pack_bf16x2(o[6], o[7]);
+              *reinterpret_cast<uint4*>(dst + c + i) = ov;
+            }
+          }
+        }
+        if (p.dgamma_k != nullptr) {
+          named_bar_sync(bar_id, 128);
+          if (j < D) {
+            float acc = 0.f;
+            for (int r = 0; r < 128; ++r) acc += red[r * (D + 1) + j];
+            atomicAdd(p.dgamma_k + j, acc);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ finalize
+template <int D>
+__global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p) {
+  using IO = RowIO<D>;
+  constexpr int E = IO::E;
+  __shared__ float red[8][D];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
+  const int64_t warps = (int64_t)gridDim.x * 8;
+  float gacc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) gacc[e] = 0.f;
+  float gm[E], gk[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    gm[e] = __ldg(p.gamma_q + lane * E + e);
+    gk[e] = __ldg(p.gamma_k + lane * E + e) * p.scale;   // dq~ = scale gamma_k G_q
+  }
+  if (blockIdx.x == 0 && p.dgamma_k != nullptr && threadIdx.x < D)
+    p.dgamma_k[threadIdx.x] = p.dgamma_k[threadIdx.x] / __ldg(p.gamma_k + threadIdx.x);
+  for (int64_t r = (int64_t)blockIdx.x * 8 + wid; r < n_q; r += warps) {
+    float x[E], dqt[E];
+    IO::load_bf16(p.q + r * D, lane, x);
+    IO::load_f32(p.dqacc + r * D, lane, dqt);
+#pragma unroll
+    for (int e = 0; e < E; ++e) dqt[e] *= gk[e];
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+    const float rq = rsqrtf(warp_sum(ss) * (1.0f / D) + p.eps);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      x[e] *= rq;                                   // x^
+      dot = fmaf(gm[e] * dqt[e], x[e], dot);
+      gacc[e] = fmaf(dqt[e], x[e], gacc[e]);
+    }
+    const float mean_dot = warp_sum(dot) * (1.0f / D);
+    float o[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = rq * (gm[e] * dqt[e] - x[e] * mean_dot);
+    IO::store_bf16(p.dq + r * D, lane, o);
+  }
+  if (p.dgamma_q != nullptr) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) red[wid][lane * E + e] = gacc[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
+      atomicAdd(p.dgamma_q + threadIdx.x, acc);
+    }
+  }
+}
+
+
+template <int D>
+cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
+                         const CUtensorMap& t_do, const BwdParams& p, int n_units, cudaStream_t stream) {
+  using L = BwdLayout<D>;
+  static uint64_t configured = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int max_optin = 0;
+  e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  const int alloc = L::kTotal + 1024 <= max_optin ? L::kTotal + 1024 : max_optin;
+  if (alloc < L::kTotal) return cudaErrorInvalidConfiguration;
+  if (dev >= 64 || !((configured >> dev) & 1u)) {
+    e = cudaFuncSetAttribute(bca_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= uint64_t(1) << dev;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q;
+  const int prep_blocks = (int)std::min<int64_t>((rows + 255) / 256, (int64_t)sms * 8);
+  if (p.seqlen_q_pad != p.seqlen_q) {
+    // padding entries of the {lse, Delta} pairs are read by full-tile loads
+    e = cudaMemsetAsync(p.ld, 0, (size_t)p.batch * p.heads_q * p.seqlen_q_pad * 2 * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
+  bca_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (n_units > 0) {
+    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, p, alloc);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t qrows = (int64_t)p.batch * p.seqlen_q * p.heads_q;
+  const int fin_blocks = (int)std::min<int64_t>((qrows + 7) / 8, (int64_t)sms * 8);
+  bca_bwd_finalize_kernel<D><<<fin_blocks, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D) {
+  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t sq_pad = (size_t)((Sq + 127) / 128) * 128;
+  BwdWorkspace w;
+  w.qn = 0;
+  w.ld = w.qn + up((size_t)B * Sq * Hq * D * 2);
+  w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 2 * 4);
+  w.total = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
+  return w;
+}
+
+cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
+                       const CUtensorMap& t_do, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream) {
+  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, p, n_units, stream);
+  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, p, n_units, stream);
+}
+
+}  // namespace magi

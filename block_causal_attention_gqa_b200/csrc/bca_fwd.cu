@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include "bca_kernels.h"
+#include "bca_norm.cuh"
 #include "sm100.cuh"
 
 namespace magi {
@@ -84,27 +85,6 @@ __device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
   return lo;
 }
 
-// Sum of squares of one [D] bf16 row stored 128B-swizzled across D/64 boxes.
-template <int D>
-__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
-  float acc = 0.f;
-#pragma unroll
-  for (int box = 0; box < D / 64; ++box) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(tile + box * 16384 + sw128_offset(row, c * 8));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xffff0000u);
-        acc = fmaf(lo, lo, acc);
-        acc = fmaf(hi, hi, acc);
-      }
-    }
-  }
-  return acc;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -149,8 +129,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  for (int d = threadIdx.x; d < D; d += kThreads)
-    qscale[d] = __ldg(p.gamma_q + d) * __ldg(p.gamma_k + d) * p.scale_log2;
+  for (int d = threadIdx.x; d < D; d += kThreads) qscale[d] = qscale_of(p.gamma_q, p.gamma_k, p.scale_log2, d);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -251,22 +230,13 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // Q prologue: RMSNorm the row and fold gains, scale and log2(e) into it.
       ok = warp_wait(&bars->q_full[s], 0, ok, p.status, kErrQ);
       if (ok) {
-        const float rq = rsqrtf(row_sumsq<D>(q_tile, r) * (1.0f / D) + p.eps);
+        const float rq = rms_inv<D>(row_sumsq_swizzled<D>(q_tile, r), p.eps);
 #pragma unroll
         for (int box = 0; box < D / 64; ++box) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint4* ptr = reinterpret_cast<uint4*>(q_tile + box * 16384 + sw128_offset(r, c * 8));
-            uint4 v = *ptr;
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            const int d0 = box * 64 + c * 8;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float lo = __uint_as_float(w[i] << 16) * rq * qscale[d0 + 2 * i];
-              const float hi = __uint_as_float(w[i] & 0xffff0000u) * rq * qscale[d0 + 2 * i + 1];
-              w[i] = pack_bf16x2(lo, hi);
-            }
-            *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+            *ptr = fold_q_chunk(*ptr, rq, qscale, box * 64 + c * 8);
           }
         }
         fence_proxy_async_smem();
@@ -290,7 +260,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // r_k of this kv tile, from the resident K tile.
         ok = warp_wait(&bars->k_full[st], (j / kStages) & 1, ok, p.status, kErrKSoft);
         float* rk = rk_buf + (j & 1) * 128;
-        if (ok) rk[r] = rsqrtf(row_sumsq<D>(smem + L::kK + st * L::kTileBytes, r) * (1.0f / D) + p.eps);
+        if (ok) rk[r] = rms_inv<D>(row_sumsq_swizzled<D>(smem + L::kK + st * L::kTileBytes, r), p.eps);
         named_bar_sync(bar_id, 128);
         if (r == 0 && ok) mbar_arrive(&bars->k_empty[st]);
 

@@ -23,6 +23,44 @@ struct FwdParams {
   int* status;                // device status word (bounded waits)
 };
 
+struct BwdParams {
+  // inputs
+  const uint16_t* q;          // [B, Sq, Hq, D] raw
+  const uint16_t* k;          // [B, Skv, Hkv, D] raw
+  const uint16_t* out;        // forward output
+  const uint16_t* dout;
+  const float* lse;           // [B, Hq, Sq] natural log
+  const float* gamma_q;
+  const float* gamma_k;
+  const int32_t* units;       // device schedule, 8 int32 per unit
+  const int32_t* q_offsets;   // device copies of the chunk offsets
+  const int32_t* kv_offsets;
+  int n_q_chunks, n_kv_chunks;
+  // outputs
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  float* dgamma_q;            // may be null
+  float* dgamma_k;            // may be null
+  // workspace
+  uint16_t* qn;               // forward query operand Q^       [B, Sq, Hq, D]
+  float* ld;                  // {lse * log2(e), Delta} pairs [B, Hq, Sq_pad, 2]
+  float* dqacc;               // fp32 G_q accumulator          [B, Sq, Hq, D]
+  int batch, seqlen_q, seqlen_kv, heads_q, heads_kv, seqlen_q_pad;
+  float scale;                // softmax scale
+  float scale_log2;           // softmax scale * log2(e)
+  float eps;
+  int* status;
+};
+
+struct BwdWorkspace {
+  size_t qn, ld, dqacc, total;  // byte offsets and total size
+};
+BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D);
+
+cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
+                       const CUtensorMap& t_do, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream);
+
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream);
 size_t fwd_smem_bytes(int head_dim);

@@ -1,0 +1,74 @@
+// RMSNorm pieces shared by the forward and the backward.
+//
+// The backward recomputes the forward's logits, so both must produce the
+// same fp32 row statistics and the same bf16 query operand bit for bit:
+// every function here fixes its summation order (feature 0, 1, 2, ... in
+// sequence) and its rounding points, whether the row sits in a 128-byte
+// swizzled shared-memory tile or in global memory.
+#pragma once
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace magi {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Accumulates x*x over the 8 bf16 of one 16-byte chunk, lowest feature first.
+__device__ __forceinline__ float sumsq_chunk(uint4 v, float acc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc = fmaf(bf16_lo(w[i]), bf16_lo(w[i]), acc);
+    acc = fmaf(bf16_hi(w[i]), bf16_hi(w[i]), acc);
+  }
+  return acc;
+}
+
+// Sum of squares of row `row` of a [128][D] bf16 tile stored as D/64 boxes
+// of [128][64] with the 128-byte swizzle.
+template <int D>
+__device__ __forceinline__ float row_sumsq_swizzled(const uint8_t* tile, int row) {
+  float acc = 0.f;
+#pragma unroll
+  for (int box = 0; box < D / 64; ++box)
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      acc = sumsq_chunk(*reinterpret_cast<const uint4*>(tile + box * 16384 + sm100::sw128_offset(row, c * 8)), acc);
+  return acc;
+}
+
+// Same sum for a contiguous row in global memory (16-byte aligned).
+template <int D>
+__device__ __forceinline__ float row_sumsq_linear(const uint16_t* row) {
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) acc = sumsq_chunk(*reinterpret_cast<const uint4*>(row + c * 8), acc);
+  return acc;
+}
+
+// 1 / RMS of a row from its sum of squares.
+template <int D>
+__device__ __forceinline__ float rms_inv(float sumsq, float eps) {
+  return rsqrtf(sumsq * (1.0f / D) + eps);
+}
+
+// The forward's query operand for one 16-byte chunk (8 features starting at d0):
+// bf16(q * r_q * qscale[d]) with qscale = gamma_q * gamma_k * softmax_scale * log2(e).
+__device__ __forceinline__ uint4 fold_q_chunk(uint4 v, float rq, const float* qscale, int d0) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float lo = bf16_lo(w[i]) * rq * qscale[d0 + 2 * i];
+    const float hi = bf16_hi(w[i]) * rq * qscale[d0 + 2 * i + 1];
+    w[i] = sm100::pack_bf16x2(lo, hi);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ float qscale_of(const float* gamma_q, const float* gamma_k, float scale_log2, int d) {
+  return __ldg(gamma_q + d) * __ldg(gamma_k + d) * scale_log2;
+}
+
+}  // namespace magi

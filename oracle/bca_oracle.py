@@ -237,7 +237,7 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
 
 def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows=None,
                   kv_rows=None, kv_heads=None, batches=None, scale=None, eps=DEFAULT_EPS,
-                  block=256):
+                  block=None):
     """Exact backward on chosen rows, without a full backward.
 
     * dq of query rows ``q_rows`` (all heads): needs only those rows' P, dP
@@ -246,12 +246,11 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
       query row that sees those keys (rows are located from the mask) and
       each such row's full softmax; cheap when the keys sit in the last chunk.
 
-    Returns dict(dq [nb, R, Hq, D], dk [nb, Rk, nkh, D], dv [nb, Rk, nkh, D]),
-    keys present only for the parts requested."""
-    q = _f64(q)
+    Only the query rows needed are converted to float64.  Returns
+    dict(dq [nb, R, Hq, D], dk [nb, Rk, nkh, D], dv [nb, Rk, nkh, D]), keys
+    present only for the parts requested."""
     k = _f64(k)
     v = _f64(v)
-    do = _f64(dout)
     gq = _f64(gamma_q)
     gk = _f64(gamma_k)
     q_offsets = np.asarray(q_offsets)
@@ -259,10 +258,17 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
     B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
     scale = 1.0 / np.sqrt(D) if not scale else float(scale)
     group = Hq // Hkv
+    if block is None:
+        block = int(max(16, min(256, (1 << 25) // Skv)))
     batches = list(range(B)) if batches is None else list(batches)
+
+    def take(x, rows):
+        return _f64(x[:, torch_index(rows)] if hasattr(x, "detach") else x[:, rows])
+
     res = {}
     if q_rows is not None:
         q_rows = np.asarray(q_rows, dtype=np.int64)
+        qsel, dsel = take(q, q_rows), take(dout, q_rows)
         dq = np.zeros((len(batches), len(q_rows), Hq, D))
         for bi, b in enumerate(batches):
             kn_all = rms_norm(k[b], gk, eps)
@@ -272,14 +278,15 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                 dqn = np.zeros((len(rr), Hq, D))
                 for h in range(Hq):
                     hk = h // group
-                    qn = rms_norm(q[b, rr, h, :], gq, eps)
+                    qn = rms_norm(qsel[b, r0:r0 + block, h, :], gq, eps)
                     o, _, p = _attend_rows(qn, kn_all[:, hk, :], v[b, :, hk, :], mask, scale)
-                    g = do[b, rr, h, :]
+                    g = dsel[b, r0:r0 + block, h, :]
                     dp = g @ v[b, :, hk, :].T
                     delta = np.sum(g * o, axis=1, keepdims=True)
-                    ds = p * (dp - delta)
-                    dqn[:, h, :] = scale * (ds @ kn_all[:, hk, :])
-                dq[bi, r0:r0 + len(rr)], _ = rms_norm_backward(q[b, rr], gq, dqn, eps)
+                    dp -= delta
+                    dp *= p
+                    dqn[:, h, :] = scale * (dp @ kn_all[:, hk, :])
+                dq[bi, r0:r0 + len(rr)], _ = rms_norm_backward(qsel[b, r0:r0 + block], gq, dqn, eps)
         res["dq"] = dq
     if kv_rows is not None:
         kv_rows = np.asarray(kv_rows, dtype=np.int64)
@@ -287,8 +294,11 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
         dk = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         dv = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         # every query row that sees at least one of the requested keys
-        cols_mask = block_causal_mask(q_offsets, kv_offsets)[:, kv_rows]
-        seeing = np.nonzero(cols_mask.any(axis=1))[0]
+        cq = chunk_of(q_offsets, Sq)
+        ck = chunk_of(kv_offsets, Skv)
+        nq, nkv = len(q_offsets) - 1, len(kv_offsets) - 1
+        seeing = np.nonzero(matched_kv_chunk(cq, nq, nkv) >= ck[kv_rows].min())[0]
+        qsel, dsel = take(q, seeing), take(dout, seeing)
         for bi, b in enumerate(batches):
             kn_all = rms_norm(k[b], gk, eps)
             for khi, hk in enumerate(kv_heads):
@@ -298,10 +308,10 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                 for h in range(hk * group, (hk + 1) * group):
                     for r0 in range(0, len(seeing), block):
                         rr = seeing[r0:r0 + block]
-                        qn = rms_norm(q[b, rr, h, :], gq, eps)
+                        qn = rms_norm(qsel[b, r0:r0 + block, h, :], gq, eps)
                         mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
                         o, _, p = _attend_rows(qn, kn, vv, mask, scale)
-                        g = do[b, rr, h, :]
+                        g = dsel[b, r0:r0 + block, h, :]
                         delta = np.sum(g * o, axis=1, keepdims=True)
                         pc = p[:, kv_rows]
                         dpc = g @ vv[kv_rows].T

@@ -47,8 +47,9 @@ def test_forward_all_rows(name):
     out, lse = run_gpu(inp, w)
     o_ref, l_ref = orc.forward(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
                                inp["gamma_q"], inp["gamma_k"])
-    assert_close(f"{name} out", to_np(out), o_ref)
-    assert_close(f"{name} lse", to_np(lse), l_ref)
+    e, r = assert_close(f"{name} out", to_np(out), o_ref)
+    el, rl = assert_close(f"{name} lse", to_np(lse), l_ref)
+    print(f"{name}: out max abs {e:.2e} rel L2 {r:.2e}; lse max abs {el:.2e} rel L2 {rl:.2e}")
     if "q_f32" in inp:
         # information only: error against the unrounded fp32 inputs
         o32, _ = orc.forward(inp["q_f32"], inp["k_f32"], inp["v_f32"], w.q_offsets, w.kv_offsets,
@@ -99,5 +100,6 @@ def test_forward_full_size_sampled_rows(name):
         o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
                                         inp["gamma_q"], inp["gamma_k"], rows, batches=[b])
         idx = torch.as_tensor(rows)
-        assert_close(f"{name} out b{b}", to_np(out_c[b:b + 1, idx]), o_ref)
-        assert_close(f"{name} lse b{b}", to_np(lse_c[b:b + 1][:, :, idx]), l_ref)
+        e, r = assert_close(f"{name} out b{b}", to_np(out_c[b:b + 1, idx]), o_ref)
+        el, rl = assert_close(f"{name} lse b{b}", to_np(lse_c[b:b + 1][:, :, idx]), l_ref)
+        print(f"{name} b{b}: out max abs {e:.2e} rel L2 {r:.2e}; lse max abs {el:.2e} rel L2 {rl:.2e}")

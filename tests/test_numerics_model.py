@@ -1,0 +1,41 @@
+"""The rounding model (tests/numerics_model.py) against the oracle, on the CPU.
+
+Pins the tolerance reading for gradients of the extra edge cases: with the
+kernels' bf16 rounding points and otherwise exact arithmetic, dk of the
+LogNormal / 8-heads-per-group case already exceeds a max-abs error of 1e-2
+(beyond bf16 output rounding) while its relative L2 stays well below 5e-3, and
+the named training workload stays inside the stated bound."""
+import numpy as np
+
+import workloads
+from oracle import bca_oracle as orc
+from tests._helpers import BF16_HALF_ULP_REL, rel_l2
+from tests.numerics_model import model_fwd_bwd
+
+
+def errors(w):
+    inp = workloads.make_inputs(w, with_grad_out=True)
+    m = model_fwd_bwd(inp, w.q_offsets, w.kv_offsets)
+    ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
+                       inp["gamma_q"], inp["gamma_k"])
+    out = {}
+    for nm in ("out", "dq", "dk", "dv"):
+        d = np.abs(m[nm] - ref[nm])
+        out[nm] = (float(np.max(d - BF16_HALF_ULP_REL * np.abs(ref[nm]))), rel_l2(m[nm], ref[nm]))
+    return out
+
+
+def test_bf16_operands_alone_exceed_1e2_on_the_gqa8_lognormal_case():
+    w = workloads.custom("gqa8_long_rows", 1, [640] * 3, None, 16, 2, 128, seed=17, token_scale=True)
+    e = errors(w)
+    assert e["dk"][0] > 1e-2          # the model's own excess, no kernel involved
+    assert e["dk"][0] < 2e-2
+    for nm in ("out", "dq", "dk", "dv"):
+        assert e[nm][1] < 4e-3
+
+
+def test_named_ragged_case_inside_the_stated_bound():
+    w = workloads.custom("ragged_d64_gqa3", 1, [70, 130, 200], None, 6, 2, 64, seed=12)
+    e = errors(w)
+    for nm in ("out", "dq", "dk", "dv"):
+        assert e[nm][0] <= 1e-2 and e[nm][1] <= 5e-3

@@ -19,7 +19,7 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
+__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_noalloc", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
            "magi_bca_status_string", "magi_bca_last_device_status", "MagiBcaError", "Dims", "library",
            "library_path", "EXPORTED_SYMBOLS"]
 
@@ -27,7 +27,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmagi_bca.so")
 
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
-                    "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version"]
+                    "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
+                    "magi_bca_bwd_noalloc"]
 
 
 class MagiBcaError(RuntimeError):
@@ -62,6 +63,9 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_bwd.argtypes = [vp, vp, vp, vp, vp, f32p, i32p, i32p, f32p, f32p, vp, vp, vp, f32p, f32p, vp,
                                  ctypes.c_size_t, dp, vp]
     lib.magi_bca_bwd.restype = ctypes.c_int
+    lib.magi_bca_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, f32p, i32p, i32p, f32p, f32p, vp, vp, vp, f32p, f32p,
+                                         dp, vp]
+    lib.magi_bca_bwd_noalloc.restype = ctypes.c_int
     lib.magi_bca_bwd_workspace_size.argtypes = [dp]
     lib.magi_bca_bwd_workspace_size.restype = ctypes.c_size_t
     lib.magi_bca_status_string.argtypes = [ctypes.c_int]
@@ -206,6 +210,44 @@ def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gam
                                     ctypes.byref(dims), _stream_handle(stream, q.device))
     if st != 0:
         raise MagiBcaError(st, "magi_bca_bwd")
+    return dq, dk, dv, dgamma_q, dgamma_k
+
+
+def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
+                         dq, dk, dv, dgamma_q=None, dgamma_k=None, softmax_scale: float = 0.0,
+                         rms_eps: float = 1e-6, stream=None):
+    """Backward through the allocation-free entry point.
+
+    For callers that cannot allocate device memory or hand the library a
+    workspace (a pooled allocator owns the GPU's memory, a plugin hook must
+    not allocate, or cudaMalloc's implicit synchronisation is unaffordable).
+    Every output is passed in by the caller; the library uses its own 64 MiB
+    device array as workspace, so calls must not overlap on the GPU.  Problems
+    too large for that array raise MagiBcaError (status -4)."""
+    _check_bf16("q", q)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    for nm, t, shp in (("k", k, (B, Skv, Hkv, D)), ("v", v, (B, Skv, Hkv, D)), ("out", out, q.shape),
+                       ("dout", dout, q.shape), ("dq", dq, q.shape), ("dk", dk, k.shape), ("dv", dv, v.shape)):
+        _check_bf16(nm, t, shp)
+    _check_f32("lse", lse, (B, Hq, Sq))
+    _check_f32("gamma_q", gamma_q, (D,))
+    _check_f32("gamma_k", gamma_k, (D,))
+    for nm, t in (("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
+        if t is not None:
+            _check_f32(nm, t, (D,))
+    qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    import torch
+    with torch.cuda.device(q.device):
+        st = library().magi_bca_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                            dout.data_ptr(), lse.data_ptr(), _i32p(qo), _i32p(ko),
+                                            gamma_q.data_ptr(), gamma_k.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                            dv.data_ptr(), dgamma_q.data_ptr() if dgamma_q is not None else None,
+                                            dgamma_k.data_ptr() if dgamma_k is not None else None,
+                                            ctypes.byref(dims), _stream_handle(stream, q.device))
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_bwd_noalloc")
     return dq, dk, dv, dgamma_q, dgamma_k
 
 

@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmagi_bca.so")
-SOURCES = ["bca_api.cu", "bca_fwd.cu", "bca_bwd.cu", "bca_sched.cpp"]
+SOURCES = ["bca_api.cu", "bca_fwd.cu", "bca_bwd.cu", "bca_noalloc.cu", "bca_sched.cpp"]
 DEPS = SOURCES + ["sm100.cuh", "bca_kernels.h", "bca_sched.h", "bca_norm.cuh"]
 
 

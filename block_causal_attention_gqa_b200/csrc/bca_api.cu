@@ -132,6 +132,23 @@ float resolve_scale(const magi_bca_dims& d) {
 }
 
 }  // namespace
+
+// Entry points for other translation units of the library.
+int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+  return make_map(m, base, B, S, H, D);
+}
+
+float resolve_softmax_scale(const magi_bca_dims& d) { return resolve_scale(d); }
+
+int device_status_word(int** out) {
+  int dev;
+  DeviceState* ds;
+  const int st = device_state(&dev, &ds);
+  if (st != MAGI_BCA_OK) return st;
+  *out = ds->status;
+  return MAGI_BCA_OK;
+}
+
 }  // namespace magi
 
 using namespace magi;

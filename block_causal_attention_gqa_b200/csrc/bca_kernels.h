@@ -6,6 +6,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "../../include/magi_bca.h"
+
 namespace magi {
 
 struct FwdParams {
@@ -64,5 +66,10 @@ cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUt
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream);
 size_t fwd_smem_bytes(int head_dim);
+
+// Shared host helpers (bca_api.cu).
+int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, int D);
+float resolve_softmax_scale(const magi_bca_dims& d);
+int device_status_word(int** out);  // the status word of the current device (checks the device once)
 
 }  // namespace magi

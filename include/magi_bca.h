@@ -111,6 +111,30 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
                  void* workspace, size_t workspace_bytes,
                  const magi_bca_dims* dims, void* stream);
 
+/* Backward that allocates nothing.  Same arguments and results as
+ * magi_bca_bwd, without the workspace: the workspace and the tile schedule live
+ * in a 64 MiB array that the library keeps in every GPU's memory from load
+ * until exit.  It is for callers that cannot allocate or pass device memory,
+ * e.g. processes whose GPU memory is owned up front by a pooled allocator,
+ * plugin hooks that must not allocate, or loops that cannot take
+ * cudaMalloc's implicit synchronisation.  (The paper has no counterpart; this
+ * is a deployment variant.)
+ *   - Problems needing more than the array (workspace + schedule) return
+ *     MAGI_BCA_WORKSPACE_TOO_SMALL; e.g. 4 chunks x 1024 tokens, 16 query heads,
+ *     head_dim 128 fits.
+ *   - The first call on a device looks up the array's device address; make that
+ *     first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents, so calls
+ *     that overlap on the GPU (several streams or threads) race.  Run them in
+ *     one stream, one at a time. */
+int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                         const magi_bca_bf16* out, const magi_bca_bf16* dout, const float* lse,
+                         const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                         const float* gamma_q, const float* gamma_k,
+                         magi_bca_bf16* dq, magi_bca_bf16* dk, magi_bca_bf16* dv,
+                         float* dgamma_q, float* dgamma_k,
+                         const magi_bca_dims* dims, void* stream);
+
 /* Static text for a status code. */
 const char* magi_bca_status_string(int status);
 

@@ -28,13 +28,16 @@ library_path = os.path.join(_HERE, "libmagi_bca.so")
 
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
-                    "magi_bca_bwd_noalloc"]
+                    "magi_bca_bwd_noalloc", "magi_bca_last_error_detail"]
 
 
 class MagiBcaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where} failed: status {status} ({magi_bca_status_string(status)})")
+        detail = ""
+        if status == -5:
+            detail = "; " + library().magi_bca_last_error_detail().decode()
+        super().__init__(f"{where} failed: status {status} ({magi_bca_status_string(status)}{detail})")
 
 
 class Dims(ctypes.Structure):
@@ -74,6 +77,8 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_last_device_status.restype = ctypes.c_int
     lib.magi_bca_fwd_schedule.argtypes = [i32p, i32p, dp, i32p, ctypes.c_int64]
     lib.magi_bca_fwd_schedule.restype = ctypes.c_int64
+    lib.magi_bca_last_error_detail.argtypes = []
+    lib.magi_bca_last_error_detail.restype = ctypes.c_char_p
     lib.magi_bca_version.argtypes = []
     lib.magi_bca_version.restype = ctypes.c_char_p
     _lib = lib

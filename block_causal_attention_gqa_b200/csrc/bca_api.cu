@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -25,6 +26,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 std::mutex g_mutex;
+
+// Text of the most recent failure on this thread (CUDA call and its error).
+thread_local char g_last_detail[256] = "";
+
+int cuda_fail(const char* what, cudaError_t e) {
+  std::snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s", what, cudaGetErrorString(e));
+  return MAGI_BCA_CUDA_ERROR;
+}
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -124,7 +133,30 @@ int make_map(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_detail, sizeof(g_last_detail), "cuTensorMapEncodeTiled (bf16) failed: CUresult %d", (int)r);
+    return MAGI_BCA_CUDA_ERROR;
+  }
+  return MAGI_BCA_OK;
+}
+
+// 4-D map over the fp32 [B, S, H, D] dq accumulator with a {32, 1, 128, 1} box
+// (128 bytes wide) and the 128-byte swizzle, for bulk reduce-adds.
+int make_map_f32(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return MAGI_BCA_CUDA_ERROR;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)S * H * D * 4};
+  cuuint32_t box[4] = {32, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_detail, sizeof(g_last_detail), "cuTensorMapEncodeTiled (fp32) failed: CUresult %d", (int)r);
+    return MAGI_BCA_CUDA_ERROR;
+  }
+  return MAGI_BCA_OK;
 }
 
 float resolve_scale(const magi_bca_dims& d) {
@@ -138,7 +170,13 @@ int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, 
   return make_map(m, base, B, S, H, D);
 }
 
+int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D) {
+  return make_map_f32(m, base, B, S, H, D);
+}
+
 float resolve_softmax_scale(const magi_bca_dims& d) { return resolve_scale(d); }
+
+int record_cuda_failure(const char* what, cudaError_t e) { return cuda_fail(what, e); }
 
 int device_status_word(int** out) {
   int dev;
@@ -223,7 +261,7 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.eps = d.rms_eps;
   p.status = ds->status;
   cudaError_t e = launch_fwd(tq, tk, tv, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
+  return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("forward launch", e);
 }
 
 size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims) {
@@ -288,15 +326,18 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = ds->status;
-  CUtensorMap t_k, t_v, t_qn, t_do;
-  if (make_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+  CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
+  if (make_map_f32(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MAGI_BCA_OK : MAGI_BCA_CUDA_ERROR;
+  cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("backward launch", e);
 }
+
+const char* magi_bca_last_error_detail(void) { return g_last_detail; }
 
 int magi_bca_last_device_status(void) {
   int host = 0;

@@ -176,7 +176,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p, const int smem_alloc) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p, const int smem_alloc) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
@@ -207,7 +207,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     mbar_init(&bars->acc_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->q_empty[s], 2);   // one arrival per warpgroup once its dq reduction has left the stage
     }
     fence_mbar_init();
   }
@@ -216,6 +216,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_qn);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 8) {
     tmem_alloc(tmem_slot, 512);
@@ -303,7 +304,6 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
                       make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
         mma_commit(&bars->dq_full);
-        mma_commit(&bars->q_empty[st]);
         if (t + 1 < n_steps) {
           const int st1 = (t + 1) & 1;
           if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
@@ -345,43 +345,41 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
       if (ok) {
         tc_fence_after();
-        uint32_t sr[64], dpr[64];
-        {
-          uint32_t (&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-          uint32_t (&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-          uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[0]);
-          uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dpr[32]);
-          tmem_ld32(tmem + lane_base + T_S + wg * 64, a0);
-          tmem_ld32(tmem + lane_base + T_S + wg * 64 + 32, a1);
-          tmem_ld32(tmem + lane_base + T_DP + wg * 64, c0);
-          tmem_ld32(tmem + lane_base + T_DP + wg * 64 + 32, c1);
-          tmem_wait_ld();
-        }
         const float2* ld = reinterpret_cast<const float2*>(smem + L::kLd + st * 1024) + wg * 64;
         const int lim = row_min - (q0 + wg * 64);   // columns c < lim are masked on diagonal steps
-        uint32_t pk[32], dk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float2 l0 = ld[c], l1 = ld[c + 1];
-          float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), rk, -l0.x));
-          float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), rk, -l1.x));
-          if (diag) {
-            p0 = c < lim ? 0.f : p0;
-            p1 = c + 1 < lim ? 0.f : p1;
-          }
-          const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y) * rk;
-          const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y) * rk;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          dk[c >> 1] = pack_bf16x2(d0, d1);
-        }
-        // P^T of this half goes to the first 32 columns of the half's own S^T
-        // columns (already read), so the two warpgroups never touch each other's.
-        tmem_st32(tmem + lane_base + T_S + wg * 64, pk);
         uint8_t* ds_box = smem + L::kDs + wg * 16384;
+        // two halves of 32 query columns each, to bound register use
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[32], dpr[32];
+          tmem_ld32(tmem + lane_base + T_S + wg * 64 + half * 32, sr);
+          tmem_ld32(tmem + lane_base + T_DP + wg * 64 + half * 32, dpr);
+          tmem_wait_ld();
+          uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, c8 * 8)) =
-              make_uint4(dk[4 * c8], dk[4 * c8 + 1], dk[4 * c8 + 2], dk[4 * c8 + 3]);
+          for (int c = 0; c < 32; c += 2) {
+            const int cc = half * 32 + c;
+            const float2 l0 = ld[cc], l1 = ld[cc + 1];
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), rk, -l0.x));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), rk, -l1.x));
+            if (diag) {
+              p0 = cc < lim ? 0.f : p0;
+              p1 = cc + 1 < lim ? 0.f : p1;
+            }
+            const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y) * rk;
+            const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y) * rk;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+            dk[c >> 1] = pack_bf16x2(d0, d1);
+          }
+          // P^T of this half goes to the half's own (already read) S^T columns:
+          // query half w, 32-column part h -> columns 64w + 16h .. +16, so the
+          // two warpgroups never touch each other's columns.
+          tmem_st16(tmem + lane_base + T_S + wg * 64 + half * 16, pk);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, half * 32 + c8 * 8)) =
+                make_uint4(dk[4 * c8], dk[4 * c8 + 1], dk[4 * c8 + 2], dk[4 * c8 + 3]);
+        }
         tmem_wait_st();
         tc_fence_before();
         fence_proxy_async_smem();
@@ -389,29 +387,49 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) mbar_arrive(&bars->ds_ready);
 
-      // drain G_q (rows = queries of this step) into the fp32 accumulator
+      // Drain G_q (TMEM lane = query row of this step) into the fp32 accumulator:
+      // TMEM -> registers (then the dP^T/G_q columns are free again), registers ->
+      // this step's Q^/dO stage (idle once dq_full has fired) as 128-byte-swizzled
+      // [128 rows][32 floats] chunks, then TMA bulk reduce-adds.  The stage goes
+      // back to the producer when the bulk engine has read it.
       ok = warp_wait(&bars->dq_full, t & 1, ok, p.status, kErrDqFull);
+      constexpr int kChunks = D / 64;  // 32-column chunks per warpgroup
+      uint32_t gq[kChunks][32];
       if (ok) {
         tc_fence_after();
-        const int row = q0 + j;
-        float* dst = p.dqacc + (((size_t)b * p.seqlen_q + row) * p.heads_q + h) * D + wg * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 2; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + T_DP + wg * (D / 2) + c, r);
-          tmem_wait_ld();
-          if (row < p.seqlen_q) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              red_add_v4(dst + c + i, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                         __uint_as_float(r[i + 3]));
-          }
-        }
+        for (int c = 0; c < kChunks; ++c) tmem_ld32(tmem + lane_base + T_DP + (wg * kChunks + c) * 32, gq[c]);
+        tmem_wait_ld();
         tc_fence_before();
       }
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) mbar_arrive(&bars->dq_drained);
+      if (ok) {
+        uint8_t* stage = smem + (wg == 0 ? L::kQn : L::kDo) + st * L::kTile;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          uint8_t* chunk = stage + c * 16384 + j * 128;
+#pragma unroll
+          for (int piece = 0; piece < 8; ++piece)
+            *reinterpret_cast<uint4*>(chunk + (((piece ^ (j & 7)) & 7) << 4)) =
+                make_uint4(gq[c][4 * piece], gq[c][4 * piece + 1], gq[c][4 * piece + 2], gq[c][4 * piece + 3]);
+        }
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(bar_id, 128);
+      if (j == 0 && ok) {
+        const uint8_t* stage = smem + (wg == 0 ? L::kQn : L::kDo) + st * L::kTile;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          tma_reduce_add_4d(&tm_dq, stage + c * 16384, (wg * kChunks + c) * 32, h, q0, b);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(&bars->q_empty[st]);
+      }
     }
+    // every bulk reduction complete before the stage buffers are reused below
+    if (j == 0) tma_store_wait_all();
+    named_bar_sync(3, 256);
 
     // ---------------------------------------------------------- epilogue
     ok = warp_wait(&bars->acc_full, 0, ok && n_steps > 0, p.status, kErrAcc);
@@ -576,7 +594,8 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
 
 template <int D>
 cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                         const CUtensorMap& t_do, const BwdParams& p, int n_units, cudaStream_t stream) {
+                         const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int n_units,
+                         cudaStream_t stream) {
   using L = BwdLayout<D>;
   static uint64_t configured = 0;
   int dev = 0;
@@ -605,7 +624,7 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (n_units > 0) {
-    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, p, alloc);
+    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, p, alloc);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -629,9 +648,10 @@ BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D
 }
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                       const CUtensorMap& t_do, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream) {
-  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, p, n_units, stream);
-  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, p, n_units, stream);
+                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int head_dim, int n_units,
+                       cudaStream_t stream) {
+  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, t_dq, p, n_units, stream);
+  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, t_dq, p, n_units, stream);
 }
 
 }  // namespace magi

@@ -61,7 +61,9 @@ struct BwdWorkspace {
 BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D);
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                       const CUtensorMap& t_do, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream);
+                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int head_dim,
+                       int n_units, cudaStream_t stream);
+int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream);
@@ -71,5 +73,6 @@ size_t fwd_smem_bytes(int head_dim);
 int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 float resolve_softmax_scale(const magi_bca_dims& d);
 int device_status_word(int** out);  // the status word of the current device (checks the device once)
+int record_cuda_failure(const char* what, cudaError_t e);  // sets the error detail, returns MAGI_BCA_CUDA_ERROR
 
 }  // namespace magi

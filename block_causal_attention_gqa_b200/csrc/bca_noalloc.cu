@@ -141,12 +141,13 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = status;
-  CUtensorMap t_k, t_v, t_qn, t_do;
-  if (make_bf16_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+  CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
+  if (make_tensor_map_f32_dq(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_bf16_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  return launch_bwd(t_k, t_v, t_qn, t_do, p, d.head_dim, n_units, s) == cudaSuccess ? MAGI_BCA_OK
-                                                                                      : MAGI_BCA_CUDA_ERROR;
+  const cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, p, d.head_dim, n_units, s);
+  return e == cudaSuccess ? MAGI_BCA_OK : record_cuda_failure("allocation-free backward launch", e);
 }

@@ -138,6 +138,11 @@ int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16* k, const m
 /* Static text for a status code. */
 const char* magi_bca_status_string(int status);
 
+/* Text describing the most recent MAGI_BCA_CUDA_ERROR on the calling thread
+ * (which CUDA call failed and its error string); "" if none.  Owned by the
+ * library, valid until the thread's next failing call. */
+const char* magi_bca_last_error_detail(void);
+
 /* Reads (and clears) the device status word that bounded waits write when
  * they give up.  Synchronises with the device; returns MAGI_BCA_OK or
  * MAGI_BCA_DEVICE_TIMEOUT (or MAGI_BCA_CUDA_ERROR if the read itself fails).

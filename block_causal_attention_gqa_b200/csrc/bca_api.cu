@@ -8,6 +8,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <vector>
 
 #include "../../include/magi_bca.h"
@@ -63,6 +64,25 @@ struct ScheduleEntry {
 
 std::map<int, DeviceState> g_devices;
 std::map<std::vector<int32_t>, ScheduleEntry> g_schedules;
+// Normalised-key buffers of the forward, one per (device, stream, bytes), so
+// calls on different streams never share one.
+std::map<std::tuple<int, uintptr_t, size_t>, void*> g_knorm_bufs;
+
+int knorm_buffer(int dev, cudaStream_t stream, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto key = std::make_tuple(dev, reinterpret_cast<uintptr_t>(stream), bytes);
+  auto it = g_knorm_bufs.find(key);
+  if (it != g_knorm_bufs.end()) {
+    *out = it->second;
+    return MAGI_BCA_OK;
+  }
+  void* ptr = nullptr;
+  const cudaError_t e = cudaMalloc(&ptr, bytes);
+  if (e != cudaSuccess) return cuda_fail("cudaMalloc (normalised-key buffer)", e);
+  g_knorm_bufs[key] = ptr;
+  *out = ptr;
+  return MAGI_BCA_OK;
+}
 
 // Checks the current device once (sm_100 family) and resolves the status word.
 int device_state(int* device_out, DeviceState** st_out) {
@@ -239,9 +259,16 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   ScheduleEntry sched;
   st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, &sched);
   if (st != MAGI_BCA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int64_t kv_rows = (int64_t)d.batch * d.seqlen_kv * d.heads_kv;
+  void* kn = nullptr;
+  st = knorm_buffer(dev, cs, (size_t)kv_rows * d.head_dim * 2, &kn);
+  if (st != MAGI_BCA_OK) return st;
+  cudaError_t ke = launch_knorm(k, static_cast<uint16_t*>(kn), kv_rows, d.head_dim, d.rms_eps, cs);
+  if (ke != cudaSuccess) return cuda_fail("key normalisation launch", ke);
   CUtensorMap tq, tk, tv;
   if (make_map(&tq, q, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
-      make_map(&tk, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&tk, kn, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&tv, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
   FwdParams p;
@@ -260,7 +287,7 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.scale_log2 = resolve_scale(d) * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = ds->status;
-  cudaError_t e = launch_fwd(tq, tk, tv, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_fwd(tq, tk, tv, p, d.head_dim, sched.n_units, cs);
   return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("forward launch", e);
 }
 
@@ -314,6 +341,7 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.dgamma_q = dgamma_q;
   p.dgamma_k = dgamma_k;
   p.qn = reinterpret_cast<uint16_t*>(w + ws.qn);
+  p.kn = reinterpret_cast<uint16_t*>(w + ws.kn);
   p.ld = reinterpret_cast<float*>(w + ws.ld);
   p.dqacc = reinterpret_cast<float*>(w + ws.dqacc);
   p.batch = d.batch;
@@ -328,7 +356,7 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.status = ds->status;
   CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
   if (make_map_f32(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
-      make_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map(&t_k, p.kn, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)

@@ -2,14 +2,15 @@
 //
 // The backward recomputes the forward's logits from the forward's own
 // operands: the folded query Q^ = bf16(q r_q gamma_q gamma_k scale log2(e))
-// and the raw keys with the per-key factor r_k, so the recomputed P matches
-// the forward's log-sum-exp up to fp32 accumulation order (the helpers in
-// bca_norm.cuh fix the rounding points for both passes).
+// and the normalised keys K^ = bf16(k r_k) from the same bca_knorm_kernel, so
+// the recomputed P matches the forward's log-sum-exp up to fp32 accumulation
+// order (the helpers in bca_norm.cuh fix the rounding points for both passes).
 //
 // Three launches on the caller's stream:
 //   1. prep      one thread per query row: Q^ into the workspace; Delta =
 //                rowsum(dO * O); {lse*log2(e), Delta} pairs in a 128-padded
-//                layout; zero the fp32 dq accumulator and dgamma.
+//                layout; zero the fp32 dq accumulator and dgamma; then K^ into
+//                the workspace (bca_knorm_kernel, one warp per key row).
 //   2. main      one CTA per (batch, kv head, 128-key tile).  It keeps K and V
 //                of its tile in shared memory and walks every (query tile,
 //                group head) that sees the tile (backward schedule, bca_sched.h):
@@ -53,7 +54,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
   kErrKv = 2001, kErrQFull = 2002, kErrQEmpty = 2003, kErrSFull = 2004, kErrDsReady = 2005,
-  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009
+  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009, kErrMmaDone = 2010
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool ok, int* status, int code) {
@@ -168,7 +169,7 @@ struct BwdLayout {
 };
 
 struct BwdBars {
-  uint64_t kv_full, s_full, ds_ready, dq_full, dq_drained, acc_full;
+  uint64_t kv_full, s_full, ds_ready, dq_full, dq_drained, acc_full, mma_done;
   uint64_t q_full[2], q_empty[2];
 };
 
@@ -205,6 +206,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_drained, 2);
     mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 2);   // one arrival per warpgroup once its dq reduction has left the stage
@@ -286,11 +288,12 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         mma_commit(&bars->s_full);
         if (!(ok = mbar_wait(&bars->ds_ready, t & 1, p.status, kErrDsReady))) break;
         tc_fence_after();
-        // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major)
+        // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 2) * 64 + (kk & 3) * 8,
-                      make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts, t > 0 || kk > 0);
+          mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
+                      make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
+        mma_commit(&bars->dq_full);   // the drain overlaps the two products below
         // G_k += dS'^T Q^ : A = dS'^T [keys][queries] (K-major), B = Q^ [queries][D] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -298,12 +301,12 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           mma_bf16_ss(tmem + T_DK, make_sw128_desc(ds_a + off, 16, 1024),
                       make_sw128_desc(qn_s + kk * 2048, 16384, 1024), id_km, t > 0 || kk > 0);
         }
-        // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
+        // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
-                      make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
-        mma_commit(&bars->dq_full);
+          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                      make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts, t > 0 || kk > 0);
+        mma_commit(&bars->mma_done);   // this step's Q^ / dO stage and dS'^T are no longer read
         if (t + 1 < n_steps) {
           const int st1 = (t + 1) & 1;
           if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
@@ -334,9 +337,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
       }
     }
-    bool ok = warp_wait(&bars->kv_full, 0, true, p.status, kErrKv);
-    // r_k of this thread's key, exactly as the forward computes it
-    const float rk = ok ? rms_inv<D>(row_sumsq_swizzled<D>(smem + L::kK, j), p.eps) : 0.f;
+    bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
       const int st = t & 1;
       const int qt = qb + t / group, h = hk * group + t % group;
@@ -360,14 +361,14 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           for (int c = 0; c < 32; c += 2) {
             const int cc = half * 32 + c;
             const float2 l0 = ld[cc], l1 = ld[cc + 1];
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[c]), rk, -l0.x));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), rk, -l1.x));
+            float p0 = fast_exp2(__uint_as_float(sr[c]) - l0.x);
+            float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - l1.x);
             if (diag) {
               p0 = cc < lim ? 0.f : p0;
               p1 = cc + 1 < lim ? 0.f : p1;
             }
-            const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y) * rk;
-            const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y) * rk;
+            const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y);
+            const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y);
             pk[c >> 1] = pack_bf16x2(p0, p1);
             dk[c >> 1] = pack_bf16x2(d0, d1);
           }
@@ -404,6 +405,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       }
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) mbar_arrive(&bars->dq_drained);
+      // the stage is staging space only once the dK~ and dV products have read it
+      ok = warp_wait(&bars->mma_done, t & 1, ok, p.status, kErrMmaDone);
       if (ok) {
         uint8_t* stage = smem + (wg == 0 ? L::kQn : L::kDo) + st * L::kTile;
 #pragma unroll
@@ -458,12 +461,14 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
       } else {
         // dk through the RMSNorm Jacobian: with k^ = k r_k and g = gamma_k * dk~
-        // (= G_k / (r_k log2 e)):  dk = r_k (g - k^ mean(g k^)).
+        // (= G_k / log2 e):  dk = r_k (g - k^ mean(g k^)).  The raw key row is
+        // read from global memory (the shared tile holds K^).
         // This tile's share of gamma_k * dgamma_k is sum_keys g * k^.
         float* red = reinterpret_cast<float*>(smem + L::kQn);  // [128][D + 1]; stage buffers are idle now
         const bool live = key < p.seqlen_kv;
-        const uint8_t* ktile = smem + L::kK;
-        const float gscale = 1.0f / (rk * kLog2e);
+        const uint16_t* krow = p.k + (((size_t)b * p.seqlen_kv + (live ? key : 0)) * p.heads_kv + hk) * D;
+        const float rk = rms_inv<D>(row_sumsq_linear<D>(krow), p.eps);
+        constexpr float gscale = 1.0f / kLog2e;
         float dot = 0.f;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
@@ -472,7 +477,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(ktile + ((c + i) >> 6) * 16384 + sw128_offset(j, (c + i) & 63));
+            const uint4 w = *reinterpret_cast<const uint4*>(krow + c + i);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -496,8 +501,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           if (live) {
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
-              const uint4 w =
-                  *reinterpret_cast<const uint4*>(ktile + ((c + i) >> 6) * 16384 + sw128_offset(j, (c + i) & 63));
+              const uint4 w = *reinterpret_cast<const uint4*>(krow + c + i);
               const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
               float o[8];
 #pragma unroll
@@ -623,6 +627,8 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   bca_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  e = launch_knorm(p.k, p.kn, (int64_t)p.batch * p.seqlen_kv * p.heads_kv, D, p.eps, stream);
+  if (e != cudaSuccess) return e;
   if (n_units > 0) {
     bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, p, alloc);
     e = cudaGetLastError();
@@ -641,7 +647,8 @@ BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D
   const size_t sq_pad = (size_t)((Sq + 127) / 128) * 128;
   BwdWorkspace w;
   w.qn = 0;
-  w.ld = w.qn + up((size_t)B * Sq * Hq * D * 2);
+  w.kn = w.qn + up((size_t)B * Sq * Hq * D * 2);
+  w.ld = w.kn + up((size_t)B * Skv * Hkv * D * 2);
   w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 2 * 4);
   w.total = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
   return w;

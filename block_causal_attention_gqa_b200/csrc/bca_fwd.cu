@@ -17,18 +17,25 @@
 // operation of the thread has, so s_full also says "O_s is up to date".
 //
 // QK-RMSNorm fold.  With r_q = rsqrt(mean q^2 + eps), r_k likewise,
-//   scale * q~.k~ = r_q r_k sum_d (q_d gamma_q[d] gamma_k[d] scale) k_d.
-// The softmax warps scale each Q row once by r_q * gamma_q*gamma_k*scale*log2(e)
-// in shared memory (the MMA then produces logits in log2 units up to the
-// per-key factor), and apply r_k of key j as a column factor on S.  r_k is
-// computed from the K tile in shared memory while it is resident.
-//
+//   scale * q~.k~ = sum_d (q_d r_q gamma_q[d] gamma_k[d] scale) (k_d r_k).
+// bca_knorm_kernel writes K^ = bf16(k r_k) once per call (one warp per key
+// row), the TMA streams K^, and the softmax warps scale each Q row once in
+// shared memory by r_q gamma_q gamma_k scale log2(e); the MMA then produces
+// the logits directly in log2 units, with nothing left to apply per element.
+
 // Online softmax with a lazy maximum: a row's reference maximum moves only
 // when a tile's maximum exceeds it by more than 8 (log2 units), so P <= 256
 // and the O rescale (TMEM load, multiply, store) is rare after the first
 // tiles.  The result is exact: O and l are always scaled by the same factor.
+//
+// Throughput of the softmax: the row is processed as fp32 pairs with the
+// .f32x2 instructions, and on unmasked tiles one exponential in four is
+// computed by a cubic on the FMA pipe instead of MUFU (exp2_poly_pair), so
+// MUFU time per tile stays below the other sub-tile's MMA time.
 #include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "bca_kernels.h"
 #include "bca_norm.cuh"
@@ -55,8 +62,7 @@ struct FwdLayout {
   static constexpr int kQ = 0;                     // 2 sub-tiles
   static constexpr int kK = kQ + 2 * kTileBytes;   // kStages
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kRk = kV + kStages * kTileBytes;  // float [2 wg][2 buf][128]
-  static constexpr int kQScale = kRk + 2 * 2 * 128 * 4;   // float [D]
+  static constexpr int kQScale = kV + kStages * kTileBytes;  // float [D]
   static constexpr int kBars = kQScale + D * 4;
   static constexpr int kNumBars = 16;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
@@ -85,6 +91,30 @@ __device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
   return lo;
 }
 
+// 2^a for a pair, a <= 8.5: j = round(a) via the 1.5*2^23 rounding constant,
+// f = a - j in [-1/2, 1/2], 2^f by a minimax cubic (relative error 7.5e-5,
+// fitted by fit_exp2_poly.py), and 2^j added to the exponent bits.  Inputs
+// below -125 are clamped there (results ~1e-38 instead of smaller); callers
+// use it only where no element is masked to -inf.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t a2, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float a0, a1;
+  f2_unpack(a2, a0, a1);
+  a2 = f2_pack(fmaxf(a0, -125.f), fmaxf(a1, -125.f));
+  const uint64_t t2 = f2_add(a2, f2_pack(kRound, kRound));
+  const uint64_t j2 = f2_add(t2, f2_pack(-kRound, -kRound));
+  const uint64_t fr = f2_fma(j2, f2_pack(-1.f, -1.f), a2);
+  uint64_t q = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), fr,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  q = f2_fma(q, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  q = f2_fma(q, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float t0, t1, q0, q1;
+  f2_unpack(t2, t0, t1);
+  f2_unpack(q, q0, q1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -100,10 +130,10 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int lane = threadIdx.x & 31;
   const int32_t* u = p.units + (size_t)blockIdx.x * 8;
   const int b = __ldg(u + 0), hk = __ldg(u + 1);
-  const int head[2] = {__ldg(u + 2), __ldg(u + 4)};
-  const int m0[2] = {__ldg(u + 3), __ldg(u + 5)};
+  const int head0 = __ldg(u + 2), head1 = __ldg(u + 4);
+  const int m00 = __ldg(u + 3), m01 = __ldg(u + 5);
   const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
-  const int n_sub = head[1] >= 0 ? 2 : 1;
+  const int n_sub = head1 >= 0 ? 2 : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -114,7 +144,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&bars->k_full[st], 1);
-      mbar_init(&bars->k_empty[st], 1 + n_sub);  // MMA commit + each softmax warpgroup's r_k pass
+      mbar_init(&bars->k_empty[st], 1);
       mbar_init(&bars->v_full[st], 1);
       mbar_init(&bars->v_empty[st], 1);
     }
@@ -142,7 +172,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_arrive_expect_tx(&bars->q_full[s], L::kTileBytes);
         for (int box = 0; box < D / 64; ++box)
           tma_load_4d(smem + L::kQ + s * L::kTileBytes + box * 16384, &tm_q, &bars->q_full[s], box * 64,
-                      head[s], m0[s], b);
+                      s ? head1 : head0, s ? m01 : m00, b);
       }
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j % kStages;
@@ -223,7 +253,6 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const uint32_t t_s = tmem + lane_base + 256 * s;        // S_s / P_s
       const uint32_t t_o = tmem + lane_base + 256 * s + 128;  // O_s
       uint8_t* q_tile = smem + L::kQ + s * L::kTileBytes;
-      float* rk_buf = reinterpret_cast<float*>(smem + L::kRk) + s * 256;
       const int bar_id = 1 + s;
       bool ok = true;
 
@@ -245,7 +274,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (r == 0 && ok) mbar_arrive(&bars->q_ready[s]);
 
       // Visible-key end of this row.
-      const int row = m0[s] + r;
+      const int row = (s ? m01 : m00) + r;
       int limit = p.seqlen_kv;
       if (row < p.seqlen_q) {
         const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
@@ -256,85 +285,98 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // Every thread runs all n_tiles iterations and reaches every named
       // barrier even after a failed wait; only the work is skipped.
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % kStages;
-        // r_k of this kv tile, from the resident K tile.
-        ok = warp_wait(&bars->k_full[st], (j / kStages) & 1, ok, p.status, kErrKSoft);
-        float* rk = rk_buf + (j & 1) * 128;
-        if (ok) rk[r] = rms_inv<D>(row_sumsq_swizzled<D>(smem + L::kK + st * L::kTileBytes, r), p.eps);
-        named_bar_sync(bar_id, 128);
-        if (r == 0 && ok) mbar_arrive(&bars->k_empty[st]);
-
         ok = warp_wait(&bars->s_full[s], j & 1, ok, p.status, kErrSFull);
         if (ok) {
-        tc_fence_after();
-        float x[128];
+          tc_fence_after();
+          // S row (log2-unit logits) as 64 fp32 pairs
+          uint64_t x2[64];
+          {
+            uint32_t raw[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(t_s + c * 32, raw);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(raw[i]);
-        }
-        float m_tile = -INFINITY;
-        const float4* rk4 = reinterpret_cast<const float4*>(rk);
-        if (j >= n_full) {
-          const int lim = limit - j * 128;
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float4 f = rk4[c];
-            x[4 * c + 0] = (4 * c + 0 < lim) ? x[4 * c + 0] * f.x : -INFINITY;
-            x[4 * c + 1] = (4 * c + 1 < lim) ? x[4 * c + 1] * f.y : -INFINITY;
-            x[4 * c + 2] = (4 * c + 2 < lim) ? x[4 * c + 2] * f.z : -INFINITY;
-            x[4 * c + 3] = (4 * c + 3 < lim) ? x[4 * c + 3] * f.w : -INFINITY;
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float4 f = rk4[c];
-            x[4 * c + 0] *= f.x;
-            x[4 * c + 1] *= f.y;
-            x[4 * c + 2] *= f.z;
-            x[4 * c + 3] *= f.w;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 128; ++c) m_tile = fmaxf(m_tile, x[c]);
-        // Lazy maximum: move the reference only when P could exceed 2^8.
-        float alpha = 1.f;
-        if (m_tile > m_ref + kRescaleThreshold) {
-          alpha = fast_exp2(m_ref - m_tile);  // 0 on the first tile (m_ref = -inf)
-          m_ref = m_tile;
-          l_sum *= alpha;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // PV(j-1) is complete (s_full of tile j is committed after it).
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c * 32, o);
+            for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, raw[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(t_o + c * 32, o);
-          }
-        }
-        float l_tile = 0.f;
+            for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = fast_exp2(x[c * 32 + 2 * i] - m_ref);
-            const float p1 = fast_exp2(x[c * 32 + 2 * i + 1] - m_ref);
-            l_tile += p0 + p1;
-            pk[i] = pack_bf16x2(p0, p1);
+              for (int i = 0; i < 16; ++i)
+                x2[c * 16 + i] = f2_pack(__uint_as_float(raw[c][2 * i]), __uint_as_float(raw[c][2 * i + 1]));
           }
-          tmem_st16(t_s + c * 16, pk);
-        }
-        l_sum += l_tile;
-        tmem_wait_st();
-        tc_fence_before();
+          const bool masked = j >= n_full;
+          if (masked) {
+            const int lim = limit - j * 128;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              float a0, a1;
+              f2_unpack(x2[c], a0, a1);
+              x2[c] = f2_pack(2 * c < lim ? a0 : -INFINITY, 2 * c + 1 < lim ? a1 : -INFINITY);
+            }
+          }
+          // row maximum as a tree (short dependency chains)
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) f2_unpack(x2[i], mx[2 * i], mx[2 * i + 1]);
+#pragma unroll
+          for (int c = 4; c < 64; c += 4)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float a0, a1;
+              f2_unpack(x2[c + i], a0, a1);
+              mx[2 * i] = fmaxf(mx[2 * i], a0);
+              mx[2 * i + 1] = fmaxf(mx[2 * i + 1], a1);
+            }
+          const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          // Lazy maximum: move the reference only when P could exceed 2^8.
+          float alpha = 1.f;
+          if (m_tile > m_ref + kRescaleThreshold) {
+            alpha = fast_exp2(m_ref - m_tile);  // 0 on the first tile (m_ref = -inf)
+            m_ref = m_tile;
+            l_sum *= alpha;
+          }
+          const uint64_t negm = f2_pack(-m_ref, -m_ref);
+          uint64_t ls2[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint64_t a2 = f2_add(x2[c * 16 + i], negm);
+              float p0, p1;
+              if ((i & 3) == 3 && !masked) {
+                exp2_poly_pair(a2, p0, p1);
+              } else {
+                float a0, a1;
+                f2_unpack(a2, a0, a1);
+                p0 = fast_exp2(a0);
+                p1 = fast_exp2(a1);
+              }
+              const uint64_t p2 = f2_pack(p0, p1);
+              ls2[i & 3] = f2_add(ls2[i & 3], p2);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(t_s + c * 16, pk);
+          }
+          {
+            float s[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) f2_unpack(ls2[i], s[2 * i], s[2 * i + 1]);
+            l_sum += ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+          }
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // PV(j-1) is complete (s_full of tile j is committed after it); PV(j) is
+            // issued only after p_ready below, so O can be rescaled here.
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(t_o + c * 32, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
         }
         named_bar_sync(bar_id, 128);
         if (r == 0 && ok) mbar_arrive(&bars->p_ready[s]);
@@ -346,7 +388,8 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
         const float inv_l = 1.f / l_sum;
         const bool live = row < p.seqlen_q;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.seqlen_q + row) * p.heads_q + head[s]) * D);
+        const int hs = s ? head1 : head0;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (((size_t)b * p.seqlen_q + row) * p.heads_q + hs) * D);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -365,7 +408,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
         if (live && p.lse != nullptr)
-          p.lse[((size_t)b * p.heads_q + head[s]) * p.seqlen_q + row] = (m_ref + log2f(l_sum)) * kLn2;
+          p.lse[((size_t)b * p.heads_q + hs) * p.seqlen_q + row] = (m_ref + log2f(l_sum)) * kLn2;
       }
     }
   }
@@ -379,6 +422,55 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 }  // namespace
+
+// K^ = bf16(k r_k), r_k = rsqrt(mean_d k^2 + eps): one warp per key row, lane l
+// holding features [l*D/32, (l+1)*D/32).  The backward runs the same kernel,
+// so both passes see identical key operands.
+template <int D>
+__global__ void __launch_bounds__(256) bca_knorm_kernel(const uint16_t* __restrict__ k, uint16_t* __restrict__ kn,
+                                                         int64_t rows, float eps) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const uint16_t* src = k + r * D + lane * E;
+    float x[E];
+    if constexpr (E == 4) {
+      const uint2 w = *reinterpret_cast<const uint2*>(src);
+      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    } else {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rk = rms_inv<D>(ss, eps);
+    if constexpr (E == 4) {
+      uint2 w;
+      w.x = pack_bf16x2(x[0] * rk, x[1] * rk);
+      w.y = pack_bf16x2(x[2] * rk, x[3] * rk);
+      *reinterpret_cast<uint2*>(kn + r * D + lane * E) = w;
+    } else {
+      *reinterpret_cast<uint32_t*>(kn + r * D + lane * E) = pack_bf16x2(x[0] * rk, x[1] * rk);
+    }
+  }
+}
+
+cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 16);
+  if (blocks <= 0) return cudaSuccess;
+  if (head_dim == 128)
+    bca_knorm_kernel<128><<<blocks, 256, 0, stream>>>(k, kn, rows, eps);
+  else
+    bca_knorm_kernel<64><<<blocks, 256, 0, stream>>>(k, kn, rows, eps);
+  return cudaGetLastError();
+}
 
 template <int D>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

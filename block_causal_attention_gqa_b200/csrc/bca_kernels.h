@@ -46,6 +46,7 @@ struct BwdParams {
   float* dgamma_k;            // may be null
   // workspace
   uint16_t* qn;               // forward query operand Q^       [B, Sq, Hq, D]
+  uint16_t* kn;               // forward key operand K^ = bf16(k r_k) [B, Skv, Hkv, D]
   float* ld;                  // {lse * log2(e), Delta} pairs [B, Hq, Sq_pad, 2]
   float* dqacc;               // fp32 G_q accumulator          [B, Sq, Hq, D]
   int batch, seqlen_q, seqlen_kv, heads_q, heads_kv, seqlen_q_pad;
@@ -56,7 +57,7 @@ struct BwdParams {
 };
 
 struct BwdWorkspace {
-  size_t qn, ld, dqacc, total;  // byte offsets and total size
+  size_t qn, kn, ld, dqacc, total;  // byte offsets and total size
 };
 BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D);
 
@@ -64,6 +65,9 @@ cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUt
                        const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int head_dim,
                        int n_units, cudaStream_t stream);
 int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
+
+// K^ = bf16(k rsqrt(mean k^2 + eps)) for `rows` rows of head_dim features.
+cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream);
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream);

@@ -129,6 +129,7 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.dgamma_q = dgamma_q;
   p.dgamma_k = dgamma_k;
   p.qn = reinterpret_cast<uint16_t*>(scratch + ws.qn);
+  p.kn = reinterpret_cast<uint16_t*>(scratch + ws.kn);
   p.ld = reinterpret_cast<float*>(scratch + ws.ld);
   p.dqacc = reinterpret_cast<float*>(scratch + ws.dqacc);
   p.batch = d.batch;
@@ -143,7 +144,7 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.status = status;
   CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
   if (make_tensor_map_f32_dq(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
-      make_bf16_map(&t_k, k, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_bf16_map(&t_k, p.kn, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)

@@ -3,12 +3,12 @@
 Reproduces, in float64 arithmetic with explicit bf16 roundings, what the CUDA
 forward and backward round and where:
 
-forward   q^ = bf16(q r_q gamma_q gamma_k scale log2 e); raw bf16 k; logits
-          x = (q^ . k) r_k (log2 units); P = exp2(x - m); O = sum bf16(P) v / sum P
+forward   q^ = bf16(q r_q gamma_q gamma_k scale log2 e); k^ = bf16(k r_k); logits
+          x = q^ . k^ (log2 units); P = exp2(x - m); O = sum bf16(P) v / sum P
           -> bf16; lse = m + log2(sum P).
 backward  P = exp2(x - lse) from the same operands; Delta = rowsum(dO * bf16(O));
           dS = P (dP - Delta); dV = bf16(P)^T dO; gamma_k dk~ and dq~ from bf16(dS)
-          with the folded query operand and raw keys; RMSNorm Jacobians in float64;
+          with the folded query operand and k^; RMSNorm Jacobians in float64;
           outputs rounded to bf16.
 
 It is used to tell bf16-operand error from defects: when the GPU result equals
@@ -40,9 +40,9 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6):
     rk = torch.rsqrt((k * k).mean(-1, keepdim=True) + eps)
     mask = torch.tensor(orc.block_causal_mask(q_offsets, kv_offsets))
     kr, vr = k.repeat_interleave(g, 2), v.repeat_interleave(g, 2)
-    rkr = rk.repeat_interleave(g, 2).squeeze(-1).permute(0, 2, 1)[:, :, None, :]
+    kh = _bf(kr * rk.repeat_interleave(g, 2))
     qh = _bf(q * rq * (gq * gk * sc * l2e))
-    x = torch.einsum("bihd,bjhd->bhij", qh, kr) * rkr
+    x = torch.einsum("bihd,bjhd->bhij", qh, kh)
     x = x.masked_fill(~mask, -np.inf)
     m = x.amax(-1, keepdim=True)
     p = torch.exp2(x - m)
@@ -57,7 +57,7 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6):
     dv = torch.einsum("bhij,bihd->bjhd", _bf(pb), do).view(B, -1, Hkv, g, D).sum(3)
     q_op = qh / (gk * sc * l2e)                      # what the folded operand represents
     dkt = sc * torch.einsum("bhij,bihd->bjhd", ds, q_op).view(B, -1, Hkv, g, D).sum(3)
-    dqt = sc * torch.einsum("bhij,bjhd->bihd", ds, kr * rk.repeat_interleave(g, 2) * gk)
+    dqt = sc * torch.einsum("bhij,bjhd->bihd", ds, kh * gk)
     dq, _ = orc.rms_norm_backward(q.numpy(), gq.numpy(), dqt.numpy(), eps)
     dk, _ = orc.rms_norm_backward(k.numpy(), gk.numpy(), dkt.numpy(), eps)
     return dict(out=out_bf.numpy(), lse=(lse2 / l2e).squeeze(-1).numpy(), dq=_bf(torch.tensor(dq)).numpy(),

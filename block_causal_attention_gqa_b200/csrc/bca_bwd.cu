@@ -29,12 +29,12 @@
 // forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
 // query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.
 //
-// Main-kernel roles: warps 0-3 / 4-7 (warpgroups 0 and 1) split the 128 query
-// columns of S^T and dP^T in halves (thread i of a warpgroup owns key row i =
-// TMEM lane i), then drain half of G_q each; warp 8 issues tcgen05 MMAs; warp 9
-// runs TMA.  TMEM: S^T [0,128) (P^T of query half w overwrites columns
-// [64w, 64w+32) once that half has been read), dP^T [128,256) (G_q overwrites
-// it), dV [256,256+D), G_k [384,384+D).
+// Main-kernel roles: warpgroups 0-3 (warps 0-15) each own 32 of the 128 query
+// columns of S^T and dP^T (thread i of a warpgroup owns key row i = TMEM lane
+// i) and 32 columns of G_q to drain; warp 16 issues tcgen05 MMAs; warp 17 runs
+// TMA.  TMEM: S^T [0,128) (P^T of warpgroup w overwrites columns [32w, 32w+16)
+// once they have been read), dP^T [128,256) (G_q overwrites it), dV [256,256+D),
+// G_k [384,384+D).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -49,7 +49,10 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kComputeWarpgroups = 4;               // each owns 32 of the 128 query columns
+constexpr int kMmaWarp = 4 * kComputeWarpgroups;      // warp 16
+constexpr int kTmaWarp = kMmaWarp + 1;                // warp 17
+constexpr int kThreads = 32 * (kTmaWarp + 1);         // 576
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
@@ -202,25 +205,25 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->ds_ready, 2);
+    mbar_init(&bars->ds_ready, kComputeWarpgroups);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_drained, 2);
+    mbar_init(&bars->dq_drained, kComputeWarpgroups);
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], 2);   // one arrival per warpgroup once its dq reduction has left the stage
+      mbar_init(&bars->q_empty[s], kComputeWarpgroups);   // each warpgroup, once its dq staging is read
     }
     fence_mbar_init();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_qn);
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -230,7 +233,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const uint32_t tmem = *tmem_slot;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
 
-  if (warp == 9) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
       mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
@@ -253,7 +256,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         bulk_load(smem + L::kLd + st * 1024, ld_src, 1024, &bars->q_full[st]);
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       constexpr uint32_t id_kk = make_idesc_bf16(128, 128, false, false);  // S^T, dP^T
@@ -273,19 +276,21 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
       };
       bool ok = mbar_wait(&bars->kv_full, 0, p.status, kErrKv);
+      // Issue order per step t: dQ~(t) | dK~(t), dV(t) | dP(t+1), S(t+1), so the
+      // next step's products queue right behind this step's without waiting
+      // for the issuing thread.
+      if (ok && n_steps > 0) {
+        ok = mbar_wait(&bars->q_full[0], 0, p.status, kErrQFull);
+        if (ok) {
+          tc_fence_after();
+          mma_kmajor(T_DP, v_a, do_a);
+          mma_kmajor(T_S, kn_a, qn_a);
+          mma_commit(&bars->s_full);
+        }
+      }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t & 1;
         const uint32_t qn_s = qn_a + st * L::kTile, do_s = do_a + st * L::kTile;
-        if (t == 0) {
-          if (!(ok = mbar_wait(&bars->q_full[0], 0, p.status, kErrQFull))) break;
-          tc_fence_after();
-          mma_kmajor(T_S, kn_a, qn_s);
-        } else {
-          if (!(ok = mbar_wait(&bars->dq_drained, (t - 1) & 1, p.status, kErrDqDrained))) break;
-          tc_fence_after();
-        }
-        mma_kmajor(T_DP, v_a, do_s);
-        mma_commit(&bars->s_full);
         if (!(ok = mbar_wait(&bars->ds_ready, t & 1, p.status, kErrDsReady))) break;
         tc_fence_after();
         // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
@@ -304,21 +309,24 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 2) * 64 + (kk & 3) * 8,
+          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 1) * 32 + (kk & 1) * 8,
                       make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts, t > 0 || kk > 0);
-        mma_commit(&bars->mma_done);   // this step's Q^ / dO stage and dS'^T are no longer read
+        mma_commit(&bars->mma_done);   // this step's Q^ / dO stage and dS^T are no longer read
         if (t + 1 < n_steps) {
           const int st1 = (t + 1) & 1;
+          if (!(ok = mbar_wait(&bars->dq_drained, t & 1, p.status, kErrDqDrained))) break;
           if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
           tc_fence_after();
+          mma_kmajor(T_DP, v_a, do_a + st1 * L::kTile);
           mma_kmajor(T_S, kn_a, qn_a + st1 * L::kTile);
+          mma_commit(&bars->s_full);
         }
       }
       if (ok) mma_commit(&bars->acc_full);
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
-    const int wg = warp >> 2;               // query-column half
+    const int wg = warp >> 2;               // owns query columns [32 wg, 32 wg + 32)
     const int j = threadIdx.x & 127;        // key row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int bar_id = 1 + wg;
@@ -337,6 +345,10 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
       }
     }
+    // G_q drain: warpgroup w owns G_q columns [32 w, 32 w + 32); with D = 64 only
+    // warpgroups 0 and 1 have columns.  Staging chunks are [128 rows][32 floats]
+    // with the 128-byte swizzle (16 KB) in this step's Q^ and dO stage buffers.
+    const bool drains = wg * 32 < D;
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
       const int st = t & 1;
@@ -346,39 +358,54 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
       if (ok) {
         tc_fence_after();
-        const float2* ld = reinterpret_cast<const float2*>(smem + L::kLd + st * 1024) + wg * 64;
-        const int lim = row_min - (q0 + wg * 64);   // columns c < lim are masked on diagonal steps
-        uint8_t* ds_box = smem + L::kDs + wg * 16384;
-        // two halves of 32 query columns each, to bound register use
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[32], dpr[32];
-          tmem_ld32(tmem + lane_base + T_S + wg * 64 + half * 32, sr);
-          tmem_ld32(tmem + lane_base + T_DP + wg * 64 + half * 32, dpr);
+        const float4* ld4 = reinterpret_cast<const float4*>(smem + L::kLd + st * 1024) + wg * 16;
+        const int lim = row_min - (q0 + wg * 32);   // columns c < lim are masked on diagonal steps
+        uint8_t* ds_box = smem + L::kDs + (wg >> 1) * 16384;
+        // two groups of 16 query columns, to keep the working set small
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          uint32_t sr[16], dpr[16];
+          tmem_ld16(tmem + lane_base + T_S + wg * 32 + grp * 16, sr);
+          tmem_ld16(tmem + lane_base + T_DP + wg * 32 + grp * 16, dpr);
           tmem_wait_ld();
-          uint32_t pk[16], dk[16];
+          uint32_t pk[8], dk[8];
+          if (!diag) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int cc = half * 32 + c;
-            const float2 l0 = ld[cc], l1 = ld[cc + 1];
-            float p0 = fast_exp2(__uint_as_float(sr[c]) - l0.x);
-            float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - l1.x);
-            if (diag) {
-              p0 = cc < lim ? 0.f : p0;
-              p1 = cc + 1 < lim ? 0.f : p1;
+            for (int c = 0; c < 16; c += 2) {
+              const float4 l = ld4[grp * 8 + (c >> 1)];   // {lse2, Delta} of columns c and c + 1
+              const uint64_t a2 =
+                  f2_add(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), f2_pack(-l.x, -l.z));
+              float a0, a1;
+              f2_unpack(a2, a0, a1);
+              const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+              const uint64_t g2 =
+                  f2_add(f2_pack(__uint_as_float(dpr[c]), __uint_as_float(dpr[c + 1])), f2_pack(-l.y, -l.w));
+              float d0, d1;
+              f2_unpack(f2_mul(g2, f2_pack(p0, p1)), d0, d1);
+              pk[c >> 1] = pack_bf16x2(p0, p1);
+              dk[c >> 1] = pack_bf16x2(d0, d1);
             }
-            const float d0 = p0 * (__uint_as_float(dpr[c]) - l0.y);
-            const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l1.y);
-            pk[c >> 1] = pack_bf16x2(p0, p1);
-            dk[c >> 1] = pack_bf16x2(d0, d1);
-          }
-          // P^T of this half goes to the half's own (already read) S^T columns:
-          // query half w, 32-column part h -> columns 64w + 16h .. +16, so the
-          // two warpgroups never touch each other's columns.
-          tmem_st16(tmem + lane_base + T_S + wg * 64 + half * 16, pk);
+          } else {
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, half * 32 + c8 * 8)) =
+            for (int c = 0; c < 16; c += 2) {
+              const int cc = grp * 16 + c;
+              const float4 l = ld4[cc >> 1];
+              const float p0 = cc < lim ? 0.f : fast_exp2(__uint_as_float(sr[c]) - l.x);
+              const float p1 = cc + 1 < lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]) - l.z);
+              const float d0 = p0 * (__uint_as_float(dpr[c]) - l.y);
+              const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l.w);
+              pk[c >> 1] = pack_bf16x2(p0, p1);
+              dk[c >> 1] = pack_bf16x2(d0, d1);
+            }
+          }
+          // P^T of these 16 queries (8 packed columns) goes into this warpgroup's
+          // own S^T columns, which have been read: group 0 -> [32w, 32w+8) (its
+          // S^T group 0 is in registers), group 1 -> [32w+8, 32w+16) (S^T group 0's
+          // columns, read before).
+          tmem_st8(tmem + lane_base + T_S + wg * 32 + grp * 8, pk);
+#pragma unroll
+          for (int c8 = 0; c8 < 2; ++c8)
+            *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, (wg & 1) * 32 + grp * 16 + c8 * 8)) =
                 make_uint4(dk[4 * c8], dk[4 * c8 + 1], dk[4 * c8 + 2], dk[4 * c8 + 3]);
         }
         tmem_wait_st();
@@ -386,20 +413,26 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         fence_proxy_async_smem();
       }
       named_bar_sync(bar_id, 128);
-      if (j == 0 && ok) mbar_arrive(&bars->ds_ready);
+      if (j == 0 && ok) {
+        mbar_arrive(&bars->ds_ready);
+        if (t > 0) {
+          // The previous step's dq reduction has had this step's MMAs and
+          // softmax to read its staging; once it has, that Q^/dO stage goes back
+          // to the producer (the next load still has this step's products to land).
+          tma_store_wait_read();
+          mbar_arrive(&bars->q_empty[st ^ 1]);
+        }
+      }
 
       // Drain G_q (TMEM lane = query row of this step) into the fp32 accumulator:
       // TMEM -> registers (then the dP^T/G_q columns are free again), registers ->
-      // this step's Q^/dO stage (idle once dq_full has fired) as 128-byte-swizzled
-      // [128 rows][32 floats] chunks, then TMA bulk reduce-adds.  The stage goes
-      // back to the producer when the bulk engine has read it.
+      // this step's Q^/dO stage (idle once mma_done has fired), then a TMA bulk
+      // reduce-add.  The stage goes back to the producer at the next step.
       ok = warp_wait(&bars->dq_full, t & 1, ok, p.status, kErrDqFull);
-      constexpr int kChunks = D / 64;  // 32-column chunks per warpgroup
-      uint32_t gq[kChunks][32];
-      if (ok) {
+      uint32_t gq[32];
+      if (ok && drains) {
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) tmem_ld32(tmem + lane_base + T_DP + (wg * kChunks + c) * 32, gq[c]);
+        tmem_ld32(tmem + lane_base + T_DP + wg * 32, gq);
         tmem_wait_ld();
         tc_fence_before();
       }
@@ -407,32 +440,31 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       if (j == 0 && ok) mbar_arrive(&bars->dq_drained);
       // the stage is staging space only once the dK~ and dV products have read it
       ok = warp_wait(&bars->mma_done, t & 1, ok, p.status, kErrMmaDone);
-      if (ok) {
-        uint8_t* stage = smem + (wg == 0 ? L::kQn : L::kDo) + st * L::kTile;
+      // chunk wg: the first D/64 chunks fill this step's Q^ stage, the rest its dO stage
+      constexpr int kChunksPerBuffer = D / 64;
+      uint8_t* chunk = wg < kChunksPerBuffer ? smem + L::kQn + st * L::kTile + wg * 16384
+                                             : smem + L::kDo + st * L::kTile + (wg - kChunksPerBuffer) * 16384;
+      if (ok && drains) {
+        uint8_t* row = chunk + j * 128;
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-          uint8_t* chunk = stage + c * 16384 + j * 128;
-#pragma unroll
-          for (int piece = 0; piece < 8; ++piece)
-            *reinterpret_cast<uint4*>(chunk + (((piece ^ (j & 7)) & 7) << 4)) =
-                make_uint4(gq[c][4 * piece], gq[c][4 * piece + 1], gq[c][4 * piece + 2], gq[c][4 * piece + 3]);
-        }
+        for (int piece = 0; piece < 8; ++piece)
+          *reinterpret_cast<uint4*>(row + (((piece ^ (j & 7)) & 7) << 4)) =
+              make_uint4(gq[4 * piece], gq[4 * piece + 1], gq[4 * piece + 2], gq[4 * piece + 3]);
         fence_proxy_async_smem();
       }
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) {
-        const uint8_t* stage = smem + (wg == 0 ? L::kQn : L::kDo) + st * L::kTile;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-          tma_reduce_add_4d(&tm_dq, stage + c * 16384, (wg * kChunks + c) * 32, h, q0, b);
-        tma_store_commit();
-        tma_store_wait_read();
-        mbar_arrive(&bars->q_empty[st]);
+        if (drains) tma_reduce_add_4d(&tm_dq, chunk, wg * 32, h, q0, b);
+        tma_store_commit();   // (an empty group when nothing was issued); released next step
       }
     }
-    // every bulk reduction complete before the stage buffers are reused below
-    if (j == 0) tma_store_wait_all();
-    named_bar_sync(3, 256);
+    // every bulk reduction complete (and the last stage released) before the
+    // stage buffers are reused below
+    if (j == 0) {
+      tma_store_wait_all();
+      if (ok && n_steps > 0) mbar_arrive(&bars->q_empty[(n_steps - 1) & 1]);
+    }
+    named_bar_sync(5, 128 * kComputeWarpgroups);
 
     // ---------------------------------------------------------- epilogue
     ok = warp_wait(&bars->acc_full, 0, ok && n_steps > 0, p.status, kErrAcc);
@@ -459,7 +491,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
           }
         }
-      } else {
+      } else if (wg == 1) {
         // dk through the RMSNorm Jacobian: with k^ = k r_k and g = gamma_k * dk~
         // (= G_k / log2 e):  dk = r_k (g - k^ mean(g k^)).  The raw key row is
         // read from global memory (the shared tile holds K^).
@@ -533,7 +565,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -28,7 +28,7 @@ library_path = os.path.join(_HERE, "libmagi_bca.so")
 
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
-                    "magi_bca_bwd_noalloc", "magi_bca_last_error_detail"]
+                    "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule"]
 
 
 class MagiBcaError(RuntimeError):
@@ -79,6 +79,8 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_fwd_schedule.restype = ctypes.c_int64
     lib.magi_bca_last_error_detail.argtypes = []
     lib.magi_bca_last_error_detail.restype = ctypes.c_char_p
+    lib.magi_bca_bwd_schedule.argtypes = [i32p, i32p, dp, ctypes.c_int32, i32p, ctypes.c_int64]
+    lib.magi_bca_bwd_schedule.restype = ctypes.c_int64
     lib.magi_bca_version.argtypes = []
     lib.magi_bca_version.restype = ctypes.c_char_p
     _lib = lib
@@ -226,7 +228,7 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
     For callers that cannot allocate device memory or hand the library a
     workspace (a pooled allocator owns the GPU's memory, a plugin hook must
     not allocate, or cudaMalloc's implicit synchronisation is unaffordable).
-    Every output is passed in by the caller; the library uses its own 64 MiB
+    Every output is passed in by the caller; the library uses its own 96 MiB
     device array as workspace, so calls must not overlap on the GPU.  Problems
     too large for that array raise MagiBcaError (status -4)."""
     _check_bf16("q", q)
@@ -266,5 +268,20 @@ def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, hea
         raise MagiBcaError(int(n), "magi_bca_fwd_schedule")
     buf = np.zeros((max(n, 1), 8), dtype=np.int32)
     n2 = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), _i32p(buf), n)
+    assert n2 == n
+    return buf[:n]
+
+
+def magi_bca_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
+                          num_sms=148) -> np.ndarray:
+    """Host-only: the backward's work units as an int32 array [n_units, 8]."""
+    qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
+    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1)
+    lib = library()
+    n = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, None, 0)
+    if n < 0:
+        raise MagiBcaError(int(n), "magi_bca_bwd_schedule")
+    buf = np.zeros((max(n, 1), 8), dtype=np.int32)
+    n2 = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, _i32p(buf), n)
     assert n2 == n
     return buf[:n]

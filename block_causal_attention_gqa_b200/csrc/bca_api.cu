@@ -123,7 +123,9 @@ int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, c
     *out = it->second;
     return MAGI_BCA_OK;
   }
-  std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d);
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d, sms);
   ScheduleEntry e;
   e.n_units = static_cast<int>(units.size() / kUnitInts);
   std::vector<int32_t> blob = units;
@@ -242,6 +244,20 @@ int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
   return n;
 }
 
+int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                              const magi_bca_dims* dims, int32_t num_sms, int32_t* units, int64_t capacity) {
+  int st = validate_dims(dims);
+  if (st != MAGI_BCA_OK) return st;
+  st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, *dims);
+  if (st != MAGI_BCA_OK) return st;
+  if ((capacity > 0 && units == nullptr) || num_sms <= 0) return MAGI_BCA_INVALID_ARG;
+  std::vector<int32_t> s = build_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, *dims, num_sms);
+  const int64_t n = (int64_t)(s.size() / kUnitInts);
+  const int64_t w = n < capacity ? n : capacity;
+  if (w > 0) std::memcpy(units, s.data(), (size_t)w * kUnitInts * sizeof(int32_t));
+  return n;
+}
+
 int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
                  const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets, const float* gamma_q,
                  const float* gamma_k, magi_bca_bf16* out, float* lse, const magi_bca_dims* dims, void* stream) {
@@ -344,6 +360,8 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.kn = reinterpret_cast<uint16_t*>(w + ws.kn);
   p.ld = reinterpret_cast<float*>(w + ws.ld);
   p.dqacc = reinterpret_cast<float*>(w + ws.dqacc);
+  p.dvacc = reinterpret_cast<float*>(w + ws.dvacc);
+  p.dkacc = reinterpret_cast<float*>(w + ws.dkacc);
   p.batch = d.batch;
   p.seqlen_q = d.seqlen_q;
   p.seqlen_kv = d.seqlen_kv;
@@ -354,14 +372,17 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = ds->status;
-  CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
+  CUtensorMap t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk;
   if (make_map_f32(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_map_f32(&t_dv, p.dvacc, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_map_f32(&t_dk, p.dkacc, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_k, p.kn, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("backward launch", e);
 }
 

@@ -7,7 +7,7 @@
 // order (the helpers in bca_norm.cuh fix the rounding points for both passes).
 //
 // Three launches on the caller's stream:
-//   1. prep      one thread per query row: Q^ into the workspace; Delta =
+//   1. prep      one warp per query row: Q^ into the workspace; Delta =
 //                rowsum(dO * O); {lse*log2(e), Delta} pairs in a 128-padded
 //                layout; zero the fp32 dq accumulator and dgamma; then K^ into
 //                the workspace (bca_knorm_kernel, one warp per key row).
@@ -21,10 +21,10 @@
 //                  G_k += dS'^T Q^      -> gamma_k * dk~ = G_k / (r_k log2 e)
 //                  G_q  = dS' K         -> dq~ = scale gamma_k * G_q, drained with
 //                                          vector red.add into the fp32 accumulator
-//                and finally writes dv, and dk through the RMSNorm Jacobian (plus
-//                this tile's share of gamma_k * dgamma_k).
-//   3. finalize  one warp per query row: dq through the RMSNorm Jacobian, dgamma_q,
-//                and dgamma_k = (gamma_k * dgamma_k) / gamma_k.
+//                and finally adds dV and G_k into fp32 accumulators (long query
+//                ranges are split into pieces, so several CTAs may add to one kv tile).
+//   3. finalize  one warp per row: dq, dk through the RMSNorm Jacobian, dv, and
+//                dgamma_q, dgamma_k.
 // These are the five matrix products of the Flash-Attention backward (2.5x the
 // forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
 // query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.
@@ -116,6 +116,8 @@ struct RowIO {
 
 template <int D>
 __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
+  using IO = RowIO<D>;
+  constexpr int E = IO::E;
   __shared__ float qscale[D];
   for (int d = threadIdx.x; d < D; d += blockDim.x) qscale[d] = qscale_of(p.gamma_q, p.gamma_k, p.scale_log2, d);
   if (blockIdx.x == 0 && threadIdx.x < D) {
@@ -123,36 +125,37 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
     if (p.dgamma_k) p.dgamma_k[threadIdx.x] = 0.f;
   }
   __syncthreads();
+  const int lane = threadIdx.x & 31;
   const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
-  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < n_q; r += (int64_t)gridDim.x * blockDim.x) {
-    // the forward's query operand, bit for bit (same helpers, same order)
-    const uint16_t* qrow = p.q + r * D;
-    const float rq = rms_inv<D>(row_sumsq_linear<D>(qrow), p.eps);
-    uint16_t* qh = p.qn + r * D;
-    float dot = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      *reinterpret_cast<uint4*>(qh + c * 8) = fold_q_chunk(*reinterpret_cast<const uint4*>(qrow + c * 8), rq, qscale, c * 8);
-      const uint4 o = *reinterpret_cast<const uint4*>(p.out + r * D + c * 8);
-      const uint4 g = *reinterpret_cast<const uint4*>(p.dout + r * D + c * 8);
-      const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  // one warp per query row, coalesced; the sum of squares uses the order that
+  // the forward's prologue reproduces, so Q^ is bit-identical to the forward's
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < n_q; r += warps) {
+    float x[E], o[E], g[E];
+    IO::load_bf16(p.q + r * D, lane, x);
+    IO::load_bf16(p.out + r * D, lane, o);
+    IO::load_bf16(p.dout + r * D, lane, g);
+    const float rq = rms_inv<D>(warp_sumsq_row<E>(x), p.eps);
+    float qh[E];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        dot = fmaf(bf16_lo(ow[i]), bf16_lo(gw[i]), dot);
-        dot = fmaf(bf16_hi(ow[i]), bf16_hi(gw[i]), dot);
-      }
-      *reinterpret_cast<float4*>(p.dqacc + r * D + c * 8) = make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(p.dqacc + r * D + c * 8 + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < E; ++e) qh[e] = x[e] * rq * qscale[lane * E + e];
+    IO::store_bf16(p.qn + r * D, lane, qh);
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) dot = fmaf(o[e], g[e], dot);
+    dot = warp_sum(dot);
+    IO::store_zero_f32(p.dqacc + r * D, lane);
+    if (lane == 0) {
+      const int h = (int)(r % p.heads_q);
+      const int64_t bs = r / p.heads_q;
+      const int s = (int)(bs % p.seqlen_q);
+      const int b = (int)(bs / p.seqlen_q);
+      const int64_t bh = (int64_t)b * p.heads_q + h;
+      float2 v;
+      v.x = __ldg(p.lse + bh * p.seqlen_q + s) * kLog2e;
+      v.y = dot;
+      *reinterpret_cast<float2*>(p.ld + (bh * p.seqlen_q_pad + s) * 2) = v;
     }
-    const int h = (int)(r % p.heads_q);
-    const int64_t bs = r / p.heads_q;
-    const int s = (int)(bs % p.seqlen_q);
-    const int b = (int)(bs / p.seqlen_q);
-    const int64_t bh = (int64_t)b * p.heads_q + h;
-    float2 v;
-    v.x = __ldg(p.lse + bh * p.seqlen_q + s) * kLog2e;
-    v.y = dot;
-    *reinterpret_cast<float2*>(p.ld + (bh * p.seqlen_q_pad + s) * 2) = v;
   }
 }
 
@@ -180,7 +183,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p, const int smem_alloc) {
+                    const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dv,
+                    const __grid_constant__ CUtensorMap tm_dk, const BwdParams p, const int smem_alloc) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
@@ -222,6 +226,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tma_prefetch_desc(&tm_qn);
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
+    tma_prefetch_desc(&tm_dv);
+    tma_prefetch_desc(&tm_dk);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -467,99 +473,34 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     named_bar_sync(5, 128 * kComputeWarpgroups);
 
     // ---------------------------------------------------------- epilogue
+    // dV and G_k of this piece (fp32 in TMEM) are added into the fp32
+    // accumulators: warpgroup w stages columns [32w, 32w+32) of each into the
+    // idle stage buffers (dV -> Q^ stages, G_k -> dO stages) and issues two
+    // bulk reduce-adds.  bca_bwd_finalize_kernel turns the sums into dv and dk.
     ok = warp_wait(&bars->acc_full, 0, ok && n_steps > 0, p.status, kErrAcc);
-    const int key = n0 + j;
-    if (ok) {
+    if (ok && drains) {
       tc_fence_after();
-      if (wg == 0) {
-        // dV -> bf16
-        uint16_t* dst = p.dv + (((size_t)b * p.seqlen_kv + key) * p.heads_kv + hk) * D;
+      uint32_t rv[32], rk32[32];
+      tmem_ld32(tmem + lane_base + T_DV + wg * 32, rv);
+      tmem_ld32(tmem + lane_base + T_DK + wg * 32, rk32);
+      tmem_wait_ld();
+      uint8_t* sv = smem + L::kQn + wg * 16384 + j * 128;
+      uint8_t* sk = smem + L::kDo + wg * 16384 + j * 128;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + T_DV + c, r);
-          tmem_wait_ld();
-          if (key < p.seqlen_kv) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-              w.y = pack_bf16x2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-              w.z = pack_bf16x2(__uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
-              w.w = pack_bf16x2(__uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
-              *reinterpret_cast<uint4*>(dst + c + i) = w;
-            }
-          }
-        }
-      } else if (wg == 1) {
-        // dk through the RMSNorm Jacobian: with k^ = k r_k and g = gamma_k * dk~
-        // (= G_k / log2 e):  dk = r_k (g - k^ mean(g k^)).  The raw key row is
-        // read from global memory (the shared tile holds K^).
-        // This tile's share of gamma_k * dgamma_k is sum_keys g * k^.
-        float* red = reinterpret_cast<float*>(smem + L::kQn);  // [128][D + 1]; stage buffers are idle now
-        const bool live = key < p.seqlen_kv;
-        const uint16_t* krow = p.k + (((size_t)b * p.seqlen_kv + (live ? key : 0)) * p.heads_kv + hk) * D;
-        const float rk = rms_inv<D>(row_sumsq_linear<D>(krow), p.eps);
-        constexpr float gscale = 1.0f / kLog2e;
-        float dot = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + T_DK + c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(krow + c + i);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float k0 = bf16_lo(ww[e]) * rk, k1 = bf16_hi(ww[e]) * rk;
-              const float g0 = __uint_as_float(r[i + 2 * e]) * gscale;
-              const float g1 = __uint_as_float(r[i + 2 * e + 1]) * gscale;
-              dot = fmaf(g0, k0, dot);
-              dot = fmaf(g1, k1, dot);
-              red[j * (D + 1) + c + i + 2 * e] = live ? g0 * k0 : 0.f;
-              red[j * (D + 1) + c + i + 2 * e + 1] = live ? g1 * k1 : 0.f;
-            }
-          }
-        }
-        const float mean_dot = dot * (1.0f / D);
-        uint16_t* dst = p.dk + (((size_t)b * p.seqlen_kv + key) * p.heads_kv + hk) * D;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + T_DK + c, r);
-          tmem_wait_ld();
-          if (live) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              const uint4 w = *reinterpret_cast<const uint4*>(krow + c + i);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-              float o[8];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float k0 = bf16_lo(ww[e]) * rk, k1 = bf16_hi(ww[e]) * rk;
-                o[2 * e] = rk * (__uint_as_float(r[i + 2 * e]) * gscale - k0 * mean_dot);
-                o[2 * e + 1] = rk * (__uint_as_float(r[i + 2 * e + 1]) * gscale - k1 * mean_dot);
-              }
-              uint4 ov;
-              ov.x = pack_bf16x2(o[0], o[1]);
-              ov.y = pack_bf16x2(o[2], o[3]);
-              ov.z = pack_bf16x2(o[4], o[5]);
-              ov.w = pack_bf16x2(o[6], o[7]);
-              *reinterpret_cast<uint4*>(dst + c + i) = ov;
-            }
-          }
-        }
-        if (p.dgamma_k != nullptr) {
-          named_bar_sync(bar_id, 128);
-          if (j < D) {
-            float acc = 0.f;
-            for (int r = 0; r < 128; ++r) acc += red[r * (D + 1) + j];
-            atomicAdd(p.dgamma_k + j, acc);
-          }
-        }
+      for (int piece = 0; piece < 8; ++piece) {
+        const uint32_t off = ((piece ^ (j & 7)) & 7) << 4;
+        *reinterpret_cast<uint4*>(sv + off) = make_uint4(rv[4 * piece], rv[4 * piece + 1], rv[4 * piece + 2], rv[4 * piece + 3]);
+        *reinterpret_cast<uint4*>(sk + off) =
+            make_uint4(rk32[4 * piece], rk32[4 * piece + 1], rk32[4 * piece + 2], rk32[4 * piece + 3]);
       }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(bar_id, 128);
+    if (j == 0 && ok && drains) {
+      tma_reduce_add_4d(&tm_dv, smem + L::kQn + wg * 16384, wg * 32, hk, n0, b);
+      tma_reduce_add_4d(&tm_dk, smem + L::kDo + wg * 16384, wg * 32, hk, n0, b);
+      tma_store_commit();
+      tma_store_wait_all();
     }
   }
 
@@ -572,66 +513,90 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 }
 
 // ------------------------------------------------------------------ finalize
+// One warp per row.  Query rows: dq~ = scale gamma_k G_q, dq through the
+// RMSNorm Jacobian, dgamma_q += dq~ q^.  Key rows: dv = bf16(dV), gamma_k dk~ =
+// G_k / log2(e), dk through the Jacobian, dgamma_k += dk~ k^.  With r = rsqrt
+// (mean x^2 + eps), x^ = x r and g = gamma dx~:  dx = r (g - x^ mean(g x^)).
 template <int D>
 __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p) {
   using IO = RowIO<D>;
   constexpr int E = IO::E;
-  __shared__ float red[8][D];
+  __shared__ float red[2][8][D];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
+  const int64_t n_k = (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
   const int64_t warps = (int64_t)gridDim.x * 8;
-  float gacc[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) gacc[e] = 0.f;
-  float gm[E], gk[E];
+  float gacc_q[E], gacc_k[E], gm[E], gk[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
+    gacc_q[e] = 0.f;
+    gacc_k[e] = 0.f;
     gm[e] = __ldg(p.gamma_q + lane * E + e);
-    gk[e] = __ldg(p.gamma_k + lane * E + e) * p.scale;   // dq~ = scale gamma_k G_q
+    gk[e] = __ldg(p.gamma_k + lane * E + e);
   }
-  if (blockIdx.x == 0 && p.dgamma_k != nullptr && threadIdx.x < D)
-    p.dgamma_k[threadIdx.x] = p.dgamma_k[threadIdx.x] / __ldg(p.gamma_k + threadIdx.x);
-  for (int64_t r = (int64_t)blockIdx.x * 8 + wid; r < n_q; r += warps) {
-    float x[E], dqt[E];
-    IO::load_bf16(p.q + r * D, lane, x);
-    IO::load_f32(p.dqacc + r * D, lane, dqt);
+  for (int64_t rr = (int64_t)blockIdx.x * 8 + wid; rr < n_q + n_k; rr += warps) {
+    const bool is_q = rr < n_q;
+    const int64_t r = is_q ? rr : rr - n_q;
+    float x[E], g[E], dqt[E];
+    IO::load_bf16((is_q ? p.q : p.k) + r * D, lane, x);
+    IO::load_f32((is_q ? p.dqacc : p.dkacc) + r * D, lane, g);
+    // g = gamma * dx~   (for query rows dq~ = scale gamma_k G_q is kept for dgamma_q)
 #pragma unroll
-    for (int e = 0; e < E; ++e) dqt[e] *= gk[e];
+    for (int e = 0; e < E; ++e) {
+      dqt[e] = g[e] * gk[e] * p.scale;
+      g[e] = is_q ? dqt[e] * gm[e] : g[e] * (1.0f / kLog2e);
+    }
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
-    const float rq = rsqrtf(warp_sum(ss) * (1.0f / D) + p.eps);
+    const float rinv = rsqrtf(warp_sum(ss) * (1.0f / D) + p.eps);
     float dot = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      x[e] *= rq;                                   // x^
-      dot = fmaf(gm[e] * dqt[e], x[e], dot);
-      gacc[e] = fmaf(dqt[e], x[e], gacc[e]);
+      x[e] *= rinv;   // x^
+      dot = fmaf(g[e], x[e], dot);
     }
     const float mean_dot = warp_sum(dot) * (1.0f / D);
     float o[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) o[e] = rq * (gm[e] * dqt[e] - x[e] * mean_dot);
-    IO::store_bf16(p.dq + r * D, lane, o);
-  }
-  if (p.dgamma_q != nullptr) {
+    for (int e = 0; e < E; ++e) o[e] = rinv * (g[e] - x[e] * mean_dot);
+    if (is_q) {
+      IO::store_bf16(p.dq + r * D, lane, o);
 #pragma unroll
-    for (int e = 0; e < E; ++e) red[wid][lane * E + e] = gacc[e];
+      for (int e = 0; e < E; ++e) gacc_q[e] = fmaf(dqt[e], x[e], gacc_q[e]);
+    } else {
+      IO::store_bf16(p.dk + r * D, lane, o);
+      float dvv[E];
+      IO::load_f32(p.dvacc + r * D, lane, dvv);
+      IO::store_bf16(p.dv + r * D, lane, dvv);
+#pragma unroll
+      for (int e = 0; e < E; ++e) gacc_k[e] = fmaf(g[e] / gk[e], x[e], gacc_k[e]);
+    }
+  }
+  if (p.dgamma_q != nullptr || p.dgamma_k != nullptr) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      red[0][wid][lane * E + e] = gacc_q[e];
+      red[1][wid][lane * E + e] = gacc_k[e];
+    }
     __syncthreads();
     if (threadIdx.x < D) {
-      float acc = 0.f;
+      float aq = 0.f, ak = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) acc += red[w][threadIdx.x];
-      atomicAdd(p.dgamma_q + threadIdx.x, acc);
+      for (int w = 0; w < 8; ++w) {
+        aq += red[0][w][threadIdx.x];
+        ak += red[1][w][threadIdx.x];
+      }
+      if (p.dgamma_q != nullptr) atomicAdd(p.dgamma_q + threadIdx.x, aq);
+      if (p.dgamma_k != nullptr) atomicAdd(p.dgamma_k + threadIdx.x, ak);
     }
   }
 }
 
-
 template <int D>
 cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                         const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int n_units,
-                         cudaStream_t stream) {
+                         const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
+                         const CUtensorMap& t_dk, const BwdParams& p, int n_units, cudaStream_t stream) {
   using L = BwdLayout<D>;
   static uint64_t configured = 0;
   int dev = 0;
@@ -650,24 +615,29 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q;
-  const int prep_blocks = (int)std::min<int64_t>((rows + 255) / 256, (int64_t)sms * 8);
+  const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 16);
   if (p.seqlen_q_pad != p.seqlen_q) {
     // padding entries of the {lse, Delta} pairs are read by full-tile loads
     e = cudaMemsetAsync(p.ld, 0, (size_t)p.batch * p.heads_q * p.seqlen_q_pad * 2 * sizeof(float), stream);
     if (e != cudaSuccess) return e;
   }
+  // dV and G_k are sums over the pieces of each kv tile
+  e = cudaMemsetAsync(p.dvacc, 0, (size_t)p.batch * p.seqlen_kv * p.heads_kv * D * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(p.dkacc, 0, (size_t)p.batch * p.seqlen_kv * p.heads_kv * D * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
   bca_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_knorm(p.k, p.kn, (int64_t)p.batch * p.seqlen_kv * p.heads_kv, D, p.eps, stream);
   if (e != cudaSuccess) return e;
   if (n_units > 0) {
-    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, p, alloc);
+    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, alloc);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const int64_t qrows = (int64_t)p.batch * p.seqlen_q * p.heads_q;
-  const int fin_blocks = (int)std::min<int64_t>((qrows + 7) / 8, (int64_t)sms * 8);
+  const int64_t frows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
+  const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * 8);
   bca_bwd_finalize_kernel<D><<<fin_blocks, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
@@ -682,15 +652,17 @@ BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D
   w.kn = w.qn + up((size_t)B * Sq * Hq * D * 2);
   w.ld = w.kn + up((size_t)B * Skv * Hkv * D * 2);
   w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 2 * 4);
-  w.total = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
+  w.dvacc = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
+  w.dkacc = w.dvacc + up((size_t)B * Skv * Hkv * D * 4);
+  w.total = w.dkacc + up((size_t)B * Skv * Hkv * D * 4);
   return w;
 }
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int head_dim, int n_units,
-                       cudaStream_t stream) {
-  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, t_dq, p, n_units, stream);
-  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, t_dq, p, n_units, stream);
+                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
+                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream) {
+  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, stream);
+  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, stream);
 }
 
 }  // namespace magi

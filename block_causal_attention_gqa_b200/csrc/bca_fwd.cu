@@ -259,7 +259,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // Q prologue: RMSNorm the row and fold gains, scale and log2(e) into it.
       ok = warp_wait(&bars->q_full[s], 0, ok, p.status, kErrQ);
       if (ok) {
-        const float rq = rms_inv<D>(row_sumsq_swizzled<D>(q_tile, r), p.eps);
+        const float rq = rms_inv<D>(row_sumsq_swizzled_warp_order<D>(q_tile, r), p.eps);
 #pragma unroll
         for (int box = 0; box < D / 64; ++box) {
 #pragma unroll

@@ -49,6 +49,8 @@ struct BwdParams {
   uint16_t* kn;               // forward key operand K^ = bf16(k r_k) [B, Skv, Hkv, D]
   float* ld;                  // {lse * log2(e), Delta} pairs [B, Hq, Sq_pad, 2]
   float* dqacc;               // fp32 G_q accumulator          [B, Sq, Hq, D]
+  float* dvacc;               // fp32 dV accumulator           [B, Skv, Hkv, D]
+  float* dkacc;               // fp32 G_k accumulator          [B, Skv, Hkv, D]
   int batch, seqlen_q, seqlen_kv, heads_q, heads_kv, seqlen_q_pad;
   float scale;                // softmax scale
   float scale_log2;           // softmax scale * log2(e)
@@ -57,13 +59,13 @@ struct BwdParams {
 };
 
 struct BwdWorkspace {
-  size_t qn, kn, ld, dqacc, total;  // byte offsets and total size
+  size_t qn, kn, ld, dqacc, dvacc, dkacc, total;  // byte offsets and total size
 };
 BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D);
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
-                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const BwdParams& p, int head_dim,
-                       int n_units, cudaStream_t stream);
+                       const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
+                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream);
 int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 
 // K^ = bf16(k rsqrt(mean k^2 + eps)) for `rows` rows of head_dim features.

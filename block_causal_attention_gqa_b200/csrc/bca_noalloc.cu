@@ -9,7 +9,7 @@
 // the backward's workspace and its tile schedule live in one file-scope
 // device array, so a call allocates nothing.
 //
-// The array is kNoallocScratchBytes (64 MiB) per device.  Every GPU that loads
+// The array is kNoallocScratchBytes (96 MiB) per device.  Every GPU that loads
 // this library holds it until the process exits.  Problems whose workspace
 // plus schedule do not fit are rejected with MAGI_BCA_WORKSPACE_TOO_SMALL.
 //
@@ -33,7 +33,7 @@
 
 namespace magi {
 
-constexpr size_t kNoallocScratchBytes = size_t(64) << 20;
+constexpr size_t kNoallocScratchBytes = size_t(96) << 20;
 
 namespace {
 
@@ -86,7 +86,12 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
 
   // Layout inside the array: [workspace][schedule units][q offsets][kv offsets].
   const BwdWorkspace ws = bwd_workspace_layout(d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim);
-  std::vector<int32_t> blob = build_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, d);
+  int sms = 148;
+  {
+    int dev0 = 0;
+    if (cudaGetDevice(&dev0) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev0);
+  }
+  std::vector<int32_t> blob = build_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, d, sms);
   const int n_units = static_cast<int>(blob.size() / kUnitInts);
   blob.insert(blob.end(), q_chunk_offsets, q_chunk_offsets + d.n_q_chunks + 1);
   blob.insert(blob.end(), kv_chunk_offsets, kv_chunk_offsets + d.n_kv_chunks + 1);
@@ -132,6 +137,8 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.kn = reinterpret_cast<uint16_t*>(scratch + ws.kn);
   p.ld = reinterpret_cast<float*>(scratch + ws.ld);
   p.dqacc = reinterpret_cast<float*>(scratch + ws.dqacc);
+  p.dvacc = reinterpret_cast<float*>(scratch + ws.dvacc);
+  p.dkacc = reinterpret_cast<float*>(scratch + ws.dkacc);
   p.batch = d.batch;
   p.seqlen_q = d.seqlen_q;
   p.seqlen_kv = d.seqlen_kv;
@@ -142,13 +149,15 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = status;
-  CUtensorMap t_k, t_v, t_qn, t_do, t_dq;
+  CUtensorMap t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk;
   if (make_tensor_map_f32_dq(&t_dq, p.dqacc, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
+      make_tensor_map_f32_dq(&t_dv, p.dvacc, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
+      make_tensor_map_f32_dq(&t_dk, p.dkacc, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_k, p.kn, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_v, v, d.batch, d.seqlen_kv, d.heads_kv, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  const cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, p, d.head_dim, n_units, s);
+  const cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, n_units, s);
   return e == cudaSuccess ? MAGI_BCA_OK : record_cuda_failure("allocation-free backward launch", e);
 }

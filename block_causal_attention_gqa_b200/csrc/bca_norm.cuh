@@ -48,6 +48,45 @@ __device__ __forceinline__ float row_sumsq_linear(const uint16_t* row) {
   return acc;
 }
 
+// The same sum in the order a warp computes it when lane l holds features
+// [l*E, l*E + E) (E = D/32): per-lane fmaf chains, then an xor butterfly
+// (offsets 16, 8, 4, 2, 1).  Floating-point addition is commutative, so every
+// lane of the warp ends with this value; warp_sumsq_row below is the warp side.
+template <int D>
+__device__ __forceinline__ float row_sumsq_swizzled_warp_order(const uint8_t* tile, int row) {
+  constexpr int E = D / 32;
+  float part[32];
+#pragma unroll
+  for (int box = 0; box < D / 64; ++box)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(tile + box * 16384 + sm100::sw128_offset(row, c * 8));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float x = (k & 1) ? bf16_hi(w[k >> 1]) : bf16_lo(w[k >> 1]);
+        const int d = box * 64 + c * 8 + k;
+        part[d / E] = (d % E == 0) ? x * x : fmaf(x, x, part[d / E]);
+      }
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int i = 0; i < o; ++i) part[i] = part[i] + part[i + o];
+  return part[0];
+}
+
+// Warp side of the above: lane holds x[0..E) of the row; returns the sum in every lane.
+template <int E>
+__device__ __forceinline__ float warp_sumsq_row(const float (&x)[E]) {
+  float s = x[0] * x[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) s = fmaf(x[e], x[e], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s = s + __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
 // 1 / RMS of a row from its sum of squares.
 template <int D>
 __device__ __forceinline__ float rms_inv(float sumsq, float eps) {

@@ -111,7 +111,7 @@ std::vector<int32_t> build_fwd_schedule(const int32_t* qo, const int32_t* ko, co
   return out;
 }
 
-std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d) {
+std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d, int num_sms) {
   const int n_qt = (d.seqlen_q + kBlockM - 1) / kBlockM;
   const int n_kt = (d.seqlen_kv + kBlockN - 1) / kBlockN;
   std::vector<int> tile_lo(n_qt);  // smallest visible end among the tile's rows
@@ -140,6 +140,24 @@ std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, co
     for (int b = 0; b < d.batch; ++b)
       for (int hk = 0; hk < d.heads_kv; ++hk) units.push_back({b, hk, n0, qb, n_qt, nd});
   }
+  // Split long query ranges so every SM gets about two pieces of similar size
+  // (pieces of one kv tile add their dK/dV partials in the fp32 accumulators).
+  int64_t visits = 0;
+  for (const Unit& u : units) visits += u.qe - u.qb;
+  const int64_t cap = std::max<int64_t>(2, (visits + 2 * num_sms - 1) / (2 * (int64_t)std::max(num_sms, 1)));
+  std::vector<Unit> pieces;
+  pieces.reserve(units.size());
+  for (const Unit& u : units) {
+    const int len = u.qe - u.qb;
+    const int n_pieces = (int)((len + cap - 1) / cap);
+    const int step = (len + n_pieces - 1) / n_pieces;
+    for (int qs = u.qb; qs < u.qe; qs += step) {
+      const int qe = std::min(qs + step, u.qe);
+      const int nd = std::max(0, std::min(qe, u.qb + u.nd) - qs);   // diagonal tiles come first
+      pieces.push_back({u.b, u.hk, u.n0, qs, qe, nd});
+    }
+  }
+  units.swap(pieces);
   std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
     const int ca = a.qe - a.qb, cb = b.qe - b.qb;
     if (ca != cb) return ca > cb;

@@ -113,7 +113,7 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
 
 /* Backward that allocates nothing.  Same arguments and results as
  * magi_bca_bwd, without the workspace: the workspace and the tile schedule live
- * in a 64 MiB array that the library keeps in every GPU's memory from load
+ * in a 96 MiB array that the library keeps in every GPU's memory from load
  * until exit.  It is for callers that cannot allocate or pass device memory,
  * e.g. processes whose GPU memory is owned up front by a pooled allocator,
  * plugin hooks that must not allocate, or loops that cannot take
@@ -163,6 +163,17 @@ int magi_bca_last_device_status(void);
  * only `capacity` units are written), or a negative status. */
 int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
                               const magi_bca_dims* dims, int32_t* units, int64_t capacity);
+
+/* Host-only view of the backward schedule (no device needed).  A unit is one
+ * 128-key tile of one (batch, kv head) and a contiguous range of the query
+ * tiles that see it; long ranges are split so that `num_sms` SMs get about two
+ * units each.  Per unit 8 int32:
+ *   {batch, kv_head, n0 (first key), q_tile_begin, q_tile_end,
+ *    n_diag (the first n_diag query tiles of the range need the mask), 0, 0}
+ * in launch order (longest first).  Returns the number of units (writing at
+ * most `capacity`), or a negative status. */
+int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                              const magi_bca_dims* dims, int32_t num_sms, int32_t* units, int64_t capacity);
 
 /* Library version string. */
 const char* magi_bca_version(void);

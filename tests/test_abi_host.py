@@ -197,3 +197,52 @@ def test_workload_shapes():
     assert (w.seqlen_q, w.heads_q, w.heads_kv, w.head_dim) == (46080, 24, 8, 128)
     w = workloads.workload("stream4of16")
     assert (w.batch, w.seqlen_q, w.seqlen_kv) == (2, 23040, 92160)
+
+
+def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148):
+    qo, ko = _offs(q_lens), _offs(kv_lens)
+    Sq, Skv = int(qo[-1]), int(ko[-1])
+    units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms)
+    ends = row_ends(qo, ko, Sq)
+    n_qt, n_kt = -(-Sq // 128), -(-Skv // 128)
+    cover = np.zeros((B, Hkv, n_kt, n_qt), np.int64)
+    lengths = []
+    for b, hk, n0, qb, qe, nd, _, _ in units:
+        assert n0 % 128 == 0 and 0 <= qb < qe <= n_qt and 0 <= nd <= qe - qb
+        cover[b, hk, n0 // 128, qb:qe] += 1
+        n_end = min(n0 + 128, Skv)
+        for t in range(qb, qe):
+            rows = ends[t * 128:min(t * 128 + 128, Sq)]
+            sees = rows > n0                          # row sees some key of the tile
+            assert sees.any()
+            needs_mask = rows.min() < n_end
+            assert needs_mask == (t - qb < nd), (t, qb, nd)
+        lengths.append(qe - qb)
+    # every (kv tile, query tile) pair where some query sees some key: exactly once
+    for kt in range(n_kt):
+        for t in range(n_qt):
+            want = int((ends[t * 128:min(t * 128 + 128, Sq)] > kt * 128).any())
+            assert (cover[:, :, kt, t] == want).all(), (kt, t)
+    assert all(a >= b for a, b in zip(lengths, lengths[1:]))
+    return units
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,B,Hq,Hkv", [
+    ([64, 64], [64, 64], 1, 2, 1),
+    ([1024] * 4, [1024] * 4, 1, 16, 4),
+    ([100, 333, 1000, 67], [100, 333, 1000, 67], 2, 4, 2),
+    ([150, 250], [300, 200, 150, 250], 2, 8, 2),
+    ([1] * 37, [1] * 37, 1, 2, 1),
+    ([5760] * 4, [5760] * 16, 2, 24, 8),
+])
+def test_bwd_schedule_covers_each_visible_tile_pair_once(q_lens, kv_lens, B, Hq, Hkv):
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv)
+
+
+def test_bwd_schedule_splits_long_ranges_for_balance():
+    units = check_bwd_schedule([1024] * 4, [1024] * 4, 1, 16, 4)
+    lengths = units[:, 4] - units[:, 3]
+    # 4 kv heads x 32 kv tiles would be 128 units of 8..32 query tiles; split for 148 SMs
+    assert len(units) > 148 and lengths.max() <= 9
+    big = check_bwd_schedule([5760] * 8, [5760] * 8, 1, 24, 8)
+    assert len(big) == 8 * 360    # large problems are not split

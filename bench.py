@@ -306,7 +306,8 @@ def run_ours(args, w, world, rank, local):
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
                 "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed alone)", "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
-                "traffic": ncu_traffic(dom, w.name), "avg_launch_ms": round(dom_ms, 4),
+                "traffic": ncu_traffic("bca_bwd_main_kernel" if dom.startswith("bca_bwd") else dom, w.name),
+                "avg_launch_ms": round(dom_ms, 4),
                 "algorithmic_bytes_per_launch": fwd_bytes(w) if dom == "bca_fwd_kernel" else None}
     launches_per_step = 1 + (bca_bwd_launches() if do_bwd else 0)
     clocks = sampler.summary()

@@ -8,34 +8,51 @@
 //
 // Three launches on the caller's stream:
 //   1. prep      one warp per query row: Q^ into the workspace; Delta =
-//                rowsum(dO * O); {lse*log2(e), Delta} pairs in a 128-padded
-//                layout; zero the fp32 dq accumulator and dgamma; then K^ into
-//                the workspace (bca_knorm_kernel, one warp per key row).
-//   2. main      one CTA per (batch, kv head, 128-key tile).  It keeps K and V
-//                of its tile in shared memory and walks every (query tile,
-//                group head) that sees the tile (backward schedule, bca_sched.h):
-//                  S^T  = K Q^^T r_k        dP^T = V dO^T                  (TMEM)
-//                  P^T  = exp2(S^T - lse log2e)   (masked on diagonal steps)
-//                  dS'^T = P^T (dP^T - Delta) r_k   (key-row scaled, bf16 in smem)
+//                rowsum(dO * O); -lse*log2(e) and -Delta, each split into three
+//                bf16 pieces, in a 16-byte row per query (128-padded layout);
+//                zero the fp32 dq accumulator and dgamma; then K^ into the
+//                workspace (bca_knorm_kernel, one warp per key row).
+//   2. main      one CTA per (batch, kv head, 128-key tile, query-tile range).
+//                It keeps K^ and V of its tile in shared memory and walks every
+//                (query tile, group head) of its range (backward schedule,
+//                bca_sched.h):
+//                  S'^T  = K^ Q^^T - lse log2e    dP'^T = V dO^T - Delta    (TMEM)
+//                  P^T   = exp2(S'^T)   (masked on diagonal steps)
+//                  dS'^T = P^T dP'^T    (bf16 in shared memory)
 //                  dV  += P^T dO        (P^T from TMEM)
 //                  G_k += dS'^T Q^      -> gamma_k * dk~ = G_k / (r_k log2 e)
-//                  G_q  = dS' K         -> dq~ = scale gamma_k * G_q, drained with
-//                                          vector red.add into the fp32 accumulator
-//                and finally adds dV and G_k into fp32 accumulators (long query
-//                ranges are split into pieces, so several CTAs may add to one kv tile).
+//                  G_q  = dS' K^        -> dq~ = scale gamma_k * G_q, drained
+//                                          through shared memory with TMA bulk
+//                                          reduce-adds into the fp32 accumulator
+//                The -lse and -Delta terms come out of the tensor core: one extra
+//                K-step of 16 multiplies constant rows (1 at the pieces' k) by the
+//                pieces, so the softmax only computes exp2 and one product.
+//                At the end the CTA adds dV and G_k into fp32 accumulators (long
+//                query ranges are split into pieces, so several CTAs may add to
+//                one kv tile).
 //   3. finalize  one warp per row: dq, dk through the RMSNorm Jacobian, dv, and
 //                dgamma_q, dgamma_k.
 // These are the five matrix products of the Flash-Attention backward (2.5x the
 // forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
 // query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.
 //
-// Main-kernel roles: warpgroups 0-3 (warps 0-15) each own 32 of the 128 query
-// columns of S^T and dP^T (thread i of a warpgroup owns key row i = TMEM lane
-// i) and 32 columns of G_q to drain; warp 16 issues tcgen05 MMAs; warp 17 runs
-// TMA.  TMEM: S^T [0,128) (P^T of warpgroup w overwrites columns [32w, 32w+16)
-// once they have been read), dP^T [128,256) (G_q overwrites it), dV [256,256+D),
-// G_k [384,384+D).
+// Main-kernel roles: warpgroups 0-3 (warps 0-15) each own query columns
+// [16w, 16w+16) and [64+16w, 64+16w+16) of S^T and dP^T (thread i of a
+// warpgroup owns key row i = TMEM lane i) and 32 columns of G_q to drain;
+// warp 16 issues tcgen05 MMAs; warp 17 runs TMA.  All warpgroups finish the
+// first 64 query columns before the second, so the dK~/dV products of the
+// first half run while the second half is computed.  TMEM: S^T [0,128) (P^T
+// of K-step k, 16 queries, overwrites columns [16k, 16k+8) once read), dP^T
+// [128,256) (G_q overwrites it), dV [256,256+D), G_k [384,384+D).
+//
+// Per step the MMA warp issues, in order: dK~/dV for queries 0..63 (after the
+// first half of the softmax), dK~/dV for 64..127 and G_q (after the second
+// half), then S^T of the next step (its P^T has been read) and, once G_q has
+// been drained to registers, dP^T of the next step.  A Q^/dO stage is used by
+// S^T, dP^T, dK~, dV, then holds the dq staging until its bulk reduction has
+// read it; L2 prefetches of the next step's tiles hide part of the reload.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -57,7 +74,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
   kErrKv = 2001, kErrQFull = 2002, kErrQEmpty = 2003, kErrSFull = 2004, kErrDsReady = 2005,
-  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009, kErrMmaDone = 2010
+  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009, kErrLdEmpty = 2010
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool ok, int* status, int code) {
@@ -114,6 +131,28 @@ struct RowIO {
   }
 };
 
+// x = hi + mid + lo with bf16 pieces (about 24 significant bits in all).
+__device__ __forceinline__ void split3(float x, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(h);
+  const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(m);
+  const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+  hi = __bfloat16_as_ushort(h);
+  mid = __bfloat16_as_ushort(m);
+  lo = __bfloat16_as_ushort(l);
+}
+// Packs the pieces of a (k = 0, 1, 2) and b (k = 3, 4, 5) into the first
+// three words of a 16-byte row: returns word 0, writes words 1 and 2.
+__device__ __forceinline__ uint32_t split3_lo2(float a, uint32_t& w1, float b, uint32_t& w2) {
+  uint16_t ah, am, al, bh, bm, bl;
+  split3(a, ah, am, al);
+  split3(b, bh, bm, bl);
+  w1 = (uint32_t)al | ((uint32_t)bh << 16);
+  w2 = (uint32_t)bm | ((uint32_t)bl << 16);
+  return (uint32_t)ah | ((uint32_t)am << 16);
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
   using IO = RowIO<D>;
@@ -151,10 +190,13 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
       const int s = (int)(bs % p.seqlen_q);
       const int b = (int)(bs / p.seqlen_q);
       const int64_t bh = (int64_t)b * p.heads_q + h;
-      float2 v;
-      v.x = __ldg(p.lse + bh * p.seqlen_q + s) * kLog2e;
-      v.y = dot;
-      *reinterpret_cast<float2*>(p.ld + (bh * p.seqlen_q_pad + s) * 2) = v;
+      // -lse (log2 units) and -Delta, each as hi + mid + lo bf16 pieces: the
+      // main kernel adds them to S^T and dP^T with one extra MMA K-step
+      const float nl = -(__ldg(p.lse + bh * p.seqlen_q + s) * kLog2e), nd = -dot;
+      uint4 v;
+      v.x = split3_lo2(nl, v.y, nd, v.z);
+      v.w = 0u;
+      *reinterpret_cast<uint4*>(p.ld + (bh * p.seqlen_q_pad + s) * 4) = v;
     }
   }
 }
@@ -168,14 +210,15 @@ struct BwdLayout {
   static constexpr int kQn = kV + kTile;         // 2 stages
   static constexpr int kDo = kQn + 2 * kTile;    // 2 stages
   static constexpr int kDs = kDo + 2 * kTile;    // dS^T [128 keys][128 queries] bf16, two 64-wide boxes
-  static constexpr int kLd = kDs + 32768;        // 2 stages x 128 x {lse2, Delta}
-  static constexpr int kBars = kLd + 2 * 1024;
+  static constexpr int kLd = kDs + 32768;        // 128 query rows x 8 bf16 {-lse2, -Delta pieces}
+  static constexpr int kOnes = kLd + 2048;       // constant A rows of the extra K-step (3 x 128 B)
+  static constexpr int kBars = kOnes + 384;
   static constexpr int kTmemSlot = kBars + 16 * 8;
   static constexpr int kTotal = kTmemSlot + 16;
 };
 
 struct BwdBars {
-  uint64_t kv_full, s_full, ds_ready, dq_full, dq_drained, acc_full, mma_done;
+  uint64_t kv_full, s_full, ld_empty, ds_half, ds_ready, dq_full, dq_drained, acc_full;
   uint64_t q_full[2], q_empty[2];
 };
 
@@ -202,24 +245,38 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int lane = threadIdx.x & 31;
   const int32_t* u = p.units + (size_t)blockIdx.x * 8;
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
-  const int qb = __ldg(u + 3), qe = __ldg(u + 4), n_diag = __ldg(u + 5);
+  // steps [s_begin, s_end) of this kv tile; step s = (query tile s / group,
+  // head s % group of the kv head's group); query tiles below diag_end need the mask
+  const int s_begin = __ldg(u + 3), s_end = __ldg(u + 4), diag_end = __ldg(u + 5);
   const int group = p.heads_q / p.heads_kv;
-  const int n_steps = (qe - qb) * group;
+  const int n_steps = s_end - s_begin;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->ds_half, kComputeWarpgroups);
+    mbar_init(&bars->ld_empty, 1);
     mbar_init(&bars->ds_ready, kComputeWarpgroups);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_drained, kComputeWarpgroups);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->mma_done, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], kComputeWarpgroups);   // each warpgroup, once its dq staging is read
     }
     fence_mbar_init();
   }
+  // A rows of the extra K-step, read with a zero row-group stride: ones at
+  // k = 0..2 (picks -lse2 for S^T), ones at k = 3..5 (picks -Delta for dP^T),
+  // and a zero core matrix for k = 8..15.
+  if (threadIdx.x < 96) {
+    const int blk = threadIdx.x >> 5, w = threadIdx.x & 31;   // 32 words per 128-byte block
+    const int k0 = (w & 3) * 2;                                 // k of the word's low half
+    auto one_at = [&](int k) { return blk < 2 && k >= 3 * blk && k < 3 * blk + 3; };
+    const uint32_t lo = one_at(k0) ? 0x3F80u : 0u, hi = one_at(k0 + 1) ? 0x3F80u : 0u;
+    reinterpret_cast<uint32_t*>(smem + L::kOnes)[threadIdx.x] = lo | (hi << 16);
+  }
+  fence_proxy_async_smem();
   if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -250,16 +307,28 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       for (int t = 0; t < n_steps; ++t) {
         const int st = t & 1;
         if (!mbar_wait(&bars->q_empty[st], ((t >> 1) & 1) ^ 1, p.status, kErrQEmpty)) break;
-        const int qt = qb + t / group, h = hk * group + t % group;
-        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 1024);
+        const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
+        // the single {-lse, -Delta} buffer: the previous step's S^T/dP^T have read it
+        if (t > 0 && !mbar_wait(&bars->ld_empty, (t - 1) & 1, p.status, kErrLdEmpty)) break;
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2048);
         for (int box = 0; box < D / 64; ++box) {
           tma_load_4d(smem + L::kQn + st * L::kTile + box * 16384, &tm_qn, &bars->q_full[st], box * 64, h,
                       qt * 128, b);
           tma_load_4d(smem + L::kDo + st * L::kTile + box * 16384, &tm_do, &bars->q_full[st], box * 64, h,
                       qt * 128, b);
         }
-        const float* ld_src = p.ld + (((size_t)b * p.heads_q + h) * p.seqlen_q_pad + (size_t)qt * 128) * 2;
-        bulk_load(smem + L::kLd + st * 1024, ld_src, 1024, &bars->q_full[st]);
+        const float* ld_src = p.ld + (((size_t)b * p.heads_q + h) * p.seqlen_q_pad + (size_t)qt * 128) * 4;
+        bulk_load(smem + L::kLd, ld_src, 2048, &bars->q_full[st]);
+        // warm L2 with the next step's tiles: their loads are issued only once
+        // a stage frees, and then wait on memory otherwise
+        if (t + 1 < n_steps) {
+          const int qt1 = (s_begin + t + 1) / group, h1 = hk * group + (s_begin + t + 1) % group;
+          for (int box = 0; box < D / 64; ++box) {
+            tma_prefetch_l2_4d(&tm_qn, box * 64, h1, qt1 * 128, b);
+            tma_prefetch_l2_4d(&tm_do, box * 64, h1, qt1 * 128, b);
+          }
+          bulk_prefetch_l2(p.ld + (((size_t)b * p.heads_q + h1) * p.seqlen_q_pad + (size_t)qt1 * 128) * 4, 2048);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -272,14 +341,23 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       const uint32_t kn_a = smem_u32(smem + L::kK), v_a = smem_u32(smem + L::kV);
       const uint32_t qn_a = smem_u32(smem + L::kQn), do_a = smem_u32(smem + L::kDo);
       const uint32_t ds_a = smem_u32(smem + L::kDs);
-      // C[128 x 128] = A[128 x D] B[128 x D]^T with both operands K-major.
-      auto mma_kmajor = [&](uint32_t d, uint32_t a, uint32_t bb) {
+      // C[128 x 128] = A[128 x D] B[128 x D]^T with both operands K-major, then
+      // one K-step more: C += ones(k in pick) x pieces^T, which adds -lse2 (S^T)
+      // or -Delta (dP^T) of each query column.  The pieces sit in 16-byte rows
+      // (no swizzle: 8-row core matrices of 128 B); the constant A rows are read
+      // with a zero row-group stride.  The B core matrix at k = 8..15 is the
+      // next row group's (finite) data, multiplied by A's zero core matrix.
+      const uint32_t ld_a = smem_u32(smem + L::kLd), ones_a = smem_u32(smem + L::kOnes);
+      const uint64_t ext_b = make_noswz_desc(ld_a, 128, 128);
+      const uint64_t ext_lse = make_noswz_desc(ones_a, 256, 0), ext_delta = make_noswz_desc(ones_a + 128, 128, 0);
+      auto mma_kmajor = [&](uint32_t d, uint32_t a, uint32_t bb, uint64_t ext_a) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
           mma_bf16_ss(tmem + d, make_sw128_desc(a + off, 16, 1024), make_sw128_desc(bb + off, 16, 1024), id_kk,
                       kk > 0);
         }
+        mma_bf16_ss(tmem + d, ext_a, ext_b, id_kk, true);
       };
       bool ok = mbar_wait(&bars->kv_full, 0, p.status, kErrKv);
       // Issue order per step t: dQ~(t) | dK~(t), dV(t) | dP(t+1), S(t+1), so the
@@ -289,43 +367,54 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ok = mbar_wait(&bars->q_full[0], 0, p.status, kErrQFull);
         if (ok) {
           tc_fence_after();
-          mma_kmajor(T_DP, v_a, do_a);
-          mma_kmajor(T_S, kn_a, qn_a);
+          mma_kmajor(T_DP, v_a, do_a, ext_delta);
+          mma_kmajor(T_S, kn_a, qn_a, ext_lse);
           mma_commit(&bars->s_full);
+          mma_commit(&bars->ld_empty);
         }
       }
       for (int t = 0; t < n_steps && ok; ++t) {
         const int st = t & 1;
         const uint32_t qn_s = qn_a + st * L::kTile, do_s = do_a + st * L::kTile;
+        // G_k += dS'^T Q^ : A = dS'^T [keys][queries] (K-major), B = Q^ [queries][D] (MN-major);
+        // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major).
+        // K-steps 0..3 (queries 0..63) as soon as that half of dS' and P^T is in place.
+        auto dkdv = [&](int k_begin) {
+#pragma unroll
+          for (int kk = k_begin; kk < k_begin + 4; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + T_DK, make_sw128_desc(ds_a + off, 16, 1024),
+                        make_sw128_desc(qn_s + kk * 2048, 16384, 1024), id_km, t > 0 || kk > 0);
+          }
+#pragma unroll
+          for (int kk = k_begin; kk < k_begin + 4; ++kk)
+            mma_bf16_ts(tmem + T_DV, tmem + T_S + kk * 16, make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts,
+                        t > 0 || kk > 0);
+        };
+        if (!(ok = mbar_wait(&bars->ds_half, t & 1, p.status, kErrDsReady))) break;
+        tc_fence_after();
+        dkdv(0);
         if (!(ok = mbar_wait(&bars->ds_ready, t & 1, p.status, kErrDsReady))) break;
         tc_fence_after();
+        dkdv(4);
         // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
                       make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
-        mma_commit(&bars->dq_full);   // the drain overlaps the two products below
-        // G_k += dS'^T Q^ : A = dS'^T [keys][queries] (K-major), B = Q^ [queries][D] (MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + T_DK, make_sw128_desc(ds_a + off, 16, 1024),
-                      make_sw128_desc(qn_s + kk * 2048, 16384, 1024), id_km, t > 0 || kk > 0);
-        }
-        // dV += P^T dO : A = P^T (TMEM, K = queries), B = dO [queries][D] (MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + T_DV, tmem + T_S + (kk >> 1) * 32 + (kk & 1) * 8,
-                      make_sw128_desc(do_s + kk * 2048, 16384, 1024), id_ts, t > 0 || kk > 0);
-        mma_commit(&bars->mma_done);   // this step's Q^ / dO stage and dS^T are no longer read
+        mma_commit(&bars->dq_full);   // G_q ready; this step's Q^ / dO stage and dS^T are no longer read
         if (t + 1 < n_steps) {
           const int st1 = (t + 1) & 1;
-          if (!(ok = mbar_wait(&bars->dq_drained, t & 1, p.status, kErrDqDrained))) break;
+          // S^T(t+1) only needs P^T(t) read (dV was issued before); dP^T(t+1)
+          // overwrites G_q and waits for the drain.
           if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
           tc_fence_after();
-          mma_kmajor(T_DP, v_a, do_a + st1 * L::kTile);
-          mma_kmajor(T_S, kn_a, qn_a + st1 * L::kTile);
+          mma_kmajor(T_S, kn_a, qn_a + st1 * L::kTile, ext_lse);
+          if (!(ok = mbar_wait(&bars->dq_drained, t & 1, p.status, kErrDqDrained))) break;
+          tc_fence_after();
+          mma_kmajor(T_DP, v_a, do_a + st1 * L::kTile, ext_delta);
           mma_commit(&bars->s_full);
+          mma_commit(&bars->ld_empty);
         }
       }
       if (ok) mma_commit(&bars->acc_full);
@@ -358,65 +447,59 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
       const int st = t & 1;
-      const int qt = qb + t / group, h = hk * group + t % group;
+      const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
       const int q0 = qt * 128;
-      const bool diag = (qt - qb) < n_diag;
+      const bool diag = qt < diag_end;
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
-      if (ok) {
-        tc_fence_after();
-        const float4* ld4 = reinterpret_cast<const float4*>(smem + L::kLd + st * 1024) + wg * 16;
-        const int lim = row_min - (q0 + wg * 32);   // columns c < lim are masked on diagonal steps
-        uint8_t* ds_box = smem + L::kDs + (wg >> 1) * 16384;
-        // two groups of 16 query columns, to keep the working set small
+      // Warpgroup w owns query columns [16w, 16w+16) of each 64-column half:
+      // the first half's dK~/dV products run while the second half is computed.
+      if (ok) tc_fence_after();
 #pragma unroll
-        for (int grp = 0; grp < 2; ++grp) {
+      for (int grp = 0; grp < 2; ++grp) {
+        if (ok) {
+          const int col0 = grp * 64 + wg * 16;
           uint32_t sr[16], dpr[16];
-          tmem_ld16(tmem + lane_base + T_S + wg * 32 + grp * 16, sr);
-          tmem_ld16(tmem + lane_base + T_DP + wg * 32 + grp * 16, dpr);
+          tmem_ld16(tmem + lane_base + T_S + col0, sr);
+          tmem_ld16(tmem + lane_base + T_DP + col0, dpr);
           tmem_wait_ld();
           uint32_t pk[8], dk[8];
           if (!diag) {
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const float4 l = ld4[grp * 8 + (c >> 1)];   // {lse2, Delta} of columns c and c + 1
-              const uint64_t a2 =
-                  f2_add(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), f2_pack(-l.x, -l.z));
-              float a0, a1;
-              f2_unpack(a2, a0, a1);
-              const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
-              const uint64_t g2 =
-                  f2_add(f2_pack(__uint_as_float(dpr[c]), __uint_as_float(dpr[c + 1])), f2_pack(-l.y, -l.w));
+              const float p0 = fast_exp2(__uint_as_float(sr[c])), p1 = fast_exp2(__uint_as_float(sr[c + 1]));
               float d0, d1;
-              f2_unpack(f2_mul(g2, f2_pack(p0, p1)), d0, d1);
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(dpr[c]), __uint_as_float(dpr[c + 1])), f2_pack(p0, p1)), d0, d1);
               pk[c >> 1] = pack_bf16x2(p0, p1);
               dk[c >> 1] = pack_bf16x2(d0, d1);
             }
           } else {
+            const int lim = row_min - (q0 + col0);   // columns c < lim cannot see key j
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const int cc = grp * 16 + c;
-              const float4 l = ld4[cc >> 1];
-              const float p0 = cc < lim ? 0.f : fast_exp2(__uint_as_float(sr[c]) - l.x);
-              const float p1 = cc + 1 < lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]) - l.z);
-              const float d0 = p0 * (__uint_as_float(dpr[c]) - l.y);
-              const float d1 = p1 * (__uint_as_float(dpr[c + 1]) - l.w);
+              const float p0 = c < lim ? 0.f : fast_exp2(__uint_as_float(sr[c]));
+              const float p1 = c + 1 < lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]));
+              const float d0 = p0 * __uint_as_float(dpr[c]);
+              const float d1 = p1 * __uint_as_float(dpr[c + 1]);
               pk[c >> 1] = pack_bf16x2(p0, p1);
               dk[c >> 1] = pack_bf16x2(d0, d1);
             }
           }
-          // P^T of these 16 queries (8 packed columns) goes into this warpgroup's
-          // own S^T columns, which have been read: group 0 -> [32w, 32w+8) (its
-          // S^T group 0 is in registers), group 1 -> [32w+8, 32w+16) (S^T group 0's
-          // columns, read before).
-          tmem_st8(tmem + lane_base + T_S + wg * 32 + grp * 8, pk);
+          // P^T of these 16 queries (8 packed columns) goes into the first half
+          // of the S^T columns just read: K-step kk = col0/16 of dV reads it there.
+          tmem_st8(tmem + lane_base + T_S + col0, pk);
+          uint8_t* ds_box = smem + L::kDs + grp * 16384;
 #pragma unroll
           for (int c8 = 0; c8 < 2; ++c8)
-            *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, (wg & 1) * 32 + grp * 16 + c8 * 8)) =
+            *reinterpret_cast<uint4*>(ds_box + sw128_offset(j, wg * 16 + c8 * 8)) =
                 make_uint4(dk[4 * c8], dk[4 * c8 + 1], dk[4 * c8 + 2], dk[4 * c8 + 3]);
+          tmem_wait_st();
+          tc_fence_before();
+          fence_proxy_async_smem();
         }
-        tmem_wait_st();
-        tc_fence_before();
-        fence_proxy_async_smem();
+        if (grp == 0) {
+          named_bar_sync(bar_id, 128);
+          if (j == 0 && ok) mbar_arrive(&bars->ds_half);
+        }
       }
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) {
@@ -432,7 +515,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
       // Drain G_q (TMEM lane = query row of this step) into the fp32 accumulator:
       // TMEM -> registers (then the dP^T/G_q columns are free again), registers ->
-      // this step's Q^/dO stage (idle once mma_done has fired), then a TMA bulk
+      // this step's Q^/dO stage (dq_full also means dK~ and dV have read it), then a TMA bulk
       // reduce-add.  The stage goes back to the producer at the next step.
       ok = warp_wait(&bars->dq_full, t & 1, ok, p.status, kErrDqFull);
       uint32_t gq[32];
@@ -444,8 +527,6 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       }
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) mbar_arrive(&bars->dq_drained);
-      // the stage is staging space only once the dK~ and dV products have read it
-      ok = warp_wait(&bars->mma_done, t & 1, ok, p.status, kErrMmaDone);
       // chunk wg: the first D/64 chunks fill this step's Q^ stage, the rest its dO stage
       constexpr int kChunksPerBuffer = D / 64;
       uint8_t* chunk = wg < kChunksPerBuffer ? smem + L::kQn + st * L::kTile + wg * 16384
@@ -618,7 +699,7 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 16);
   if (p.seqlen_q_pad != p.seqlen_q) {
     // padding entries of the {lse, Delta} pairs are read by full-tile loads
-    e = cudaMemsetAsync(p.ld, 0, (size_t)p.batch * p.heads_q * p.seqlen_q_pad * 2 * sizeof(float), stream);
+    e = cudaMemsetAsync(p.ld, 0, (size_t)p.batch * p.heads_q * p.seqlen_q_pad * 16, stream);
     if (e != cudaSuccess) return e;
   }
   // dV and G_k are sums over the pieces of each kv tile
@@ -651,7 +732,7 @@ BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D
   w.qn = 0;
   w.kn = w.qn + up((size_t)B * Sq * Hq * D * 2);
   w.ld = w.kn + up((size_t)B * Skv * Hkv * D * 2);
-  w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 2 * 4);
+  w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 16);
   w.dvacc = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
   w.dkacc = w.dvacc + up((size_t)B * Skv * Hkv * D * 4);
   w.total = w.dkacc + up((size_t)B * Skv * Hkv * D * 4);

@@ -47,7 +47,7 @@ struct BwdParams {
   // workspace
   uint16_t* qn;               // forward query operand Q^       [B, Sq, Hq, D]
   uint16_t* kn;               // forward key operand K^ = bf16(k r_k) [B, Skv, Hkv, D]
-  float* ld;                  // {lse * log2(e), Delta} pairs [B, Hq, Sq_pad, 2]
+  float* ld;                  // 16-byte rows of bf16 pieces of -lse*log2(e), -Delta [B, Hq, Sq_pad, 8 x bf16]
   float* dqacc;               // fp32 G_q accumulator          [B, Sq, Hq, D]
   float* dvacc;               // fp32 dV accumulator           [B, Skv, Hkv, D]
   float* dkacc;               // fp32 G_k accumulator          [B, Skv, Hkv, D]

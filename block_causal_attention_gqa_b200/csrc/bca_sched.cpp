@@ -3,6 +3,8 @@
 
 #include <algorithm>
 #include <cmath>
+#include <functional>
+#include <queue>
 #include <tuple>
 
 namespace magi {
@@ -111,62 +113,103 @@ std::vector<int32_t> build_fwd_schedule(const int32_t* qo, const int32_t* ko, co
   return out;
 }
 
+namespace {
+
+// Longest-processing-time list scheduling of `costs` (sorted, largest first)
+// on `machines` identical machines: the CTA scheduler starts the next CTA in
+// launch order on whichever SM frees first.  Returns the makespan.
+double lpt_makespan(const std::vector<double>& costs, int machines) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> load;
+  for (int m = 0; m < machines; ++m) load.push(0.0);
+  double span = 0.0;
+  for (double c : costs) {
+    const double t = load.top() + c;
+    load.pop();
+    load.push(t);
+    span = std::max(span, t);
+  }
+  return span;
+}
+
+}  // namespace
+
 std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d, int num_sms) {
   const int n_qt = (d.seqlen_q + kBlockM - 1) / kBlockM;
   const int n_kt = (d.seqlen_kv + kBlockN - 1) / kBlockN;
+  const int group = d.heads_q / d.heads_kv;
   std::vector<int> tile_lo(n_qt);  // smallest visible end among the tile's rows
   for (int t = 0; t < n_qt; ++t) tile_lo[t] = row_kv_end(qo, ko, d, t * kBlockM);
-  struct Unit {
-    int b, hk, n0, qb, qe, nd;
+  // One step = (query tile qt, head g of the kv head's group), numbered qt * group + g.
+  struct Seq {
+    int b, hk, n0, s_begin, s_end, diag_end;
   };
-  std::vector<Unit> units;
+  std::vector<Seq> seqs;
   for (int kt = 0; kt < n_kt; ++kt) {
     const int n0 = kt * kBlockN;
     const int n_end = std::min(n0 + kBlockN, d.seqlen_kv);
-    // first query row whose visible end exceeds n0
-    int qrow = d.seqlen_q;
-    {
-      int lo = 0, hi = d.seqlen_q;  // binary search on the non-decreasing row ends
-      while (lo < hi) {
-        const int mid = (lo + hi) / 2;
-        if (row_kv_end(qo, ko, d, mid) > n0) hi = mid; else lo = mid + 1;
-      }
-      qrow = lo;
+    int lo = 0, hi = d.seqlen_q;  // first query row whose visible end exceeds n0 (row ends are non-decreasing)
+    while (lo < hi) {
+      const int mid = (lo + hi) / 2;
+      if (row_kv_end(qo, ko, d, mid) > n0) hi = mid; else lo = mid + 1;
     }
-    if (qrow >= d.seqlen_q) continue;  // nobody sees this kv tile
-    const int qb = qrow / kBlockM;
-    int nd = 0;
-    for (int t = qb; t < n_qt && tile_lo[t] < n_end; ++t) ++nd;
+    if (lo >= d.seqlen_q) continue;  // nobody sees this kv tile
+    const int qb = lo / kBlockM;
+    int diag_end = qb;
+    while (diag_end < n_qt && tile_lo[diag_end] < n_end) ++diag_end;
     for (int b = 0; b < d.batch; ++b)
-      for (int hk = 0; hk < d.heads_kv; ++hk) units.push_back({b, hk, n0, qb, n_qt, nd});
+      for (int hk = 0; hk < d.heads_kv; ++hk) seqs.push_back({b, hk, n0, qb * group, n_qt * group, diag_end});
   }
-  // Split long query ranges so every SM gets about two pieces of similar size
-  // (pieces of one kv tile add their dK/dV partials in the fp32 accumulators).
-  int64_t visits = 0;
-  for (const Unit& u : units) visits += u.qe - u.qb;
-  const int64_t cap = std::max<int64_t>(2, (visits + 2 * num_sms - 1) / (2 * (int64_t)std::max(num_sms, 1)));
-  std::vector<Unit> pieces;
-  pieces.reserve(units.size());
-  for (const Unit& u : units) {
-    const int len = u.qe - u.qb;
-    const int n_pieces = (int)((len + cap - 1) / cap);
-    const int step = (len + n_pieces - 1) / n_pieces;
-    for (int qs = u.qb; qs < u.qe; qs += step) {
-      const int qe = std::min(qs + step, u.qe);
-      const int nd = std::max(0, std::min(qe, u.qb + u.nd) - qs);   // diagonal tiles come first
-      pieces.push_back({u.b, u.hk, u.n0, qs, qe, nd});
+  // Cut every sequence into k near-equal pieces of at most `len` steps; pick
+  // `len` by simulating the CTA scheduler, charging each piece a fixed
+  // overhead (its K/V load and pipeline fill, and the dV/dK reduction at the
+  // end) of about two steps.
+  constexpr double kPieceOverhead = 2.0;
+  const int sms = std::max(num_sms, 1);
+  int max_len = 1;
+  int64_t total = 0;
+  for (const Seq& q : seqs) {
+    max_len = std::max(max_len, q.s_end - q.s_begin);
+    total += q.s_end - q.s_begin;
+  }
+  // pieces shorter than an eighth of an SM's share only add overhead
+  const double min_len = std::max(4.0, (double)total / (8.0 * sms));
+  std::vector<int> candidates;
+  for (double c = max_len; c >= min_len; c /= 1.08) candidates.push_back((int)std::lround(c));
+  if (candidates.empty()) candidates.push_back(max_len);
+  int best_len = max_len;
+  double best_span = 0.0;
+  std::vector<double> costs;
+  for (int len : candidates) {
+    if (len <= 0) continue;
+    costs.clear();
+    for (const Seq& q : seqs) {
+      const int n = q.s_end - q.s_begin;
+      const int k = (n + len - 1) / len;
+      for (int i = 0; i < k; ++i) costs.push_back((double)(n * (i + 1) / k - n * i / k) + kPieceOverhead);
+    }
+    std::sort(costs.begin(), costs.end(), std::greater<double>());
+    const double span = lpt_makespan(costs, sms);
+    if (best_span == 0.0 || span < best_span - 1e-9) {
+      best_span = span;
+      best_len = len;
     }
   }
-  units.swap(pieces);
-  std::stable_sort(units.begin(), units.end(), [](const Unit& a, const Unit& b) {
-    const int ca = a.qe - a.qb, cb = b.qe - b.qb;
+  std::vector<Seq> pieces;
+  for (const Seq& q : seqs) {
+    const int n = q.s_end - q.s_begin;
+    const int k = (n + best_len - 1) / best_len;
+    for (int i = 0; i < k; ++i)
+      pieces.push_back({q.b, q.hk, q.n0, q.s_begin + n * i / k, q.s_begin + n * (i + 1) / k, q.diag_end});
+  }
+  std::stable_sort(pieces.begin(), pieces.end(), [](const Seq& a, const Seq& b) {
+    const int ca = a.s_end - a.s_begin, cb = b.s_end - b.s_begin;
     if (ca != cb) return ca > cb;
-    return std::tie(a.b, a.hk, a.n0) < std::tie(b.b, b.hk, b.n0);
+    return std::tie(a.b, a.hk, a.s_begin, a.n0) < std::tie(b.b, b.hk, b.s_begin, b.n0);
   });
   std::vector<int32_t> out;
-  out.reserve(units.size() * kUnitInts);
-  for (const Unit& u : units) {
-    const int32_t v[kUnitInts] = {u.b, u.hk, u.n0, u.qb, u.qe, u.nd, 0, 0};
+  out.reserve(pieces.size() * kUnitInts);
+  for (const Seq& u : pieces) {
+    const int32_t v[kUnitInts] = {u.b, u.hk, u.n0, u.s_begin, u.s_end, u.diag_end, 0, 0};
     out.insert(out.end(), v, v + kUnitInts);
   }
   return out;

@@ -48,10 +48,12 @@ std::vector<int32_t> build_fwd_schedule(const int32_t* q_offsets, const int32_t*
 // the query tiles that see any of its keys are the q tiles [q_begin, n_qt):
 // since visibility only grows with the chunk index, every query row at or
 // after the first row whose visible end exceeds t*128 sees some key of it.
-// Long ranges are cut into pieces so that `num_sms` SMs get about two pieces
-// each.  Emits per unit {batch, kv_head, n0, q_tile_begin, q_tile_end,
-// n_diag_q_tiles, 0, 0} where the first n_diag_q_tiles q tiles of the range
-// need the mask; units are sorted longest first.
+// A step is one (query tile qt, head g of the kv head's group), numbered
+// qt * group + g; each kv tile's steps are cut into near-equal pieces whose
+// length is chosen by simulating list scheduling of the pieces on `num_sms`
+// SMs.  Emits per unit {batch, kv_head, n0, step_begin, step_end, diag_end,
+// 0, 0}, where query tiles below diag_end need the mask; units are sorted
+// longest first.
 std::vector<int32_t> build_bwd_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                                         const magi_bca_dims& d, int num_sms);
 

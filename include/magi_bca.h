@@ -165,11 +165,13 @@ int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
                               const magi_bca_dims* dims, int32_t* units, int64_t capacity);
 
 /* Host-only view of the backward schedule (no device needed).  A unit is one
- * 128-key tile of one (batch, kv head) and a contiguous range of the query
- * tiles that see it; long ranges are split so that `num_sms` SMs get about two
- * units each.  Per unit 8 int32:
- *   {batch, kv_head, n0 (first key), q_tile_begin, q_tile_end,
- *    n_diag (the first n_diag query tiles of the range need the mask), 0, 0}
+ * 128-key tile of one (batch, kv head) and a contiguous range of its "steps":
+ * a step is one (query tile qt, query head g of the kv head's group) that sees
+ * the tile, numbered qt * G + g with G = heads_q / heads_kv.  Each tile's steps
+ * are cut into near-equal pieces whose length is chosen by simulating how
+ * `num_sms` SMs would run them.  Per unit 8 int32:
+ *   {batch, kv_head, n0 (first key), step_begin, step_end,
+ *    diag_end (query tiles below it need the mask), 0, 0}
  * in launch order (longest first).  Returns the number of units (writing at
  * most `capacity`), or a negative status. */
 int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,

@@ -202,27 +202,27 @@ def test_workload_shapes():
 def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
+    G = Hq // Hkv
     units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms)
     ends = row_ends(qo, ko, Sq)
     n_qt, n_kt = -(-Sq // 128), -(-Skv // 128)
-    cover = np.zeros((B, Hkv, n_kt, n_qt), np.int64)
+    cover = np.zeros((B, Hkv, n_kt, n_qt, G), np.int64)
     lengths = []
-    for b, hk, n0, qb, qe, nd, _, _ in units:
-        assert n0 % 128 == 0 and 0 <= qb < qe <= n_qt and 0 <= nd <= qe - qb
-        cover[b, hk, n0 // 128, qb:qe] += 1
+    for b, hk, n0, s0, s1, diag_end, _, _ in units:
+        assert n0 % 128 == 0 and 0 <= s0 < s1 <= n_qt * G
         n_end = min(n0 + 128, Skv)
-        for t in range(qb, qe):
+        for s in range(s0, s1):
+            t, g = divmod(s, G)
+            cover[b, hk, n0 // 128, t, g] += 1
             rows = ends[t * 128:min(t * 128 + 128, Sq)]
-            sees = rows > n0                          # row sees some key of the tile
-            assert sees.any()
-            needs_mask = rows.min() < n_end
-            assert needs_mask == (t - qb < nd), (t, qb, nd)
-        lengths.append(qe - qb)
-    # every (kv tile, query tile) pair where some query sees some key: exactly once
+            assert (rows > n0).any()                  # some row of the tile sees some key
+            assert (rows.min() < n_end) == (t < diag_end), (t, diag_end)
+        lengths.append(s1 - s0)
+    # every (kv tile, query tile, head) where some query sees some key: exactly once
     for kt in range(n_kt):
         for t in range(n_qt):
             want = int((ends[t * 128:min(t * 128 + 128, Sq)] > kt * 128).any())
-            assert (cover[:, :, kt, t] == want).all(), (kt, t)
+            assert (cover[:, :, kt, t, :] == want).all(), (kt, t)
     assert all(a >= b for a, b in zip(lengths, lengths[1:]))
     return units
 
@@ -235,14 +235,31 @@ def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148):
     ([1] * 37, [1] * 37, 1, 2, 1),
     ([5760] * 4, [5760] * 16, 2, 24, 8),
 ])
-def test_bwd_schedule_covers_each_visible_tile_pair_once(q_lens, kv_lens, B, Hq, Hkv):
+def test_bwd_schedule_covers_each_visible_step_once(q_lens, kv_lens, B, Hq, Hkv):
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv)
 
 
-def test_bwd_schedule_splits_long_ranges_for_balance():
+def lpt_span(costs, machines):
+    import heapq
+    load = [0.0] * machines
+    for c in sorted(costs, reverse=True):
+        heapq.heapreplace(load, load[0] + c)
+    return max(load)
+
+
+def test_bwd_schedule_balances_the_sms():
+    """train4k: 128 kv tiles with 32, 24, 16 or 8 visible query tiles x 4 heads.
+    Whole tiles (or the earlier 8-query-tile pieces: 320 units, three waves)
+    leave SMs idle; the step-granular pieces must come within 15% of perfect
+    balance, counting two steps of overhead per piece."""
     units = check_bwd_schedule([1024] * 4, [1024] * 4, 1, 16, 4)
-    lengths = units[:, 4] - units[:, 3]
-    # 4 kv heads x 32 kv tiles would be 128 units of 8..32 query tiles; split for 148 SMs
-    assert len(units) > 148 and lengths.max() <= 9
+    steps = units[:, 4] - units[:, 3]
+    assert steps.sum() == 4 * 8 * (32 + 24 + 16 + 8) * 4
+    span = lpt_span(list(steps + 2.0), 148)
+    ideal = (steps.sum() + 2.0 * len(steps)) / 148
+    assert span <= 1.15 * ideal, (span, ideal, len(steps))
+    old = lpt_span([32 + 2.0] * 320, 148)
+    assert span < 0.85 * old
+    # a problem with far more work than SMs is left in whole kv tiles
     big = check_bwd_schedule([5760] * 8, [5760] * 8, 1, 24, 8)
-    assert len(big) == 8 * 360    # large problems are not split
+    assert len(big) == 8 * 360

@@ -302,15 +302,25 @@ def run_ours(args, w, world, rank, local):
     else:
         dom, dom_flops, dom_ms = "bca_fwd_kernel", fwd_flops(w), fwd_avg
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
+    clocks = sampler.summary()
+    # Burst peak for a kernel that runs at full clock; the sustained one (a
+    # seconds-long GEMM loop under the 1 kW cap) once the timed region itself
+    # ran into the power cap or well below the maximum clock.
+    capped = "sw_power_cap" in clocks.get("reasons", []) or (
+        clocks.get("sm_mhz") and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    if capped:
+        peak = peaks["bf16_tflops_sustained"]
+        peak_note = f"{peak_src} bf16_tflops_sustained (the timed region ran at the power cap)"
+    else:
+        peak = peaks["bf16_tflops"]
+        peak_note = f"{peak_src} bf16_tflops (burst; full clock during the timed region)"
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
-                "peak_source": f"{peak_src} bf16_tflops (burst; kernel timed alone)", "unit": "TFLOP/s",
+                "peak_source": peak_note, "unit": "TFLOP/s",
                 "frac": round(achieved / peak, 4), "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
                 "traffic": ncu_traffic("bca_bwd_main_kernel" if dom.startswith("bca_bwd") else dom, w.name),
                 "avg_launch_ms": round(dom_ms, 4),
                 "algorithmic_bytes_per_launch": fwd_bytes(w) if dom == "bca_fwd_kernel" else None}
-    launches_per_step = 1 + (bca_bwd_launches() if do_bwd else 0)
-    clocks = sampler.summary()
+    launches_per_step = bca_fwd_launches() + (bca_bwd_launches() if do_bwd else 0)
     res = {
         "metric": "block-causal attention useful TFLOP/s on 1 B200 and % of dense BF16 peak",
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -336,8 +346,12 @@ def run_ours(args, w, world, rank, local):
     return res
 
 
+def bca_fwd_launches():
+    return 2   # key pre-pass, forward kernel
+
+
 def bca_bwd_launches():
-    return 3   # prep, main, finalize (plus a memset of the padded lse rows when Sq % 128 != 0)
+    return 3   # prep (query and key rows), main, finalize (plus a memset of the padded lse rows when Sq % 128 != 0)
 
 
 # ------------------------------------------------------------------ oracle (CPU)

@@ -7,11 +7,12 @@
 // order (the helpers in bca_norm.cuh fix the rounding points for both passes).
 //
 // Three launches on the caller's stream:
-//   1. prep      one warp per query row: Q^ into the workspace; Delta =
+//   1. prep      one warp per row.  Query rows: Q^ into the workspace; Delta =
 //                rowsum(dO * O); -lse*log2(e) and -Delta, each split into three
 //                bf16 pieces, in a 16-byte row per query (128-padded layout);
-//                zero the fp32 dq accumulator and dgamma; then K^ into the
-//                workspace (bca_knorm_kernel, one warp per key row).
+//                zero the row's fp32 dq accumulator.  Key rows: K^ into the
+//                workspace (knorm_row, as the forward's key pre-pass) and zero
+//                the row's fp32 dV / G_k accumulators.  Also zeroes dgamma.
 //   2. main      one CTA per (batch, kv head, 128-key tile, query-tile range).
 //                It keeps K^ and V of its tile in shared memory and walks every
 //                (query tile, group head) of its range (backward schedule,
@@ -167,9 +168,21 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
   const int lane = threadIdx.x & 31;
   const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
-  // one warp per query row, coalesced; the sum of squares uses the order that
-  // the forward's prologue reproduces, so Q^ is bit-identical to the forward's
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < n_q; r += warps) {
+  const int64_t n_k = (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
+  // One warp per row: query rows [0, n_q), then key rows.  For a query row the
+  // sum of squares uses the order that the forward's prologue reproduces, so
+  // Q^ is bit-identical to the forward's.  For a key row, K^ = bf16(k r_k)
+  // exactly as the forward's key pre-pass computes it, and the row's fp32
+  // dV / G_k accumulators are zeroed.
+  for (int64_t rr = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); rr < n_q + n_k; rr += warps) {
+    if (rr >= n_q) {
+      const int64_t r = rr - n_q;
+      knorm_row<D>(p.k + r * D, p.kn + r * D, lane, p.eps);
+      IO::store_zero_f32(p.dvacc + r * D, lane);
+      IO::store_zero_f32(p.dkacc + r * D, lane);
+      continue;
+    }
+    const int64_t r = rr;
     float x[E], o[E], g[E];
     IO::load_bf16(p.q + r * D, lane, x);
     IO::load_bf16(p.out + r * D, lane, o);
@@ -615,12 +628,12 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
     gm[e] = __ldg(p.gamma_q + lane * E + e);
     gk[e] = __ldg(p.gamma_k + lane * E + e);
   }
-  for (int64_t rr = (int64_t)blockIdx.x * 8 + wid; rr < n_q + n_k; rr += warps) {
+  // Two rows per warp and iteration, all loads issued before the arithmetic,
+  // so each warp keeps two rows' reads in flight.
+  auto finish_row = [&](int64_t rr, float (&x)[E], float (&g)[E], const float (&dvv)[E]) {
     const bool is_q = rr < n_q;
     const int64_t r = is_q ? rr : rr - n_q;
-    float x[E], g[E], dqt[E];
-    IO::load_bf16((is_q ? p.q : p.k) + r * D, lane, x);
-    IO::load_f32((is_q ? p.dqacc : p.dkacc) + r * D, lane, g);
+    float dqt[E];
     // g = gamma * dx~   (for query rows dq~ = scale gamma_k G_q is kept for dgamma_q)
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -647,12 +660,26 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
       for (int e = 0; e < E; ++e) gacc_q[e] = fmaf(dqt[e], x[e], gacc_q[e]);
     } else {
       IO::store_bf16(p.dk + r * D, lane, o);
-      float dvv[E];
-      IO::load_f32(p.dvacc + r * D, lane, dvv);
       IO::store_bf16(p.dv + r * D, lane, dvv);
 #pragma unroll
       for (int e = 0; e < E; ++e) gacc_k[e] = fmaf(g[e] / gk[e], x[e], gacc_k[e]);
     }
+  };
+  auto load_row = [&](int64_t rr, float (&x)[E], float (&g)[E], float (&dvv)[E]) {
+    const bool is_q = rr < n_q;
+    const int64_t r = is_q ? rr : rr - n_q;
+    IO::load_bf16((is_q ? p.q : p.k) + r * D, lane, x);
+    IO::load_f32((is_q ? p.dqacc : p.dkacc) + r * D, lane, g);
+    if (!is_q) IO::load_f32(p.dvacc + r * D, lane, dvv);
+  };
+  const int64_t total = n_q + n_k;
+  for (int64_t rr = (int64_t)blockIdx.x * 8 + wid; rr < total; rr += 2 * warps) {
+    const int64_t rr2 = rr + warps;
+    float x0[E], g0[E], v0[E], x1[E], g1[E], v1[E];
+    load_row(rr, x0, g0, v0);
+    if (rr2 < total) load_row(rr2, x1, g1, v1);
+    finish_row(rr, x0, g0, v0);
+    if (rr2 < total) finish_row(rr2, x1, g1, v1);
   }
   if (p.dgamma_q != nullptr || p.dgamma_k != nullptr) {
 #pragma unroll
@@ -695,22 +722,26 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q;
-  const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 16);
+  const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
+  // one wave of the row kernels (grid-stride loops over one warp per row)
+  static int prep_per_sm[2] = {0, 0}, fin_per_sm[2] = {0, 0};
+  int& prep_occ = prep_per_sm[D == 128];
+  int& fin_occ = fin_per_sm[D == 128];
+  if (prep_occ == 0) {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_prep_kernel<D>, 256, 0);
+    prep_occ = std::max(n, 1);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D>, 256, 0);
+    fin_occ = std::max(n, 1);
+  }
+  const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * prep_occ);
   if (p.seqlen_q_pad != p.seqlen_q) {
     // padding entries of the {lse, Delta} pairs are read by full-tile loads
     e = cudaMemsetAsync(p.ld, 0, (size_t)p.batch * p.heads_q * p.seqlen_q_pad * 16, stream);
     if (e != cudaSuccess) return e;
   }
-  // dV and G_k are sums over the pieces of each kv tile
-  e = cudaMemsetAsync(p.dvacc, 0, (size_t)p.batch * p.seqlen_kv * p.heads_kv * D * sizeof(float), stream);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(p.dkacc, 0, (size_t)p.batch * p.seqlen_kv * p.heads_kv * D * sizeof(float), stream);
-  if (e != cudaSuccess) return e;
   bca_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = launch_knorm(p.k, p.kn, (int64_t)p.batch * p.seqlen_kv * p.heads_kv, D, p.eps, stream);
   if (e != cudaSuccess) return e;
   if (n_units > 0) {
     bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, alloc);
@@ -718,7 +749,7 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
     if (e != cudaSuccess) return e;
   }
   const int64_t frows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
-  const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * 8);
+  const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * fin_occ);
   bca_bwd_finalize_kernel<D><<<fin_blocks, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -429,34 +429,10 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 template <int D>
 __global__ void __launch_bounds__(256) bca_knorm_kernel(const uint16_t* __restrict__ k, uint16_t* __restrict__ kn,
                                                          int64_t rows, float eps) {
-  constexpr int E = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const uint16_t* src = k + r * D + lane * E;
-    float x[E];
-    if constexpr (E == 4) {
-      const uint2 w = *reinterpret_cast<const uint2*>(src);
-      x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-    } else {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
-      x[0] = bf16_lo(w); x[1] = bf16_hi(w);
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rk = rms_inv<D>(ss, eps);
-    if constexpr (E == 4) {
-      uint2 w;
-      w.x = pack_bf16x2(x[0] * rk, x[1] * rk);
-      w.y = pack_bf16x2(x[2] * rk, x[3] * rk);
-      *reinterpret_cast<uint2*>(kn + r * D + lane * E) = w;
-    } else {
-      *reinterpret_cast<uint32_t*>(kn + r * D + lane * E) = pack_bf16x2(x[0] * rk, x[1] * rk);
-    }
-  }
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps)
+    knorm_row<D>(k + r * D, kn + r * D, lane, eps);
 }
 
 cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream) {

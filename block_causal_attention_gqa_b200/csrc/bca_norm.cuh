@@ -93,6 +93,36 @@ __device__ __forceinline__ float rms_inv(float sumsq, float eps) {
   return rsqrtf(sumsq * (1.0f / D) + eps);
 }
 
+// One key row: dst = bf16(src * r_k), r_k = 1 / RMS(src), by one warp (lane
+// holds features [lane*D/32, lane*D/32 + D/32)).  The forward's key pre-pass
+// and the backward's prep both call this, so both see the same K^ bits.
+template <int D>
+__device__ __forceinline__ void knorm_row(const uint16_t* src, uint16_t* dst, int lane, float eps) {
+  constexpr int E = D / 32;
+  float x[E];
+  if constexpr (E == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src + lane * E);
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  } else {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(src + lane * E);
+    x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rk = rms_inv<D>(ss, eps);
+  if constexpr (E == 4) {
+    uint2 w;
+    w.x = sm100::pack_bf16x2(x[0] * rk, x[1] * rk);
+    w.y = sm100::pack_bf16x2(x[2] * rk, x[3] * rk);
+    *reinterpret_cast<uint2*>(dst + lane * E) = w;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst + lane * E) = sm100::pack_bf16x2(x[0] * rk, x[1] * rk);
+  }
+}
+
 // The forward's query operand for one 16-byte chunk (8 features starting at d0):
 // bf16(q * r_q * qscale[d]) with qscale = gamma_q * gamma_k * softmax_scale * log2(e).
 __device__ __forceinline__ uint4 fold_q_chunk(uint4 v, float rq, const float* qscale, int d0) {

@@ -373,9 +373,9 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         mma_bf16_ss(tmem + d, ext_a, ext_b, id_kk, true);
       };
       bool ok = mbar_wait(&bars->kv_full, 0, p.status, kErrKv);
-      // Issue order per step t: dQ~(t) | dK~(t), dV(t) | dP(t+1), S(t+1), so the
-      // next step's products queue right behind this step's without waiting
-      // for the issuing thread.
+      // Issue order per step t: dK~/dV (queries 0..63) | dK~/dV (64..127), G_q |
+      // S^T(t+1) | dP^T(t+1), so the next step's products queue right behind
+      // this step's without waiting for the issuing thread.
       if (ok && n_steps > 0) {
         ok = mbar_wait(&bars->q_full[0], 0, p.status, kErrQFull);
         if (ok) {
@@ -434,7 +434,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
   } else {
     // ------------------------------------------------------------ compute warpgroups
-    const int wg = warp >> 2;               // owns query columns [32 wg, 32 wg + 32)
+    const int wg = warp >> 2;               // query columns [16 wg, +16) of each 64-column half
     const int j = threadIdx.x & 127;        // key row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int bar_id = 1 + wg;

@@ -29,13 +29,17 @@
 // tiles.  The result is exact: O and l are always scaled by the same factor.
 //
 // Throughput of the softmax: the row is processed as fp32 pairs with the
-// .f32x2 instructions, and on unmasked tiles one exponential in four is
-// computed by a cubic on the FMA pipe instead of MUFU (exp2_poly_pair), so
-// MUFU time per tile stays below the other sub-tile's MMA time.
+// .f32x2 instructions, the row maximum with three-input max, and on unmasked
+// tiles one exponential in four is computed by a cubic on the FMA pipe
+// instead of MUFU (exp2_poly_pair).  The masked and unmasked exponential
+// loops are separate straight-line code: a per-pair branch on the mask flag
+// split the loop into small blocks the compiler could not interleave, which
+// had made the exponential phase three times its MUFU time.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "bca_kernels.h"
 #include "bca_norm.cuh"
@@ -314,15 +318,22 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // row maximum as a tree (short dependency chains)
           float mx[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) f2_unpack(x2[i], mx[2 * i], mx[2 * i + 1]);
+          for (int i = 0; i < 4; ++i) {
+            float a0, a1, b0, b1;
+            f2_unpack(x2[i], a0, a1);
+            f2_unpack(x2[4 + i], b0, b1);
+            mx[2 * i] = fmaxf(a0, b0);
+            mx[2 * i + 1] = fmaxf(a1, b1);
+          }
 #pragma unroll
-          for (int c = 4; c < 64; c += 4)
+          for (int c = 8; c < 64; c += 8)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              float a0, a1;
+              float a0, a1, b0, b1;
               f2_unpack(x2[c + i], a0, a1);
-              mx[2 * i] = fmaxf(mx[2 * i], a0);
-              mx[2 * i + 1] = fmaxf(mx[2 * i + 1], a1);
+              f2_unpack(x2[c + 4 + i], b0, b1);
+              mx[2 * i] = fmax3(mx[2 * i], a0, b0);
+              mx[2 * i + 1] = fmax3(mx[2 * i + 1], a1, b1);
             }
           const float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
@@ -335,27 +346,36 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           const uint64_t negm = f2_pack(-m_ref, -m_ref);
           uint64_t ls2[4] = {0, 0, 0, 0};
+          // P = exp2(S - m) -> bf16 pairs in TMEM.  The two variants are
+          // separate straight-line loops (no per-pair branch), so the
+          // compiler can interleave the exponentials of many pairs.
+          auto exp_row = [&](auto use_poly) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
+            for (int c = 0; c < 4; ++c) {
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const uint64_t a2 = f2_add(x2[c * 16 + i], negm);
-              float p0, p1;
-              if ((i & 3) == 3 && !masked) {
-                exp2_poly_pair(a2, p0, p1);
-              } else {
-                float a0, a1;
-                f2_unpack(a2, a0, a1);
-                p0 = fast_exp2(a0);
-                p1 = fast_exp2(a1);
+              for (int i = 0; i < 16; ++i) {
+                const uint64_t a2 = f2_add(x2[c * 16 + i], negm);
+                float p0, p1;
+                if (decltype(use_poly)::value && (i & 3) == 3) {
+                  exp2_poly_pair(a2, p0, p1);
+                } else {
+                  float a0, a1;
+                  f2_unpack(a2, a0, a1);
+                  p0 = fast_exp2(a0);
+                  p1 = fast_exp2(a1);
+                }
+                const uint64_t p2 = f2_pack(p0, p1);
+                ls2[i & 3] = f2_add(ls2[i & 3], p2);
+                pk[i] = pack_bf16x2(p0, p1);
               }
-              const uint64_t p2 = f2_pack(p0, p1);
-              ls2[i & 3] = f2_add(ls2[i & 3], p2);
-              pk[i] = pack_bf16x2(p0, p1);
+              tmem_st16(t_s + c * 16, pk);
             }
-            tmem_st16(t_s + c * 16, pk);
-          }
+          };
+          if (masked)
+            exp_row(std::false_type{});
+          else
+            exp_row(std::true_type{});
           {
             float s[8];
 #pragma unroll

@@ -27,7 +27,8 @@
 //                                          reduce-adds into the fp32 accumulator
 //                The -lse and -Delta terms come out of the tensor core: one extra
 //                K-step of 16 multiplies constant rows (1 at the pieces' k) by the
-//                pieces, so the softmax only computes exp2 and one product.
+//                pieces, so the softmax only computes exp2 (one pair in four by
+//                a cubic on the FMA pipe, off MUFU) and one product.
 //                At the end the CTA adds dV and G_k into fp32 accumulators (long
 //                query ranges are split into pieces, so several CTAs may add to
 //                one kv tile).
@@ -479,7 +480,14 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           if (!diag) {
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const float p0 = fast_exp2(__uint_as_float(sr[c])), p1 = fast_exp2(__uint_as_float(sr[c + 1]));
+              // one pair in four on the FMA pipe (cubic), the rest on MUFU
+              float p0, p1;
+              if (((c >> 1) & 3) == 3) {
+                exp2_poly_pair(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), p0, p1);
+              } else {
+                p0 = fast_exp2(__uint_as_float(sr[c]));
+                p1 = fast_exp2(__uint_as_float(sr[c + 1]));
+              }
               float d0, d1;
               f2_unpack(f2_mul(f2_pack(__uint_as_float(dpr[c]), __uint_as_float(dpr[c + 1])), f2_pack(p0, p1)), d0, d1);
               pk[c >> 1] = pack_bf16x2(p0, p1);

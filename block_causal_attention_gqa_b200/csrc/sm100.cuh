@@ -400,6 +400,30 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^a for a pair, a <= 8.5: j = round(a) via the 1.5*2^23 rounding constant,
+// f = a - j in [-1/2, 1/2], 2^f by a minimax cubic (relative error 7.5e-5,
+// fitted by fit_exp2_poly.py in the package), and 2^j added to the exponent bits.  Inputs
+// below -125 are clamped there (results ~1e-38 instead of smaller); callers
+// use it only where no element is masked to -inf.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t a2, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float a0, a1;
+  f2_unpack(a2, a0, a1);
+  a2 = f2_pack(fmaxf(a0, -125.f), fmaxf(a1, -125.f));
+  const uint64_t t2 = f2_add(a2, f2_pack(kRound, kRound));
+  const uint64_t j2 = f2_add(t2, f2_pack(-kRound, -kRound));
+  const uint64_t fr = f2_fma(j2, f2_pack(-1.f, -1.f), a2);
+  uint64_t q = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), fr,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  q = f2_fma(q, fr, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  q = f2_fma(q, fr, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float t0, t1, q0, q1;
+  f2_unpack(t2, t0, t1);
+  f2_unpack(q, q0, q1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));

@@ -20,7 +20,8 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 
 __all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_noalloc", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
-           "magi_bca_status_string", "magi_bca_last_device_status", "MagiBcaError", "Dims", "library",
+           "magi_bca_status_string", "magi_bca_last_device_status", "magi_bca_profile_events", "MagiBcaError",
+           "Dims", "library",
            "library_path", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,8 @@ library_path = os.path.join(_HERE, "libmagi_bca.so")
 
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
-                    "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule"]
+                    "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule",
+                    "magi_bca_profile_events"]
 
 
 class MagiBcaError(RuntimeError):
@@ -83,6 +85,8 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_bwd_schedule.restype = ctypes.c_int64
     lib.magi_bca_version.argtypes = []
     lib.magi_bca_version.restype = ctypes.c_char_p
+    lib.magi_bca_profile_events.argtypes = [vp, vp]
+    lib.magi_bca_profile_events.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -93,6 +97,23 @@ def magi_bca_status_string(status: int) -> str:
 
 def magi_bca_last_device_status() -> int:
     return int(library().magi_bca_last_device_status())
+
+
+def magi_bca_profile_events(begin=None, end=None) -> None:
+    """Diagnostic: while set, each forward/backward call records the two
+    events (torch.cuda.Event with timing enabled, or raw cudaEvent_t handles)
+    around its main kernel's launch.  ``magi_bca_profile_events()`` clears."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if hasattr(ev, "cuda_event"):
+            if ev.cuda_event == 0:   # torch creates the CUDA event on its first record
+                ev.record()
+            return ev.cuda_event
+        return int(ev)
+    st = library().magi_bca_profile_events(handle(begin), handle(end))
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_profile_events")
 
 
 def _offsets(x) -> np.ndarray:

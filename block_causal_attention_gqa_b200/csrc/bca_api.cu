@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -19,6 +20,14 @@ namespace magi {
 
 // Device status word written by bounded waits that give up (0 = fine).
 __device__ int g_device_status;
+
+// Diagnostic timing events (magi_bca_profile_events); null when unset.
+std::atomic<void*> g_profile_begin{nullptr}, g_profile_end{nullptr};
+
+void profile_mark(int which, cudaStream_t stream) {
+  void* ev = which == 0 ? g_profile_begin.load() : g_profile_end.load();
+  if (ev != nullptr) cudaEventRecord(static_cast<cudaEvent_t>(ev), stream);
+}
 
 namespace {
 
@@ -217,6 +226,13 @@ extern "C" {
 
 const char* magi_bca_version(void) { return "magi_bca 0.1 (sm_100a)"; }
 
+int magi_bca_profile_events(void* event_begin, void* event_end) {
+  if ((event_begin == nullptr) != (event_end == nullptr)) return MAGI_BCA_INVALID_ARG;
+  magi::g_profile_begin.store(event_begin);
+  magi::g_profile_end.store(event_end);
+  return MAGI_BCA_OK;
+}
+
 const char* magi_bca_status_string(int status) {
   switch (status) {
     case MAGI_BCA_OK: return "ok";
@@ -303,7 +319,9 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.scale_log2 = resolve_scale(d) * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = ds->status;
+  profile_mark(0, cs);
   cudaError_t e = launch_fwd(tq, tk, tv, p, d.head_dim, sched.n_units, cs);
+  profile_mark(1, cs);
   return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("forward launch", e);
 }
 

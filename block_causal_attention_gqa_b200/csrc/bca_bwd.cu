@@ -751,11 +751,13 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   bca_bwd_prep_kernel<D><<<prep_blocks, 256, 0, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  profile_mark(0, stream);
   if (n_units > 0) {
     bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, alloc);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  profile_mark(1, stream);
   const int64_t frows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
   const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * fin_occ);
   bca_bwd_finalize_kernel<D><<<fin_blocks, 256, 0, stream>>>(p);

@@ -75,6 +75,10 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int head_dim, int n_units, cudaStream_t stream);
 size_t fwd_smem_bytes(int head_dim);
 
+// Records the diagnostic timing events (magi_bca_profile_events) on `stream`:
+// which = 0 before a main-kernel launch, 1 after it.  No-op when unset.
+void profile_mark(int which, cudaStream_t stream);
+
 // Shared host helpers (bca_api.cu).
 int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 float resolve_softmax_scale(const magi_bca_dims& d);

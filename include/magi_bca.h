@@ -149,6 +149,17 @@ const char* magi_bca_last_error_detail(void);
  * Meant for tests and diagnostics, not for the hot path. */
 int magi_bca_last_device_status(void);
 
+/* Diagnostic timing hook (the paper has no counterpart).  `event_begin` and
+ * `event_end` are cudaEvent_t handles created by the caller.  While both are
+ * non-NULL, every magi_bca_fwd / magi_bca_bwd / magi_bca_bwd_noalloc call
+ * records event_begin on its stream immediately before launching its main
+ * kernel (bca_fwd_kernel or bca_bwd_main_kernel) and event_end immediately
+ * after, so the caller can time that kernel alone with cudaEventElapsedTime.
+ * Pass NULL, NULL to stop.  Process-wide setting; not for concurrent calls on
+ * several streams.  Returns MAGI_BCA_OK, or MAGI_BCA_INVALID_ARG if exactly
+ * one handle is NULL. */
+int magi_bca_profile_events(void* event_begin, void* event_end);
+
 /* Host-only view of the tile schedule the kernels run (no device needed).
  * A work unit is up to two 128-row query tiles ("sub-tiles") that read the
  * same key/value head and visit the same kv tiles, so every K/V tile the

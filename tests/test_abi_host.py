@@ -263,3 +263,10 @@ def test_bwd_schedule_balances_the_sms():
     # a problem with far more work than SMs is left in whole kv tiles
     big = check_bwd_schedule([5760] * 8, [5760] * 8, 1, 24, 8)
     assert len(big) == 8 * 360
+
+
+def test_profile_events_argument_check():
+    lib = bca.library()
+    assert lib.magi_bca_profile_events(256, None) == INVALID_ARG
+    assert lib.magi_bca_profile_events(None, 256) == INVALID_ARG
+    assert lib.magi_bca_profile_events(None, None) == OK

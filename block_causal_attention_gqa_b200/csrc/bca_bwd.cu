@@ -566,10 +566,10 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tma_store_commit();   // (an empty group when nothing was issued); released next step
       }
     }
-    // every bulk reduction complete (and the last stage released) before the
-    // stage buffers are reused below
+    // every bulk reduction has read its staging (and the last stage is
+    // released) before the stage buffers are reused below
     if (j == 0) {
-      tma_store_wait_all();
+      tma_store_wait_read();
       if (ok && n_steps > 0) mbar_arrive(&bars->q_empty[(n_steps - 1) & 1]);
     }
     named_bar_sync(5, 128 * kComputeWarpgroups);
@@ -602,7 +602,9 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       tma_reduce_add_4d(&tm_dv, smem + L::kQn + wg * 16384, wg * 32, hk, n0, b);
       tma_reduce_add_4d(&tm_dk, smem + L::kDo + wg * 16384, wg * 32, hk, n0, b);
       tma_store_commit();
-      tma_store_wait_all();
+      // the reductions only need to have read shared memory before the CTA
+      // exits; their global writes complete before the kernel does
+      tma_store_wait_read();
     }
   }
 
@@ -620,7 +622,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // G_k / log2(e), dk through the Jacobian, dgamma_k += dk~ k^.  With r = rsqrt
 // (mean x^2 + eps), x^ = x r and g = gamma dx~:  dx = r (g - x^ mean(g x^)).
 template <int D>
-__global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(256, 4) bca_bwd_finalize_kernel(const BwdParams p) {
   using IO = RowIO<D>;
   constexpr int E = IO::E;
   __shared__ float red[2][8][D];

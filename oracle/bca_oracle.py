@@ -24,6 +24,11 @@ folding of scales):
    ``n_kv - n_q + c``: the query chunks are the last ``n_q`` chunks of the
    key/value sequence (streaming layout: active chunks after the cached clean
    chunks, MAGI-1 §2 and §2.4.4; identity when n_q == n_kv).
+   Optional KV range R (MAGI-1 §2.4.4 and §2.6, Fig. 12: "restricting the KV
+   range to preceding content"; KV range 1 means no access to earlier video
+   content): with R > 0 the kv chunk index must also be at least
+   ``n_kv - n_q + c - R + 1``, so a chunk sees itself and the R - 1 chunks
+   before it; R = 0 means no limit.
 4. Softmax attention with scale ``1/sqrt(D)`` (a reading: the pages give no
    scale), ``O = softmax(scale * q~ k~^T + mask) v``; the log-sum-exp
    ``lse = ln sum_j exp(scale * q~_i . k~_j)`` over unmasked j, natural log, in
@@ -99,10 +104,12 @@ def matched_kv_chunk(q_chunk, n_q_chunks, n_kv_chunks):
     return n_kv_chunks - n_q_chunks + np.asarray(q_chunk)
 
 
-def block_causal_mask(q_offsets, kv_offsets, rows=None):
+def block_causal_mask(q_offsets, kv_offsets, rows=None, kv_range=0):
     """Boolean mask M[i, j]: query token i may attend key token j.
 
-    Built token by token from chunk ids, not from tile arithmetic."""
+    Built token by token from chunk ids, not from tile arithmetic.  With
+    ``kv_range`` R > 0, key chunks more than R - 1 chunks before the query's
+    own kv chunk are masked as well."""
     q_offsets = np.asarray(q_offsets)
     kv_offsets = np.asarray(kv_offsets)
     nq, nkv = len(q_offsets) - 1, len(kv_offsets) - 1
@@ -110,7 +117,11 @@ def block_causal_mask(q_offsets, kv_offsets, rows=None):
     ck = chunk_of(kv_offsets, int(kv_offsets[-1]))
     if rows is not None:
         cq = cq[np.asarray(rows)]
-    return ck[None, :] <= matched_kv_chunk(cq, nq, nkv)[:, None]
+    own = matched_kv_chunk(cq, nq, nkv)[:, None]
+    m = ck[None, :] <= own
+    if kv_range and kv_range > 0:
+        m &= ck[None, :] >= own - (int(kv_range) - 1)
+    return m
 
 
 def torch_index(rows):
@@ -144,7 +155,7 @@ def _attend_rows(qn_rows, kn, vv, mask_rows, scale):
 
 
 def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=None,
-                 batches=None, scale=None, eps=DEFAULT_EPS, block=None):
+                 batches=None, scale=None, eps=DEFAULT_EPS, block=None, kv_range=0):
     """Forward on a subset of query rows.
 
     ``rows`` is an int array of query-token indices; ``heads`` / ``batches``
@@ -175,22 +186,22 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
             for r0 in range(0, len(rows), block):
                 rr = rows[r0:r0 + block]
                 qn = rms_norm(qsel[b, r0:r0 + block, h, :], gamma_q, eps)
-                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
                 o, ls, _ = _attend_rows(qn, kn, vv, mask, scale)
                 out[bi, r0:r0 + len(rr), hi, :] = o
                 lse[bi, hi, r0:r0 + len(rr)] = ls
     return out, lse
 
 
-def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS):
+def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS, kv_range=0):
     """Full forward.  Returns (out [B, Sq, Hq, D], lse [B, Hq, Sq]), float64."""
     Sq = q.shape[1]
     return forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k,
-                        rows=np.arange(Sq), scale=scale, eps=eps)
+                        rows=np.arange(Sq), scale=scale, eps=eps, kv_range=kv_range)
 
 
 def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
-             eps=DEFAULT_EPS):
+             eps=DEFAULT_EPS, kv_range=0):
     """Full analytic backward in float64.
 
     Returns dict(dq, dk, dv, dgamma_q, dgamma_k, out, lse); dq/dk are the
@@ -206,7 +217,7 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
     B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
     scale = 1.0 / np.sqrt(D) if not scale else float(scale)
     group = Hq // Hkv
-    mask = block_causal_mask(q_offsets, kv_offsets)
+    mask = block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range)
     dqn = np.zeros_like(q)
     dkn = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -237,7 +248,7 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
 
 def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows=None,
                   kv_rows=None, kv_heads=None, batches=None, scale=None, eps=DEFAULT_EPS,
-                  block=None):
+                  block=None, kv_range=0):
     """Exact backward on chosen rows, without a full backward.
 
     * dq of query rows ``q_rows`` (all heads): needs only those rows' P, dP
@@ -274,7 +285,7 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
             kn_all = rms_norm(k[b], gk, eps)
             for r0 in range(0, len(q_rows), block):
                 rr = q_rows[r0:r0 + block]
-                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
                 dqn = np.zeros((len(rr), Hq, D))
                 for h in range(Hq):
                     hk = h // group
@@ -294,10 +305,7 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
         dk = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         dv = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         # every query row that sees at least one of the requested keys
-        cq = chunk_of(q_offsets, Sq)
-        ck = chunk_of(kv_offsets, Skv)
-        nq, nkv = len(q_offsets) - 1, len(kv_offsets) - 1
-        seeing = np.nonzero(matched_kv_chunk(cq, nq, nkv) >= ck[kv_rows].min())[0]
+        seeing = np.nonzero(block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range)[:, kv_rows].any(axis=1))[0]
         qsel, dsel = take(q, seeing), take(dout, seeing)
         for bi, b in enumerate(batches):
             kn_all = rms_norm(k[b], gk, eps)
@@ -309,7 +317,7 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                     for r0 in range(0, len(seeing), block):
                         rr = seeing[r0:r0 + block]
                         qn = rms_norm(qsel[b, r0:r0 + block, h, :], gq, eps)
-                        mask = block_causal_mask(q_offsets, kv_offsets, rows=rr)
+                        mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
                         o, _, p = _attend_rows(qn, kn, vv, mask, scale)
                         g = dsel[b, r0:r0 + block, h, :]
                         delta = np.sum(g * o, axis=1, keepdims=True)

@@ -47,10 +47,12 @@ def read_mask_fixture(name):
 
 # ---------------------------------------------------------------- the mask
 
-@pytest.mark.parametrize("name", ["mask_train_2_1_3.txt", "mask_stream_2of3.txt"])
+@pytest.mark.parametrize("name", ["mask_train_2_1_3.txt", "mask_stream_2of3.txt",
+                                  "mask_kvrange2_train_2_1_2_1.txt", "mask_kvrange3_stream_2of4.txt"])
 def test_mask_matches_hand_written_fixture(name):
     meta, want = read_mask_fixture(name)
-    got = orc.block_causal_mask(offs(meta["q_chunks"]), offs(meta["kv_chunks"]))
+    got = orc.block_causal_mask(offs(meta["q_chunks"]), offs(meta["kv_chunks"]),
+                                kv_range=meta.get("kv_range", [0])[0])
     assert got.shape == want.shape
     assert np.array_equal(got, want)
 
@@ -362,3 +364,94 @@ def test_backward_structure_and_identities():
     np.testing.assert_allclose(g2["dk"][:, 4:], g["dk"][:, 4:], rtol=0, atol=1e-13)
     np.testing.assert_allclose(g2["dv"][:, 4:], g["dv"][:, 4:], rtol=0, atol=1e-13)
     assert not np.allclose(g2["dk"][:, :4], g["dk"][:, :4])
+
+
+# ---------------------------------------------------------------- KV range
+
+def test_kv_range_one_is_full_attention_inside_each_chunk():
+    """KV range 1 (no access to earlier chunks) = independent bidirectional
+    attention per chunk, computed by torch SDPA without a mask."""
+    rng = np.random.default_rng(31)
+    lens = [5, 9, 3, 7]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, lens, lens, 4, 2, 16)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=1)
+    for c in range(len(lens)):
+        sl = slice(qo[c], qo[c + 1])
+        n = lens[c]
+        want = torch_reference(q[:, sl], k[:, sl], v[:, sl], offs([n]), offs([n]), gq, gk,
+                               mask=torch.ones(n, n, dtype=torch.bool))
+        np.testing.assert_allclose(o[:, sl], want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("R", [1, 2, 5])
+def test_kv_range_on_unit_chunks_is_sliding_window_causal_attention(R):
+    """One-token chunks with KV range R: token i sees tokens i-R+1 .. i, the
+    textbook sliding-window causal mask (built here with torch band ops)."""
+    rng = np.random.default_rng(32 + R)
+    n = 19
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [1] * n, [1] * n, 2, 1, 8)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=R)
+    ones = torch.ones(n, n, dtype=torch.bool)
+    band = ones.tril() & ones.triu(-(R - 1))
+    np.testing.assert_allclose(o, torch_reference(q, k, v, qo, ko, gq, gk, mask=band), rtol=0, atol=1e-12)
+
+
+def test_kv_range_covering_every_chunk_changes_nothing():
+    rng = np.random.default_rng(33)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [4, 6], [3, 5, 4, 6], 4, 2, 8)
+    o0, l0 = orc.forward(q, k, v, qo, ko, gq, gk)
+    for R in (4, 5, 100):
+        o, l = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=R)
+        assert np.array_equal(o, o0) and np.array_equal(l, l0)
+    o3, _ = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=3)
+    assert not np.allclose(o3, o0)   # the first active chunk loses kv chunk 0
+
+
+def test_kv_outside_every_window_does_not_change_outputs():
+    rng = np.random.default_rng(34)
+    lens = [4, 5, 6, 3]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 4, 2, 8)
+    o1, l1 = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=2)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :4] += rng.standard_normal(k2[:, :4].shape)   # chunk 0: outside the windows of chunks 2 and 3
+    v2[:, :4] += 1.0
+    o2, l2 = orc.forward(q, k2, v2, qo, ko, gq, gk, kv_range=2)
+    late = slice(qo[2], qo[4])
+    assert np.array_equal(o1[:, late], o2[:, late]) and np.array_equal(l1[..., late], l2[..., late])
+    assert not np.allclose(o1[:, :qo[2]], o2[:, :qo[2]])
+
+
+def test_kv_range_backward_matches_central_finite_differences():
+    rng = np.random.default_rng(35)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [2, 1, 2], [2, 1, 2], 2, 1, 4)
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk, kv_range=2)
+    params = [q, k, v, gq, gk]
+    h = 1e-6
+    for pi, name in enumerate(["dq", "dk", "dv", "dgamma_q", "dgamma_k"]):
+        base = params[pi]
+        num = np.zeros_like(base)
+        it = np.nditer(base, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            pp = [p.copy() for p in params]
+            pp[pi][idx] += h
+            lp = float(np.sum(orc.forward(*pp[:3], qo, ko, *pp[3:], kv_range=2)[0] * do))
+            pp[pi][idx] -= 2 * h
+            lm = float(np.sum(orc.forward(*pp[:3], qo, ko, *pp[3:], kv_range=2)[0] * do))
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_kv_range_backward_rows_match_full_backward():
+    rng = np.random.default_rng(36)
+    lens = [5, 4, 6, 3]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 4, 2, 8)
+    do = rng.standard_normal(q.shape)
+    full = orc.backward(q, k, v, do, qo, ko, gq, gk, kv_range=2)
+    rows = np.array([0, 4, 9, 12, 17])
+    kv_rows = np.array([1, 6, 10, 16])
+    part = orc.backward_rows(q, k, v, do, qo, ko, gq, gk, q_rows=rows, kv_rows=kv_rows, kv_range=2)
+    np.testing.assert_allclose(part["dq"][0], full["dq"][0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dk"][0], full["dk"][0, kv_rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dv"][0], full["dv"][0, kv_rows], rtol=0, atol=1e-12)

@@ -36,18 +36,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------ work model
-def row_kv_ends(w):
-    """Visible-key end of every query row (query chunk c = kv chunk n_kv - n_q + c)."""
+def row_visible_keys(w):
+    """Visible keys of every query row: query chunk c is kv chunk c' = n_kv - n_q + c
+    and sees kv chunks [c' - R + 1, c'] under a KV range R, else [0, c']."""
     qo, ko = w.q_offsets, w.kv_offsets
     nq, nkv = len(qo) - 1, len(ko) - 1
-    ends = np.empty(w.seqlen_q, np.int64)
+    n = np.empty(w.seqlen_q, np.int64)
     for c in range(nq):
-        ends[qo[c]:qo[c + 1]] = ko[nkv - nq + c + 1]
-    return ends
+        own = nkv - nq + c
+        first = max(own - w.kv_range + 1, 0) if w.kv_range > 0 else 0
+        n[qo[c]:qo[c + 1]] = ko[own + 1] - ko[first]
+    return n
 
 
 def fwd_flops(w):
-    return 4.0 * w.head_dim * w.batch * w.heads_q * float(row_kv_ends(w).sum())
+    return 4.0 * w.head_dim * w.batch * w.heads_q * float(row_visible_keys(w).sum())
 
 
 def bwd_flops(w):
@@ -214,14 +217,15 @@ def run_ours(args, w, world, rank, local):
             ev[0].record(stream)
         if kev is not None and not do_bwd:
             bca.magi_bca_profile_events(kev[0], kev[1])
-        bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, out=out, lse=lse, stream=stream)
+        bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, out=out, lse=lse, stream=stream,
+                         kv_range=w.kv_range)
         if ev is not None:
             ev[1].record(stream)
         if do_bwd:
             if kev is not None:
                 bca.magi_bca_profile_events(kev[0], kev[1])
             bca.magi_bca_bwd(q, k, v, out, inp["dout"], lse, w.q_offsets, w.kv_offsets, gq, gk, dq=dq, dk=dk,
-                             dv=dv, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream)
+                             dv=dv, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range)
             if ev is not None:
                 ev[2].record(stream)
         if kev is not None:
@@ -303,11 +307,11 @@ def run_ours(args, w, world, rank, local):
         if i >= 2:
             stream.wait_event(ev_out[n])               # step i-2's results are out of this set
         bca.magi_bca_fwd(b["q"], b["k"], b["v"], w.q_offsets, w.kv_offsets, gq, gk, out=b["out"], lse=b["lse"],
-                         stream=stream)
+                         stream=stream, kv_range=w.kv_range)
         if do_bwd:
             bca.magi_bca_bwd(b["q"], b["k"], b["v"], b["out"], b["dout"], b["lse"], w.q_offsets, w.kv_offsets,
                              gq, gk, dq=b["dq"], dk=b["dk"], dv=b["dv"], dgamma_q=dgq, dgamma_k=dgk, workspace=ws,
-                             stream=stream)
+                             stream=stream, kv_range=w.kv_range)
         ev_done[n].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[n])
@@ -383,7 +387,8 @@ def run_ours(args, w, world, rank, local):
         "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
                    "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
                    "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
-                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "parallelism": f"replicas x{world}",
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range,
+                   "parallelism": f"replicas x{world}",
                    "l2": "flushed (512 MB write) between timed steps, outside the step events",
                    "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4) if do_bwd else None,
                    "useful_tflop_per_step": round(flops_step / 1e12, 4)},
@@ -412,15 +417,15 @@ def oracle_sample(w, inp, rows, do_bwd):
     """Runs the oracle on the given query rows (all heads, batch 0)."""
     from oracle import bca_oracle as orc
     orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
-                     inp["gamma_k"], rows, batches=[0])
+                     inp["gamma_k"], rows, batches=[0], kv_range=w.kv_range)
     if do_bwd:
         orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0])
+                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0], kv_range=w.kv_range)
 
 
 def sample_flops(w, rows, do_bwd):
-    ends = row_kv_ends(w)[rows]
-    f = 4.0 * w.head_dim * w.heads_q * float(ends.sum())
+    keys = row_visible_keys(w)[rows]
+    f = 4.0 * w.head_dim * w.heads_q * float(keys.sum())
     return f * (1 + (2.5 if do_bwd else 0.0))
 
 

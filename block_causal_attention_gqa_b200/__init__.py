@@ -46,7 +46,7 @@ class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("seqlen_q", ctypes.c_int32), ("seqlen_kv", ctypes.c_int32),
                 ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("n_q_chunks", ctypes.c_int32), ("n_kv_chunks", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("kv_range", ctypes.c_int32)]
 
 
 _lib = None
@@ -130,9 +130,9 @@ def _i32p(a: np.ndarray):
 
 
 def make_dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-              softmax_scale=0.0, rms_eps=1e-6) -> Dims:
+              softmax_scale=0.0, rms_eps=1e-6, kv_range=0) -> Dims:
     return Dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-                float(softmax_scale), float(rms_eps))
+                float(softmax_scale), float(rms_eps), int(kv_range))
 
 
 def _check_bf16(name, t, shape=None):
@@ -163,7 +163,8 @@ def _stream_handle(stream, device):
 
 
 def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out=None, lse=None,
-                 softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True):
+                 softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True,
+                 kv_range: int = 0):
     """Forward.  q [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] bf16; gammas fp32 [D];
     offsets: host int arrays of chunk boundaries.  Returns (out, lse)."""
     import torch
@@ -183,7 +184,7 @@ def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, o
         lse = torch.empty(B, Hq, Sq, device=q.device, dtype=torch.float32)
     if lse is not None:
         _check_f32("lse", lse, (B, Hq, Sq))
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
     with torch.cuda.device(q.device):
         st = library().magi_bca_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _i32p(qo), _i32p(ko),
                                     gamma_q.data_ptr(), gamma_k.data_ptr(), out.data_ptr(),
@@ -200,7 +201,8 @@ def magi_bca_bwd_workspace_size(dims: Dims) -> int:
 
 def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                  dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
-                 workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None):
+                 workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
+                 kv_range: int = 0):
     """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
     respect to the raw (pre-norm) q and k."""
     import torch
@@ -215,7 +217,7 @@ def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gam
     _check_f32("gamma_q", gamma_q, (D,))
     _check_f32("gamma_k", gamma_k, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -243,7 +245,7 @@ def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gam
 
 def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                          dq, dk, dv, dgamma_q=None, dgamma_k=None, softmax_scale: float = 0.0,
-                         rms_eps: float = 1e-6, stream=None):
+                         rms_eps: float = 1e-6, stream=None, kv_range: int = 0):
     """Backward through the allocation-free entry point.
 
     For callers that cannot allocate device memory or hand the library a
@@ -265,7 +267,7 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
         if t is not None:
             _check_f32(nm, t, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
     import torch
     with torch.cuda.device(q.device):
         st = library().magi_bca_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -279,25 +281,28 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
     return dq, dk, dv, dgamma_q, dgamma_k
 
 
-def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim) -> np.ndarray:
-    """Host-only: the forward's work units as an int32 array [n_units, 8]."""
+def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
+                          kv_range=0) -> np.ndarray:
+    """Host-only: the forward's work units as an int32 array [n_units, 12]."""
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1)
+    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1,
+                     kv_range=kv_range)
     lib = library()
     n = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), None, 0)
     if n < 0:
         raise MagiBcaError(int(n), "magi_bca_fwd_schedule")
-    buf = np.zeros((max(n, 1), 8), dtype=np.int32)
+    buf = np.zeros((max(n, 1), 12), dtype=np.int32)
     n2 = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), _i32p(buf), n)
     assert n2 == n
     return buf[:n]
 
 
 def magi_bca_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
-                          num_sms=148) -> np.ndarray:
+                          num_sms=148, kv_range=0) -> np.ndarray:
     """Host-only: the backward's work units as an int32 array [n_units, 8]."""
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1)
+    dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1,
+                     kv_range=kv_range)
     lib = library()
     n = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, None, 0)
     if n < 0:

@@ -116,7 +116,7 @@ int device_state(int* device_out, DeviceState** st_out) {
 
 std::vector<int32_t> schedule_key(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko) {
   std::vector<int32_t> key = {dev, kind, d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim,
-                              d.n_q_chunks, d.n_kv_chunks};
+                              d.n_q_chunks, d.n_kv_chunks, d.kv_range};
   key.insert(key.end(), qo, qo + d.n_q_chunks + 1);
   key.insert(key.end(), ko, ko + d.n_kv_chunks + 1);
   return key;
@@ -136,7 +136,7 @@ int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, c
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d, sms);
   ScheduleEntry e;
-  e.n_units = static_cast<int>(units.size() / kUnitInts);
+  e.n_units = static_cast<int>(units.size() / (kind == 0 ? kFwdUnitInts : kUnitInts));
   std::vector<int32_t> blob = units;
   blob.insert(blob.end(), qo, qo + d.n_q_chunks + 1);
   blob.insert(blob.end(), ko, ko + d.n_kv_chunks + 1);
@@ -254,9 +254,9 @@ int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
   if (st != MAGI_BCA_OK) return st;
   if (capacity > 0 && units == nullptr) return MAGI_BCA_INVALID_ARG;
   std::vector<int32_t> s = build_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, *dims);
-  const int64_t n = (int64_t)(s.size() / kUnitInts);
+  const int64_t n = (int64_t)(s.size() / kFwdUnitInts);
   const int64_t w = n < capacity ? n : capacity;
-  if (w > 0) std::memcpy(units, s.data(), (size_t)w * kUnitInts * sizeof(int32_t));
+  if (w > 0) std::memcpy(units, s.data(), (size_t)w * kFwdUnitInts * sizeof(int32_t));
   return n;
 }
 
@@ -305,10 +305,11 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
     return MAGI_BCA_CUDA_ERROR;
   FwdParams p;
   p.units = sched.dev;
-  p.q_offsets = sched.dev + (size_t)sched.n_units * kUnitInts;
+  p.q_offsets = sched.dev + (size_t)sched.n_units * kFwdUnitInts;
   p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
+  p.kv_range = d.kv_range;
   p.gamma_q = gamma_q;
   p.gamma_k = gamma_k;
   p.out = out;
@@ -369,6 +370,7 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
+  p.kv_range = d.kv_range;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

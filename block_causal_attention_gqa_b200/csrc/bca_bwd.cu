@@ -260,8 +260,10 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int32_t* u = p.units + (size_t)blockIdx.x * 8;
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
   // steps [s_begin, s_end) of this kv tile; step s = (query tile s / group,
-  // head s % group of the kv head's group); query tiles below diag_end need the mask
+  // head s % group of the kv head's group); query tiles below diag_end or from
+  // diag_hi_begin on (KV range) need the mask
   const int s_begin = __ldg(u + 3), s_end = __ldg(u + 4), diag_end = __ldg(u + 5);
+  const int diag_hi_begin = __ldg(u + 6);
   const int group = p.heads_q / p.heads_kv;
   const int n_steps = s_end - s_begin;
 
@@ -454,6 +456,19 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
       }
     }
+    // First query row that no longer sees key n0 + j (KV range R): query chunk
+    // c's first visible key is kv_offsets[max(0, n_kv - n_q + c - R + 1)].
+    int row_max = p.seqlen_q;
+    if (p.kv_range > 0) {
+      const int key = n0 + j;
+      const int shift = p.n_kv_chunks - p.n_q_chunks - p.kv_range + 1;
+      int lo = 0, hi = p.n_q_chunks;  // first c with a first visible key above `key`
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.kv_offsets + max(shift + mid, 0)) > key) hi = mid; else lo = mid + 1;
+      }
+      row_max = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
+    }
     // G_q drain: warpgroup w owns G_q columns [32 w, 32 w + 32); with D = 64 only
     // warpgroups 0 and 1 have columns.  Staging chunks are [128 rows][32 floats]
     // with the 128-byte swizzle (16 KB) in this step's Q^ and dO stage buffers.
@@ -463,7 +478,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       const int st = t & 1;
       const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
       const int q0 = qt * 128;
-      const bool diag = qt < diag_end;
+      const bool diag = qt < diag_end || qt >= diag_hi_begin;
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
       // Warpgroup w owns query columns [16w, 16w+16) of each 64-column half:
       // the first half's dK~/dV products run while the second half is computed.
@@ -494,11 +509,12 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
               dk[c >> 1] = pack_bf16x2(d0, d1);
             }
           } else {
-            const int lim = row_min - (q0 + col0);   // columns c < lim cannot see key j
+            // columns c < lim and c >= hi_lim cannot see key j
+            const int lim = row_min - (q0 + col0), hi_lim = row_max - (q0 + col0);
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const float p0 = c < lim ? 0.f : fast_exp2(__uint_as_float(sr[c]));
-              const float p1 = c + 1 < lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]));
+              const float p0 = c < lim || c >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c]));
+              const float p1 = c + 1 < lim || c + 1 >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]));
               const float d0 = p0 * __uint_as_float(dpr[c]);
               const float d1 = p1 * __uint_as_float(dpr[c + 1]);
               pk[c >> 1] = pack_bf16x2(p0, p1);

@@ -109,11 +109,16 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int32_t* u = p.units + (size_t)blockIdx.x * 8;
+  const int32_t* u = p.units + (size_t)blockIdx.x * 12;
   const int b = __ldg(u + 0), hk = __ldg(u + 1);
   const int head0 = __ldg(u + 2), head1 = __ldg(u + 4);
   const int m00 = __ldg(u + 3), m01 = __ldg(u + 5);
   const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
+  // kv tiles [t_begin, n_tiles) are visited (t_begin > 0 only under a KV
+  // range); tiles below t_full_begin or from n_full on need the per-row mask.
+  // Loop indices below count visited tiles from 0: tile = t_begin + j.
+  const int t_begin = __ldg(u + 8), t_full_begin = __ldg(u + 9);
+  const int n_vis = n_tiles - t_begin;
   const int n_sub = head1 >= 0 ? 2 : 1;
 
   if (threadIdx.x == 0) {
@@ -155,19 +160,19 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tma_load_4d(smem + L::kQ + s * L::kTileBytes + box * 16384, &tm_q, &bars->q_full[s], box * 64,
                       s ? head1 : head0, s ? m01 : m00, b);
       }
-      for (int j = 0; j < n_tiles; ++j) {
+      for (int j = 0; j < n_vis; ++j) {
         const int st = j % kStages;
         const uint32_t par = ((j / kStages) & 1) ^ 1;
         if (!mbar_wait(&bars->k_empty[st], par, p.status, kErrKEmpty)) break;
         mbar_arrive_expect_tx(&bars->k_full[st], L::kTileBytes);
         for (int box = 0; box < D / 64; ++box)
           tma_load_4d(smem + L::kK + st * L::kTileBytes + box * 16384, &tm_k, &bars->k_full[st], box * 64, hk,
-                      j * 128, b);
+                      (t_begin + j) * 128, b);
         if (!mbar_wait(&bars->v_empty[st], par, p.status, kErrVEmpty)) break;
         mbar_arrive_expect_tx(&bars->v_full[st], L::kTileBytes);
         for (int box = 0; box < D / 64; ++box)
           tma_load_4d(smem + L::kV + st * L::kTileBytes + box * 16384, &tm_v, &bars->v_full[st], box * 64, hk,
-                      j * 128, b);
+                      (t_begin + j) * 128, b);
       }
     }
   } else if (warp == 8) {
@@ -198,10 +203,10 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         mma_commit(&bars->k_empty[0]);
       }
-      for (int j = 0; j < n_tiles && ok; ++j) {
+      for (int j = 0; j < n_vis && ok; ++j) {
         const int st = j % kStages;
         if (!mbar_wait(&bars->v_full[st], (j / kStages) & 1, p.status, kErrVFull)) break;
-        const bool has_next = j + 1 < n_tiles;
+        const bool has_next = j + 1 < n_vis;
         const int st1 = (j + 1) % kStages;
         for (int s = 0; s < n_sub; ++s) {
           if (!mbar_wait(&bars->p_ready[s], j & 1, p.status, kErrPReady)) { ok = false; break; }
@@ -256,16 +261,18 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
       // Visible-key end of this row.
       const int row = (s ? m01 : m00) + r;
-      int limit = p.seqlen_kv;
+      int limit = p.seqlen_kv, kv_first = 0;   // visible keys [kv_first, limit)
       if (row < p.seqlen_q) {
         const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
         limit = __ldg(p.kv_offsets + p.n_kv_chunks - p.n_q_chunks + c + 1);
+        if (p.kv_range > 0)
+          kv_first = __ldg(p.kv_offsets + max(p.n_kv_chunks - p.n_q_chunks + c - p.kv_range + 1, 0));
       }
 
       float m_ref = -INFINITY, l_sum = 0.f;
-      // Every thread runs all n_tiles iterations and reaches every named
+      // Every thread runs all n_vis iterations and reaches every named
       // barrier even after a failed wait; only the work is skipped.
-      for (int j = 0; j < n_tiles; ++j) {
+      for (int j = 0; j < n_vis; ++j) {
         ok = warp_wait(&bars->s_full[s], j & 1, ok, p.status, kErrSFull);
         if (ok) {
           tc_fence_after();
@@ -282,14 +289,16 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               for (int i = 0; i < 16; ++i)
                 x2[c * 16 + i] = f2_pack(__uint_as_float(raw[c][2 * i]), __uint_as_float(raw[c][2 * i + 1]));
           }
-          const bool masked = j >= n_full;
+          const int tile = t_begin + j;
+          const bool masked = tile < t_full_begin || tile >= n_full;
           if (masked) {
-            const int lim = limit - j * 128;
+            const int lim = limit - tile * 128, lo = kv_first - tile * 128;
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
               float a0, a1;
               f2_unpack(x2[c], a0, a1);
-              x2[c] = f2_pack(2 * c < lim ? a0 : -INFINITY, 2 * c + 1 < lim ? a1 : -INFINITY);
+              x2[c] = f2_pack(2 * c >= lo && 2 * c < lim ? a0 : -INFINITY,
+                              2 * c + 1 >= lo && 2 * c + 1 < lim ? a1 : -INFINITY);
             }
           }
           // row maximum as a tree (short dependency chains)
@@ -321,7 +330,10 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             m_ref = m_tile;
             l_sum *= alpha;
           }
-          const uint64_t negm = f2_pack(-m_ref, -m_ref);
+          // (a row whose visited tiles so far were all masked keeps m_ref = -inf
+          // and gets P = 0 from exp2(-inf - 0))
+          const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
+          const uint64_t negm = f2_pack(nm, nm);
           uint64_t ls2[4] = {0, 0, 0, 0};
           // P = exp2(S - m) -> bf16 pairs in TMEM.  The two variants are
           // separate straight-line loops (no per-pair branch), so the
@@ -380,7 +392,7 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
 
       // Epilogue: wait for the last PV, then O / l -> bf16, and the LSE.
-      ok = warp_wait(&bars->s_full[s], n_tiles & 1, ok, p.status, kErrSFull);
+      ok = warp_wait(&bars->s_full[s], n_vis & 1, ok, p.status, kErrSFull);
       if (ok) {
         tc_fence_after();
         const float inv_l = 1.f / l_sum;

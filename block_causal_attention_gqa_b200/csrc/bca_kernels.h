@@ -11,10 +11,11 @@
 namespace magi {
 
 struct FwdParams {
-  const int32_t* units;       // device, 8 int32 per unit (see magi_bca_fwd_schedule)
+  const int32_t* units;       // device, 12 int32 per unit (see magi_bca_fwd_schedule)
   const int32_t* q_offsets;   // device copy of the query chunk offsets
   const int32_t* kv_offsets;  // device copy of the kv chunk offsets
   int n_q_chunks, n_kv_chunks;
+  int kv_range;               // 0 = no limit, else chunks visible back from the row's own
   const float* gamma_q;
   const float* gamma_k;
   uint16_t* out;              // [B, Sq, Hq, D] bf16
@@ -38,6 +39,7 @@ struct BwdParams {
   const int32_t* q_offsets;   // device copies of the chunk offsets
   const int32_t* kv_offsets;
   int n_q_chunks, n_kv_chunks;
+  int kv_range;               // 0 = no limit, else chunks visible back from the row's own
   // outputs
   uint16_t* dq;
   uint16_t* dk;

@@ -128,6 +128,7 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
+  p.kv_range = d.kv_range;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

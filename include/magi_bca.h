@@ -82,6 +82,9 @@ typedef struct {
   int32_t n_kv_chunks;
   float softmax_scale;  /* 0 selects 1/sqrt(head_dim) */
   float rms_eps;        /* RMSNorm epsilon; must be >= 0 (1e-6 is the usual value) */
+  int32_t kv_range;     /* KV range in chunks (MAGI-1 §2.4.4, §2.6, Fig. 12): > 0 limits the query
+                         * chunk matched to kv chunk c to kv chunks [c - kv_range + 1, c] (1 = its
+                         * own chunk only); 0 = no limit (every kv chunk up to c).  Must be >= 0. */
 } magi_bca_dims;
 
 /* Forward.  Writes out (bf16) and lse (fp32; may be NULL when the caller

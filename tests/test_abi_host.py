@@ -135,27 +135,99 @@ def row_ends(qo, ko, Sq):
     return ends
 
 
-def check_schedule(q_lens, kv_lens, B, Hq, Hkv, D=128):
+def row_intervals(qo, ko, kv_range=0):
+    """Per query row the visible keys [begin, end): its matched kv chunk's end,
+    and (KV range R) the start of the chunk R - 1 before it.  Checked against
+    the oracle's token-level mask on small shapes below."""
+    nq, nkv = len(qo) - 1, len(ko) - 1
+    Sq = int(qo[-1])
+    begin = np.zeros(Sq, np.int64)
+    end = np.empty(Sq, np.int64)
+    for c in range(nq):
+        own = nkv - nq + c
+        end[qo[c]:qo[c + 1]] = ko[own + 1]
+        if kv_range > 0:
+            begin[qo[c]:qo[c + 1]] = ko[max(own - kv_range + 1, 0)]
+    return begin, end
+
+
+class TileMask:
+    """any()/all() of the visibility of a (query rows, keys) block from row intervals."""
+
+    def __init__(self, qo, ko, kv_range=0):
+        self.begin, self.end = row_intervals(qo, ko, kv_range)
+        self.Sq, self.Skv = int(qo[-1]), int(ko[-1])
+
+    def any(self, r0, r1, k0, k1):
+        b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
+        return bool(((b < min(k1, self.Skv)) & (e > k0)).any())
+
+    def all(self, r0, r1, k0, k1):
+        b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
+        return bool(((b <= k0) & (e >= min(k1, self.Skv))).all())
+
+    def any_tiles(self, r0, r1, n_tiles):
+        """any() for key tiles 0..n_tiles-1 at once (128-key tiles)."""
+        b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
+        k0 = np.arange(n_tiles) * 128
+        k1 = np.minimum(k0 + 128, self.Skv)
+        return ((b[:, None] < k1[None, :]) & (e[:, None] > k0[None, :])).any(axis=0)
+
+    def any_row_tiles(self, n_qt, k0, k1):
+        """any() for query tiles 0..n_qt-1 at once against keys [k0, k1)."""
+        k1 = min(k1, self.Skv)
+        hit = (self.begin < k1) & (self.end > k0)
+        pad = np.zeros(n_qt * 128, bool)
+        pad[:self.Sq] = hit
+        return pad.reshape(n_qt, 128).any(axis=1)
+
+    def all_row_tiles(self, n_qt, k0, k1):
+        """all() for query tiles 0..n_qt-1 at once against keys [k0, k1) (rows past Sq ignored)."""
+        k1 = min(k1, self.Skv)
+        ok = (self.begin <= k0) & (self.end >= k1)
+        pad = np.ones(n_qt * 128, bool)
+        pad[:self.Sq] = ok
+        return pad.reshape(n_qt, 128).all(axis=1)
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,R", [([2, 3, 1], [2, 3, 1], 0), ([2, 3, 1], [2, 3, 1], 2),
+                                              ([3, 2], [1, 2, 3, 2], 2), ([1] * 9, [1] * 9, 3)])
+def test_row_intervals_match_the_oracle_mask(q_lens, kv_lens, R):
+    from oracle import bca_oracle as orc
+    qo, ko = _offs(q_lens), _offs(kv_lens)
+    M = orc.block_causal_mask(qo, ko, kv_range=R)
+    b, e = row_intervals(qo, ko, R)
+    keys = np.arange(int(ko[-1]))
+    assert np.array_equal(M, (keys[None, :] >= b[:, None]) & (keys[None, :] < e[:, None]))
+
+
+def check_schedule(q_lens, kv_lens, B, Hq, Hkv, D=128, kv_range=0):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
-    units = bca.magi_bca_fwd_schedule(qo, ko, B, Hq, Hkv, D)
-    ends = row_ends(qo, ko, Sq)
+    units = bca.magi_bca_fwd_schedule(qo, ko, B, Hq, Hkv, D, kv_range=kv_range)
+    assert units.shape[1] == 12
+    M = TileMask(qo, ko, kv_range)
+    n_kt = -(-Skv // 128)
     g = Hq // Hkv
     seen = np.zeros((B, Hq, (Sq + 127) // 128), np.int64)
     costs = []
-    for b, hk, h0, m00, h1, m01, n_full, n_tiles in units:
+    checked = set()   # visibility depends only on the query tile, not on batch or head
+    for b, hk, h0, m00, h1, m01, n_full, n_tiles, t_begin, t_full_begin, z0, z1 in units:
+        assert z0 == 0 and z1 == 0
         subs = [(h0, m00)] + ([(h1, m01)] if h1 >= 0 else [])
         for h, m0 in subs:
             assert h // g == hk and m0 % 128 == 0
             seen[b, h, m0 // 128] += 1
-            rows = ends[m0:min(m0 + 128, Sq)]
-            # tiles [0, n_full) fully visible to every row; tile n_full.. needs the mask
-            assert n_full == rows.min() // 128
-            assert n_tiles == -(-rows.max() // 128)
-            assert n_tiles * 128 >= rows.max() and (n_tiles - 1) * 128 < rows.max()
-            # no visited tile is fully masked for every row
-            assert (n_tiles - 1) * 128 < rows.max()
-        costs.append(n_tiles * len(subs))
+            if (m0, n_full, n_tiles, t_begin, t_full_begin) in checked:
+                continue
+            checked.add((m0, n_full, n_tiles, t_begin, t_full_begin))
+            tiles_seen = list(np.nonzero(M.any_tiles(m0, m0 + 128, n_kt))[0])
+            # exactly the tiles with some visible (row, key) pair are visited
+            assert tiles_seen == list(range(t_begin, n_tiles)), (tiles_seen, t_begin, n_tiles)
+            # tiles the kernel leaves unmasked are fully visible to every row
+            for t in range(max(t_begin, t_full_begin), min(n_full, n_tiles)):
+                assert M.all(m0, m0 + 128, t * 128, t * 128 + 128), t
+        costs.append((n_tiles - t_begin) * len(subs))
     # every (batch, head, query tile) exactly once
     assert (seen == 1).all()
     # longest first
@@ -175,6 +247,18 @@ def check_schedule(q_lens, kv_lens, B, Hq, Hkv, D=128):
 ])
 def test_fwd_schedule_covers_each_query_tile_once_with_correct_extents(q_lens, kv_lens, B, Hq, Hkv):
     check_schedule(q_lens, kv_lens, B, Hq, Hkv)
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,R", [
+    ([64, 64, 64], [64, 64, 64], 1),
+    ([300, 200, 150, 250, 100], [300, 200, 150, 250, 100], 2),
+    ([150, 250], [300, 200, 150, 250], 2),
+    ([1024] * 8, [1024] * 8, 3),
+    ([1] * 37, [1] * 37, 5),
+    ([5760] * 4, [5760] * 16, 8),
+])
+def test_fwd_schedule_with_kv_range(q_lens, kv_lens, R):
+    check_schedule(q_lens, kv_lens, 2, 8, 2, kv_range=R)
 
 
 def test_aligned_chunks_need_no_mask():
@@ -199,30 +283,33 @@ def test_workload_shapes():
     assert (w.batch, w.seqlen_q, w.seqlen_kv) == (2, 23040, 92160)
 
 
-def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148):
+def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=0):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
     G = Hq // Hkv
-    units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms)
-    ends = row_ends(qo, ko, Sq)
+    units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms, kv_range=kv_range)
+    M = TileMask(qo, ko, kv_range)
     n_qt, n_kt = -(-Sq // 128), -(-Skv // 128)
     cover = np.zeros((B, Hkv, n_kt, n_qt, G), np.int64)
     lengths = []
-    for b, hk, n0, s0, s1, diag_end, _, _ in units:
+    tile_any, tile_all = {}, {}
+    for b, hk, n0, s0, s1, diag_end, diag_hi_begin, z in units:
+        assert z == 0
         assert n0 % 128 == 0 and 0 <= s0 < s1 <= n_qt * G
-        n_end = min(n0 + 128, Skv)
-        for s in range(s0, s1):
-            t, g = divmod(s, G)
-            cover[b, hk, n0 // 128, t, g] += 1
-            rows = ends[t * 128:min(t * 128 + 128, Sq)]
-            assert (rows > n0).any()                  # some row of the tile sees some key
-            assert (rows.min() < n_end) == (t < diag_end), (t, diag_end)
+        if n0 not in tile_any:
+            tile_any[n0] = M.any_row_tiles(n_qt, n0, n0 + 128)
+            tile_all[n0] = M.all_row_tiles(n_qt, n0, n0 + 128)
+        steps = np.arange(s0, s1)
+        t, g = steps // G, steps % G
+        np.add.at(cover, (b, hk, n0 // 128, t, g), 1)
+        assert tile_any[n0][t].all()                         # some row of each tile sees some key
+        plain = ~((t < diag_end) | (t >= diag_hi_begin))     # left unmasked: fully visible
+        assert tile_all[n0][t[plain]].all(), (n0, diag_end, diag_hi_begin)
         lengths.append(s1 - s0)
-    # every (kv tile, query tile, head) where some query sees some key: exactly once
+    # every (kv tile, query tile, head) with a visible pair: exactly once
     for kt in range(n_kt):
-        for t in range(n_qt):
-            want = int((ends[t * 128:min(t * 128 + 128, Sq)] > kt * 128).any())
-            assert (cover[:, :, kt, t, :] == want).all(), (kt, t)
+        want = M.any_row_tiles(n_qt, kt * 128, kt * 128 + 128).astype(np.int64)
+        assert (cover[:, :, kt, :, :] == want[None, None, :, None]).all(), kt
     assert all(a >= b for a, b in zip(lengths, lengths[1:]))
     return units
 
@@ -237,6 +324,18 @@ def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148):
 ])
 def test_bwd_schedule_covers_each_visible_step_once(q_lens, kv_lens, B, Hq, Hkv):
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv)
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,R", [
+    ([64, 64, 64], [64, 64, 64], 1),
+    ([300, 200, 150, 250, 100], [300, 200, 150, 250, 100], 2),
+    ([150, 250], [300, 200, 150, 250], 2),
+    ([1024] * 8, [1024] * 8, 3),
+    ([1] * 37, [1] * 37, 5),
+    ([5760] * 4, [5760] * 16, 8),
+])
+def test_bwd_schedule_with_kv_range(q_lens, kv_lens, R):
+    check_bwd_schedule(q_lens, kv_lens, 2, 8, 2, kv_range=R)
 
 
 def lpt_span(costs, machines):

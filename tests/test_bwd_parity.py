@@ -21,7 +21,8 @@ from tests.test_fwd_parity import SMALL
 pytestmark = pytest.mark.gpu
 
 BWD_SMALL = ["train4k", "ragged_d128", "ragged_d64_gqa3", "stream_small", "single_chunk_mha", "token_causal",
-             "many_chunks", "gqa8_long_rows", "tiny"]
+             "many_chunks", "gqa8_long_rows", "tiny", "window_r1_ragged", "window_r2_ragged",
+             "window_stream_r3_d64", "window_token_r5", "window_aligned_r3"]
 # The five named workloads use the stated bound (max abs 1e-2, rel L2 5e-3).  The
 # extra edge cases (ragged chunks, 1-token chunks, LogNormal token scales with 8
 # query heads per kv head) keep rel L2 5e-3 but allow max abs 2e-2 on the
@@ -36,8 +37,9 @@ def gpu_fwd_bwd(inp, w):
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
     gq, gk = inp["gamma_q"].to(dev), inp["gamma_k"].to(dev)
     dout = inp["dout"].to(dev)
-    out, lse = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk)
-    dq, dk, dv, dgq, dgk = bca.magi_bca_bwd(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk)
+    out, lse = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, kv_range=w.kv_range)
+    dq, dk, dv, dgq, dgk = bca.magi_bca_bwd(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk,
+                                            kv_range=w.kv_range)
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
     return dq, dk, dv, dgq, dgk
@@ -49,7 +51,7 @@ def test_backward_all_rows(name):
     inp = workloads.make_inputs(w, with_grad_out=True)
     dq, dk, dv, dgq, dgk = gpu_fwd_bwd(inp, w)
     ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                       inp["gamma_q"], inp["gamma_k"])
+                       inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
     bound = 1e-2 if name in NAMED else 2e-2
     for nm, got in (("dq", dq), ("dk", dk), ("dv", dv)):
         e, r = assert_close(f"{name} {nm}", to_np(got), ref[nm], max_abs=bound)
@@ -102,7 +104,7 @@ def identities(name, w, inp, dq, dk, dv):
         assert float(cos.max()) <= 2e-2, f"{name}: {nm}.x not ~0 (max cos {float(cos.max()):.2e})"
 
 
-@pytest.mark.parametrize("name,kv_heads", [("model46k", [0, 5]), ("long262k", None)])
+@pytest.mark.parametrize("name,kv_heads", [("model46k", [0, 5]), ("long262k", None), ("window262k", None)])
 def test_backward_full_size_sampled(name, kv_heads):
     w = workloads.workload(name)
     inp = workloads.make_inputs(w, with_grad_out=True)
@@ -112,7 +114,7 @@ def test_backward_full_size_sampled(name, kv_heads):
     identities(name, w, inp, dq, dk, dv)
     rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, 4096, seed=200)
     ref = orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                            inp["gamma_q"], inp["gamma_k"], q_rows=rows)
+                            inp["gamma_q"], inp["gamma_k"], q_rows=rows, kv_range=w.kv_range)
     idx = torch.as_tensor(rows)
     e, r = assert_close(f"{name} dq rows", to_np(dq[:, idx]), ref["dq"])
     print(f"{name} dq rows: max abs {e:.2e} rel L2 {r:.2e}")
@@ -120,7 +122,7 @@ def test_backward_full_size_sampled(name, kv_heads):
         last = int(w.kv_offsets[-2])
         kr = np.sort(np.random.default_rng(201).choice(np.arange(last, w.seqlen_kv), 256, replace=False))
         ref = orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                                inp["gamma_q"], inp["gamma_k"], kv_rows=kr, kv_heads=kv_heads)
+                                inp["gamma_q"], inp["gamma_k"], kv_rows=kr, kv_heads=kv_heads, kv_range=w.kv_range)
         kidx = torch.as_tensor(kr)
         for nm, got in (("dk", dk), ("dv", dv)):
             e, r = assert_close(f"{name} {nm} rows", to_np(got[:, kidx][:, :, kv_heads]), ref[nm])

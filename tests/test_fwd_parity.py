@@ -20,7 +20,7 @@ def run_gpu(inp, w, lse=True):
     dev = "cuda"
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
     out, l = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, inp["gamma_q"].to(dev),
-                              inp["gamma_k"].to(dev), want_lse=lse)
+                              inp["gamma_k"].to(dev), want_lse=lse, kv_range=w.kv_range)
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
     return out, l
@@ -37,6 +37,16 @@ SMALL = {
     "many_chunks": workloads.custom("many_chunks", 1, [50] * 20, None, 4, 1, 128, seed=16),
     "gqa8_long_rows": workloads.custom("gqa8_long_rows", 1, [640] * 3, None, 16, 2, 128, seed=17,
                                        token_scale=True),
+    # KV range (MAGI-1 §2.4.4, Fig. 12): each chunk sees itself and the R - 1 chunks before it
+    "window_r1_ragged": workloads.custom("window_r1_ragged", 2, [100, 333, 200, 67], None, 4, 2, 128, seed=21,
+                                         kv_range=1),
+    "window_r2_ragged": workloads.custom("window_r2_ragged", 1, [300, 200, 150, 250, 100], None, 8, 2, 128,
+                                         seed=22, kv_range=2),
+    "window_stream_r3_d64": workloads.custom("window_stream_r3_d64", 2, [150, 250], [300, 200, 150, 250], 8, 2, 64,
+                                             seed=23, kv_range=3),
+    "window_token_r5": workloads.custom("window_token_r5", 1, [1] * 37, None, 2, 1, 64, seed=24, kv_range=5),
+    "window_aligned_r3": workloads.custom("window_aligned_r3", 1, [256] * 8, None, 4, 1, 128, seed=25,
+                                          kv_range=3),
 }
 
 
@@ -46,14 +56,14 @@ def test_forward_all_rows(name):
     inp = workloads.make_inputs(w, with_grad_out=False)
     out, lse = run_gpu(inp, w)
     o_ref, l_ref = orc.forward(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
-                               inp["gamma_q"], inp["gamma_k"])
+                               inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
     e, r = assert_close(f"{name} out", to_np(out), o_ref)
     el, rl = assert_close(f"{name} lse", to_np(lse), l_ref)
     print(f"{name}: out max abs {e:.2e} rel L2 {r:.2e}; lse max abs {el:.2e} rel L2 {rl:.2e}")
     if "q_f32" in inp:
         # information only: error against the unrounded fp32 inputs
         o32, _ = orc.forward(inp["q_f32"], inp["k_f32"], inp["v_f32"], w.q_offsets, w.kv_offsets,
-                             inp["gamma_q"], inp["gamma_k"])
+                             inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
         print(f"{name}: rel L2 vs unrounded fp32 inputs {rel_l2(to_np(out), o32):.3e}")
 
 
@@ -82,7 +92,7 @@ def test_forward_is_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-LARGE = ["model46k", "stream4of16", "long262k"]
+LARGE = ["model46k", "stream4of16", "long262k", "window262k"]
 
 
 @pytest.mark.parametrize("name", LARGE)
@@ -98,7 +108,7 @@ def test_forward_full_size_sampled_rows(name):
     for b in range(w.batch):
         rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, per_batch, seed=100 + b)
         o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
-                                        inp["gamma_q"], inp["gamma_k"], rows, batches=[b])
+                                        inp["gamma_q"], inp["gamma_k"], rows, batches=[b], kv_range=w.kv_range)
         idx = torch.as_tensor(rows)
         e, r = assert_close(f"{name} out b{b}", to_np(out_c[b:b + 1, idx]), o_ref)
         el, rl = assert_close(f"{name} lse b{b}", to_np(lse_c[b:b + 1][:, :, idx]), l_ref)

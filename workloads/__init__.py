@@ -48,6 +48,7 @@ class Workload:
     input_dtype: str = "bf16"    # "fp32" = drawn fp32 then rounded to bf16 at the boundary
     gamma: str = "perturbed"     # "ones" or "perturbed" (1 + N(0, 0.1) per head-dim)
     token_scale: bool = False    # LogNormal(0, 0.5) per-token scale on q and k
+    kv_range: int = 0            # KV range in chunks (0 = every earlier chunk); MAGI-1 §2.4.4, Fig. 12
 
     @property
     def seqlen_q(self) -> int:
@@ -86,9 +87,13 @@ WORKLOADS = {
     # long context: 32 chunks x 8192 tokens, GQA 16/2, LogNormal per-token q/k scales.
     "long262k": Workload("long262k", 1, uniform_offsets(32, 8192), uniform_offsets(32, 8192),
                          16, 2, 128, seed=4, backward=True, token_scale=True),
+    # long context with a KV range of 8 chunks (MAGI-1 §2.4.4 and §2.6: each chunk limited to
+    # the preceding content, KV range 8 for long videos), otherwise as long262k.
+    "window262k": Workload("window262k", 1, uniform_offsets(32, 8192), uniform_offsets(32, 8192),
+                           16, 2, 128, seed=5, backward=True, token_scale=True, kv_range=8),
 }
 
-ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k"]
+ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k"]
 
 
 def workload(name_or_index) -> Workload:
@@ -99,10 +104,10 @@ def workload(name_or_index) -> Workload:
 
 def custom(name: str, batch: int, q_chunks: Sequence[int], kv_chunks: Optional[Sequence[int]],
            heads_q: int, heads_kv: int, head_dim: int, seed: int, backward: bool = True,
-           gamma: str = "perturbed", token_scale: bool = False) -> Workload:
+           gamma: str = "perturbed", token_scale: bool = False, kv_range: int = 0) -> Workload:
     kv = tuple(kv_chunks) if kv_chunks is not None else tuple(q_chunks)
     return Workload(name, batch, tuple(q_chunks), kv, heads_q, heads_kv, head_dim, seed,
-                    backward, gamma=gamma, token_scale=token_scale)
+                    backward, gamma=gamma, token_scale=token_scale, kv_range=kv_range)
 
 
 def make_inputs(w: Workload, device: str = "cpu", with_grad_out: Optional[bool] = None) -> dict:

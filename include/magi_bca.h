@@ -32,8 +32,12 @@
  *   *_chunk_offsets  : host int32 [n_chunks + 1], offsets[0] = 0, strictly
  *                      increasing, offsets[n] = seqlen; the same chunking
  *                      applies to every batch element.  Matched chunks
- *                      (query chunk c and kv chunk n_kv - n_q + c) must have
- *                      equal lengths.
+ *                      (query chunk c and kv chunk n_kv - n_q + c) may differ
+ *                      in length: self-attention has them equal; one query
+ *                      chunk against one key/value chunk of another length is
+ *                      cross-attention (MAGI-1 §2.2.2, text K/V), and with
+ *                      kv_range = 1 each query chunk attends only to its own
+ *                      key/value chunk (chunk-wise text conditioning, MAGI-1 §7).
  *
  * Ownership: every tensor pointer is caller-owned device memory; the chunk
  * offsets are host memory read during the call.  The library keeps one

@@ -63,7 +63,7 @@ def dims_for(qo, ko, B=1, Hq=4, Hkv=2, D=128, eps=1e-6, scale=0.0):
     ("batch0", INVALID_ARG), ("neg_eps", INVALID_ARG), ("nan_scale", INVALID_ARG),
     ("head_dim_96", UNSUPPORTED), ("gqa_indivisible", UNSUPPORTED),
     ("first_not_zero", BAD_OFFSETS), ("last_not_seqlen", BAD_OFFSETS), ("empty_chunk", BAD_OFFSETS),
-    ("decreasing", BAD_OFFSETS), ("more_q_than_kv_chunks", BAD_OFFSETS), ("unmatched_lengths", BAD_OFFSETS),
+    ("decreasing", BAD_OFFSETS), ("more_q_than_kv_chunks", BAD_OFFSETS), ("negative_kv_range", INVALID_ARG),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(case, expect):
     qo, ko = _offs([10, 20]), _offs([10, 20])
@@ -99,10 +99,16 @@ def test_invalid_arguments_are_rejected_on_the_host(case, expect):
     elif case == "more_q_than_kv_chunks":
         qo, ko = _offs([10, 10, 10]), _offs([15, 15])
         d = dims_for(qo, ko)
-    elif case == "unmatched_lengths":
-        qo, ko = _offs([10, 20]), _offs([5, 15, 10])
-        d = dims_for(qo, ko)
+    elif case == "negative_kv_range":
+        d.kv_range = -1
     assert call_fwd(d, qo, ko, **kw) == expect
+
+
+def test_matched_chunks_of_different_lengths_are_accepted():
+    """Cross-attention: query chunks may differ in length from their kv chunks."""
+    for q_lens, kv_lens in (([1000], [333]), ([300, 200, 250], [77, 120, 64]), ([10, 20], [5, 15, 10])):
+        qo, ko = _offs(q_lens), _offs(kv_lens)
+        assert call_fwd(dims_for(qo, ko), qo, ko) not in (INVALID_ARG, BAD_OFFSETS)
 
 
 def test_valid_arguments_reach_the_device_check():
@@ -256,6 +262,9 @@ def test_fwd_schedule_covers_each_query_tile_once_with_correct_extents(q_lens, k
     ([1024] * 8, [1024] * 8, 3),
     ([1] * 37, [1] * 37, 5),
     ([5760] * 4, [5760] * 16, 8),
+    ([1000], [333], 0),                    # cross-attention against a text sequence
+    ([77], [1000], 0),
+    ([300, 200, 250], [77, 120, 64], 1),   # chunk-wise text conditioning
 ])
 def test_fwd_schedule_with_kv_range(q_lens, kv_lens, R):
     check_schedule(q_lens, kv_lens, 2, 8, 2, kv_range=R)
@@ -333,6 +342,9 @@ def test_bwd_schedule_covers_each_visible_step_once(q_lens, kv_lens, B, Hq, Hkv)
     ([1024] * 8, [1024] * 8, 3),
     ([1] * 37, [1] * 37, 5),
     ([5760] * 4, [5760] * 16, 8),
+    ([1000], [333], 0),
+    ([77], [1000], 0),
+    ([300, 200, 250], [77, 120, 64], 1),
 ])
 def test_bwd_schedule_with_kv_range(q_lens, kv_lens, R):
     check_bwd_schedule(q_lens, kv_lens, 2, 8, 2, kv_range=R)

@@ -22,7 +22,8 @@ pytestmark = pytest.mark.gpu
 
 BWD_SMALL = ["train4k", "ragged_d128", "ragged_d64_gqa3", "stream_small", "single_chunk_mha", "token_causal",
              "many_chunks", "gqa8_long_rows", "tiny", "window_r1_ragged", "window_r2_ragged",
-             "window_stream_r3_d64", "window_token_r5", "window_aligned_r3"]
+             "window_stream_r3_d64", "window_token_r5", "window_aligned_r3", "xattn_video_text",
+             "xattn_short_q_d64", "xattn_chunkwise"]
 # The five named workloads use the stated bound (max abs 1e-2, rel L2 5e-3).  The
 # extra edge cases (ragged chunks, 1-token chunks, LogNormal token scales with 8
 # query heads per kv head) keep rel L2 5e-3 but allow max abs 2e-2 on the
@@ -104,7 +105,8 @@ def identities(name, w, inp, dq, dk, dv):
         assert float(cos.max()) <= 2e-2, f"{name}: {nm}.x not ~0 (max cos {float(cos.max()):.2e})"
 
 
-@pytest.mark.parametrize("name,kv_heads", [("model46k", [0, 5]), ("long262k", None), ("window262k", None)])
+@pytest.mark.parametrize("name,kv_heads", [("model46k", [0, 5]), ("long262k", None), ("window262k", None),
+                                           ("xattn46k", [0, 7])])
 def test_backward_full_size_sampled(name, kv_heads):
     w = workloads.workload(name)
     inp = workloads.make_inputs(w, with_grad_out=True)

@@ -47,6 +47,11 @@ SMALL = {
     "window_token_r5": workloads.custom("window_token_r5", 1, [1] * 37, None, 2, 1, 64, seed=24, kv_range=5),
     "window_aligned_r3": workloads.custom("window_aligned_r3", 1, [256] * 8, None, 4, 1, 128, seed=25,
                                           kv_range=3),
+    # cross-attention (MAGI-1 §2.2.2 text K/V; §7 chunk-wise text conditioning)
+    "xattn_video_text": workloads.custom("xattn_video_text", 2, [1000], [333], 8, 2, 128, seed=26),
+    "xattn_short_q_d64": workloads.custom("xattn_short_q_d64", 1, [77], [1000], 4, 2, 64, seed=27),
+    "xattn_chunkwise": workloads.custom("xattn_chunkwise", 1, [300, 200, 250], [77, 120, 64], 8, 2, 128,
+                                        seed=28, kv_range=1),
 }
 
 
@@ -92,7 +97,7 @@ def test_forward_is_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-LARGE = ["model46k", "stream4of16", "long262k", "window262k"]
+LARGE = ["model46k", "stream4of16", "long262k", "window262k", "xattn46k"]
 
 
 @pytest.mark.parametrize("name", LARGE)

@@ -455,3 +455,30 @@ def test_kv_range_backward_rows_match_full_backward():
     np.testing.assert_allclose(part["dq"][0], full["dq"][0, rows], rtol=0, atol=1e-12)
     np.testing.assert_allclose(part["dk"][0], full["dk"][0, kv_rows], rtol=0, atol=1e-12)
     np.testing.assert_allclose(part["dv"][0], full["dv"][0, kv_rows], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- cross-attention
+
+def test_one_chunk_pair_of_different_lengths_is_full_cross_attention():
+    """One query chunk against one key/value chunk of another length (text K/V,
+    MAGI-1 §2.2.2): every query sees every key, as torch SDPA without a mask."""
+    rng = np.random.default_rng(41)
+    for Sq, Skv in ((23, 9), (7, 31)):
+        q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [Sq], [Skv], 6, 2, 16)
+        o, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+        want = torch_reference(q, k, v, qo, ko, gq, gk, mask=torch.ones(Sq, Skv, dtype=torch.bool))
+        np.testing.assert_allclose(o, want, rtol=0, atol=1e-12)
+
+
+def test_chunkwise_text_conditioning_is_cross_attention_per_chunk():
+    """KV range 1 with text chunks of their own lengths (MAGI-1 §7, chunk-wise text
+    conditioning): query chunk c attends exactly to text chunk c."""
+    rng = np.random.default_rng(42)
+    q_lens, t_lens = [6, 9, 4], [3, 5, 7]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, q_lens, t_lens, 4, 2, 8)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=1)
+    for c in range(3):
+        qs, ks = slice(qo[c], qo[c + 1]), slice(ko[c], ko[c + 1])
+        want = torch_reference(q[:, qs], k[:, ks], v[:, ks], offs([q_lens[c]]), offs([t_lens[c]]), gq, gk,
+                               mask=torch.ones(q_lens[c], t_lens[c], dtype=torch.bool))
+        np.testing.assert_allclose(o[:, qs], want, rtol=0, atol=1e-12)

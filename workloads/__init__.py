@@ -91,9 +91,14 @@ WORKLOADS = {
     # the preceding content, KV range 8 for long videos), otherwise as long262k.
     "window262k": Workload("window262k", 1, uniform_offsets(32, 8192), uniform_offsets(32, 8192),
                            16, 2, 128, seed=5, backward=True, token_scale=True, kv_range=8),
+
+    # cross-attention of the model-scale video sequence (one chunk of 8 x 5760 tokens)
+    # against 1024 text tokens (MAGI-1 §2.2.2: cross-attention with QK-norm and GQA
+    # to the T5 text condition; the text length is a reading), GQA 24/8.
+    "xattn46k": Workload("xattn46k", 1, (46080,), (1024,), 24, 8, 128, seed=6, backward=True),
 }
 
-ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k"]
+ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k"]
 
 
 def workload(name_or_index) -> Workload:

@@ -160,15 +160,20 @@ def ncu_traffic(kernel, workload_name):
 
 # ------------------------------------------------------------------ distributed
 def dist_setup():
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE): NCCL on
+    GPUs; gloo when no GPU is present (the host-side logic's CPU tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -184,9 +189,16 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(world, flops_per_step_per_rank, steps, slowest_rank_ms):
+    """Throughput of the whole job: every rank runs `steps` steps of its own
+    (replica) workload; the job takes as long as its slowest rank."""
+    return world * flops_per_step_per_rank * steps / (slowest_rank_ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------ our arm
@@ -343,8 +355,8 @@ def run_ours(args, w, world, rank, local):
     d2h = (q.numel() + 2 * k.numel()) * 2 if do_bwd else q.numel() * 2 + lse.numel() * 4
 
     flops_step = fwd_flops(w) + (bwd_flops(w) if do_bwd else 0.0)
-    value = world * flops_step * args.steps / (step_ms_total * 1e-3) / 1e12
-    e2e_value = world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops_step, args.steps, step_ms_total)
+    e2e_value = whole_job_tflops(world, flops_step, e2e_steps, e2e_ms)
 
     peaks, peak_src = load_peaks()
     # dominant kernel (the backward main kernel when there is a backward, else
@@ -492,8 +504,9 @@ def run_reference(args, w, world, rank):
         "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
-                   "seqlen_kv": w.seqlen_kv, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
-                   "head_dim": w.head_dim},
+                   "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
+                   "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -39,6 +39,14 @@ folding of scales):
    dq~ = scale dS k~, dk~ = scale dS^T q~, summed over each query-head group
    for k and v, then the RMSNorm Jacobian back to the raw q and k, and the
    gain gradients dgamma = sum over (batch, token, head) of dx~ * x_hat.
+6. Optional rotary position embedding before the norm (MAGI-1 §2.2.2 and the
+   notes' DiT-block sketch: learnable 3D RoPE applied to q and k, then
+   QK-norm).  The pages give no formula; the reading here: per token an angle
+   for each of the D/2 feature pairs (i, i + D/2), shared by all heads and
+   batch elements (the 3D split and the learnable frequencies produce these
+   angles outside the attention), ``y_i = x_i cos t - x_{i+D/2} sin t``,
+   ``y_{i+D/2} = x_{i+D/2} cos t + x_i sin t``.  The backward returns the
+   angle gradients as well, summed over batch and heads.
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against
 brute force, a library routine or an invariant; none is "parity unpinned".
@@ -49,7 +57,7 @@ import numpy as np
 
 __all__ = ["rms_norm", "rms_norm_backward", "chunk_of", "matched_kv_chunk",
            "block_causal_mask", "forward", "forward_rows", "backward", "backward_rows",
-           "DEFAULT_EPS"]
+           "rope", "rope_backward", "DEFAULT_EPS"]
 
 DEFAULT_EPS = 1e-6
 
@@ -62,6 +70,38 @@ def _f64(x):
             x = x.float()
         x = x.numpy()
     return np.asarray(x, dtype=np.float64)
+
+
+def rope(x, angles):
+    """Rotary embedding over the last axis of x [..., S, H, D]: feature pair
+    (i, i + D/2) of token s rotates by angles[s, i] (angles [S, D/2])."""
+    x = _f64(x)
+    if angles is None:
+        return x
+    t = _f64(angles)
+    h = x.shape[-1] // 2
+    c, s = np.cos(t)[:, None, :], np.sin(t)[:, None, :]
+    a, b = x[..., :h], x[..., h:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def rope_backward(x, angles, dy):
+    """Gradients of y = rope(x, angles) given dy: (dx, dangles), dangles [S, D/2]
+    summed over every leading axis and the heads."""
+    x = _f64(x)
+    dy = _f64(dy)
+    if angles is None:
+        return dy, None
+    t = _f64(angles)
+    h = x.shape[-1] // 2
+    c, s = np.cos(t)[:, None, :], np.sin(t)[:, None, :]
+    y = rope(x, angles)
+    ga, gb = dy[..., :h], dy[..., h:]
+    dx = np.concatenate([ga * c + gb * s, gb * c - ga * s], axis=-1)
+    # dy_a/dt = -y_b, dy_b/dt = y_a
+    dt = -ga * y[..., h:] + gb * y[..., :h]
+    dt = dt.reshape((-1,) + dt.shape[-3:]).sum(axis=(0, 2))
+    return dx, dt
 
 
 def rms_norm(x, gamma, eps=DEFAULT_EPS):
@@ -155,7 +195,8 @@ def _attend_rows(qn_rows, kn, vv, mask_rows, scale):
 
 
 def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=None,
-                 batches=None, scale=None, eps=DEFAULT_EPS, block=None, kv_range=0):
+                 batches=None, scale=None, eps=DEFAULT_EPS, block=None, kv_range=0, rope_q=None,
+                 rope_k=None):
     """Forward on a subset of query rows.
 
     ``rows`` is an int array of query-token indices; ``heads`` / ``batches``
@@ -169,6 +210,8 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
     B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
     # only the requested query rows are converted (row i of qsel is rows[i])
     qsel = _f64(q[:, rows]) if not hasattr(q, "detach") else _f64(q[:, torch_index(rows)])
+    qsel = rope(qsel, None if rope_q is None else _f64(rope_q)[rows])
+    k = rope(k, rope_k)
     scale = 1.0 / np.sqrt(D) if not scale else float(scale)
     heads = list(range(Hq)) if heads is None else list(heads)
     batches = list(range(B)) if batches is None else list(batches)
@@ -193,19 +236,22 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
     return out, lse
 
 
-def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS, kv_range=0):
+def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS, kv_range=0,
+            rope_q=None, rope_k=None):
     """Full forward.  Returns (out [B, Sq, Hq, D], lse [B, Hq, Sq]), float64."""
     Sq = q.shape[1]
     return forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k,
-                        rows=np.arange(Sq), scale=scale, eps=eps, kv_range=kv_range)
+                        rows=np.arange(Sq), scale=scale, eps=eps, kv_range=kv_range, rope_q=rope_q,
+                        rope_k=rope_k)
 
 
 def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
-             eps=DEFAULT_EPS, kv_range=0):
+             eps=DEFAULT_EPS, kv_range=0, rope_q=None, rope_k=None):
     """Full analytic backward in float64.
 
-    Returns dict(dq, dk, dv, dgamma_q, dgamma_k, out, lse); dq/dk are the
-    gradients with respect to the raw (pre-norm) q and k."""
+    Returns dict(dq, dk, dv, dgamma_q, dgamma_k, out, lse) and, with rotary
+    angles, drope_q, drope_k; dq/dk are the gradients with respect to the raw
+    (pre-rotation, pre-norm) q and k."""
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
@@ -223,6 +269,8 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
     dv = np.zeros_like(v)
     out = np.zeros_like(q)
     lse = np.zeros((B, Hq, Sq))
+    q_raw, k_raw = q, k
+    q, k = rope(q_raw, rope_q), rope(k_raw, rope_k)
     qn_all = rms_norm(q, gq, eps)
     kn_all = rms_norm(k, gk, eps)
     for b in range(B):
@@ -243,12 +291,19 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
             dkn[b, :, hk, :] += scale * (ds.T @ qn)
     dq, dgq = rms_norm_backward(q, gq, dqn, eps)
     dk, dgk = rms_norm_backward(k, gk, dkn, eps)
-    return dict(dq=dq, dk=dk, dv=dv, dgamma_q=dgq, dgamma_k=dgk, out=out, lse=lse)
+    dq, drq = rope_backward(q_raw, rope_q, dq)
+    dk, drk = rope_backward(k_raw, rope_k, dk)
+    res = dict(dq=dq, dk=dk, dv=dv, dgamma_q=dgq, dgamma_k=dgk, out=out, lse=lse)
+    if rope_q is not None:
+        res["drope_q"] = drq
+    if rope_k is not None:
+        res["drope_k"] = drk
+    return res
 
 
 def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows=None,
                   kv_rows=None, kv_heads=None, batches=None, scale=None, eps=DEFAULT_EPS,
-                  block=None, kv_range=0):
+                  block=None, kv_range=0, rope_q=None, rope_k=None):
     """Exact backward on chosen rows, without a full backward.
 
     * dq of query rows ``q_rows`` (all heads): needs only those rows' P, dP
@@ -277,12 +332,15 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
         return _f64(x[:, torch_index(rows)] if hasattr(x, "detach") else x[:, rows])
 
     res = {}
+    rk = None if rope_k is None else _f64(rope_k)
     if q_rows is not None:
         q_rows = np.asarray(q_rows, dtype=np.int64)
-        qsel, dsel = take(q, q_rows), take(dout, q_rows)
+        qraw, dsel = take(q, q_rows), take(dout, q_rows)
+        rq = None if rope_q is None else _f64(rope_q)[q_rows]
+        qsel = rope(qraw, rq)
         dq = np.zeros((len(batches), len(q_rows), Hq, D))
         for bi, b in enumerate(batches):
-            kn_all = rms_norm(k[b], gk, eps)
+            kn_all = rms_norm(rope(k[b], rk), gk, eps)
             for r0 in range(0, len(q_rows), block):
                 rr = q_rows[r0:r0 + block]
                 mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
@@ -297,7 +355,9 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                     dp -= delta
                     dp *= p
                     dqn[:, h, :] = scale * (dp @ kn_all[:, hk, :])
-                dq[bi, r0:r0 + len(rr)], _ = rms_norm_backward(qsel[b, r0:r0 + block], gq, dqn, eps)
+                dqr, _ = rms_norm_backward(qsel[b, r0:r0 + block], gq, dqn, eps)
+                dq[bi, r0:r0 + len(rr)], _ = rope_backward(qraw[b, r0:r0 + block],
+                                                           None if rq is None else rq[r0:r0 + block], dqr)
         res["dq"] = dq
     if kv_rows is not None:
         kv_rows = np.asarray(kv_rows, dtype=np.int64)
@@ -307,8 +367,10 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
         # every query row that sees at least one of the requested keys
         seeing = np.nonzero(block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range)[:, kv_rows].any(axis=1))[0]
         qsel, dsel = take(q, seeing), take(dout, seeing)
+        qsel = rope(qsel, None if rope_q is None else _f64(rope_q)[seeing])
         for bi, b in enumerate(batches):
-            kn_all = rms_norm(k[b], gk, eps)
+            kr_all = rope(k[b], rk)
+            kn_all = rms_norm(kr_all, gk, eps)
             for khi, hk in enumerate(kv_heads):
                 kn = kn_all[:, hk, :]
                 vv = v[b, :, hk, :]
@@ -326,7 +388,12 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                         dsc = pc * (dpc - delta)
                         dv[bi, :, khi, :] += pc.T @ g
                         dkn += scale * (dsc.T @ qn)
-                dk[bi, :, khi, :], _ = rms_norm_backward(k[b, kv_rows, hk, :], gk, dkn, eps)
+                dkr, _ = rms_norm_backward(kr_all[kv_rows, hk, :], gk, dkn, eps)
+                if rk is None:
+                    dk[bi, :, khi, :] = dkr
+                else:
+                    dkx, _ = rope_backward(k[b, kv_rows, hk, :][:, None, :], rk[kv_rows], dkr[:, None, :])
+                    dk[bi, :, khi, :] = dkx[:, 0, :]
         res["dk"] = dk
         res["dv"] = dv
     return res

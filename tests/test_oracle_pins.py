@@ -482,3 +482,82 @@ def test_chunkwise_text_conditioning_is_cross_attention_per_chunk():
         want = torch_reference(q[:, qs], k[:, ks], v[:, ks], offs([q_lens[c]]), offs([t_lens[c]]), gq, gk,
                                mask=torch.ones(q_lens[c], t_lens[c], dtype=torch.bool))
         np.testing.assert_allclose(o[:, qs], want, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- rotary embedding
+
+def test_rope_with_zero_angles_changes_nothing():
+    rng = np.random.default_rng(51)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [5, 7], [5, 7], 4, 2, 8)
+    z = np.zeros((12, 4))
+    o0, l0 = orc.forward(q, k, v, qo, ko, gq, gk)
+    o1, l1 = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=z, rope_k=z)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def test_rope_with_one_angle_table_row_for_every_token_changes_nothing():
+    """The same rotation of every q and k leaves all dot products unchanged (unit
+    gains: the norm's per-feature gain would not commute with the rotation)."""
+    rng = np.random.default_rng(52)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [4, 6, 3], [4, 6, 3], 4, 2, 16, gamma=False)
+    t = np.tile(rng.uniform(-3, 3, (1, 8)), (13, 1))
+    o0, _ = orc.forward(q, k, v, qo, ko, gq, gk)
+    o1, _ = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=t, rope_k=t)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    t2 = rng.uniform(-3, 3, (13, 8))
+    o2, _ = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=t2, rope_k=t2)
+    assert not np.allclose(o2, o0)
+
+
+def test_rope_on_positions_depends_only_on_relative_position():
+    """Angles s * w_i (one axis): shifting every position by the same amount
+    leaves the attention unchanged (unit gains)."""
+    rng = np.random.default_rng(53)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [5, 4, 6], [5, 4, 6], 4, 1, 16, gamma=False)
+    w = 1.0 / (100.0 ** (np.arange(8) / 8))
+    pos = np.arange(15)[:, None]
+    o0, l0 = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=pos * w, rope_k=pos * w)
+    o1, l1 = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=(pos + 37) * w, rope_k=(pos + 37) * w)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=1e-12)
+
+
+def test_rope_backward_matches_central_finite_differences():
+    rng = np.random.default_rng(54)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [2, 3], [1, 2, 3], 2, 1, 4)
+    tq = rng.uniform(-2, 2, (5, 2))
+    tk = rng.uniform(-2, 2, (6, 2))
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk, rope_q=tq, rope_k=tk)
+    params = [q, k, v, gq, gk, tq, tk]
+
+    def loss(pp):
+        o, _ = orc.forward(pp[0], pp[1], pp[2], qo, ko, pp[3], pp[4], rope_q=pp[5], rope_k=pp[6])
+        return float(np.sum(o * do))
+
+    h = 1e-6
+    for pi, name in enumerate(["dq", "dk", "dv", "dgamma_q", "dgamma_k", "drope_q", "drope_k"]):
+        num = np.zeros_like(params[pi])
+        it = np.nditer(params[pi], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            pp = [p.copy() for p in params]
+            pp[pi][idx] += h
+            lp = loss(pp)
+            pp[pi][idx] -= 2 * h
+            num[idx] = (lp - loss(pp)) / (2 * h)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_rope_backward_rows_match_full_backward():
+    rng = np.random.default_rng(55)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [5, 4, 6], [5, 4, 6], 4, 2, 8)
+    tq = rng.uniform(-3, 3, (15, 4))
+    tk = rng.uniform(-3, 3, (15, 4))
+    do = rng.standard_normal(q.shape)
+    full = orc.backward(q, k, v, do, qo, ko, gq, gk, rope_q=tq, rope_k=tk)
+    rows, kv_rows = np.array([0, 6, 9, 14]), np.array([2, 7, 12])
+    part = orc.backward_rows(q, k, v, do, qo, ko, gq, gk, q_rows=rows, kv_rows=kv_rows, rope_q=tq, rope_k=tk)
+    np.testing.assert_allclose(part["dq"][0], full["dq"][0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dk"][0], full["dk"][0, kv_rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dv"][0], full["dv"][0, kv_rows], rtol=0, atol=1e-12)

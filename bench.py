@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 DATASHEET_BF16_TFLOPS = 2250.0   # NVIDIA HGX B200 dense bf16, for context only
+HEAD_START_CYCLES = 2_000_000   # GPU spin queued ahead of each timed step (~1 ms at 1.965 GHz)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -221,6 +222,27 @@ def run_ours(args, w, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     l2_flush = torch.empty(512 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
 
+    # rotary angle tables (workloads with rope) stay on the device: a training loop
+    # computes them there from its learnable frequencies
+    rq, rk = inp.get("rope_q"), inp.get("rope_k")
+
+    def fwd_call(q_, k_, v_, out_, lse_):
+        if w.rope:
+            bca.magi_bca_fwd_rope(q_, k_, v_, w.q_offsets, w.kv_offsets, gq, gk, rq, rk, out=out_, lse=lse_,
+                                  stream=stream, kv_range=w.kv_range)
+        else:
+            bca.magi_bca_fwd(q_, k_, v_, w.q_offsets, w.kv_offsets, gq, gk, out=out_, lse=lse_, stream=stream,
+                             kv_range=w.kv_range)
+
+    def bwd_call(q_, k_, v_, out_, do_, lse_, dq_, dk_, dv_):
+        if w.rope:
+            bca.magi_bca_bwd_rope(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, rq, rk, dq=dq_,
+                                  dk=dk_, dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream,
+                                  kv_range=w.kv_range)
+        else:
+            bca.magi_bca_bwd(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, dq=dq_, dk=dk_,
+                             dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range)
+
     def step(ev=None, kev=None):
         # ev: events around the forward and backward calls; kev: a pair the
         # library records around the dominant main kernel (the backward's when
@@ -229,15 +251,13 @@ def run_ours(args, w, world, rank, local):
             ev[0].record(stream)
         if kev is not None and not do_bwd:
             bca.magi_bca_profile_events(kev[0], kev[1])
-        bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, out=out, lse=lse, stream=stream,
-                         kv_range=w.kv_range)
+        fwd_call(q, k, v, out, lse)
         if ev is not None:
             ev[1].record(stream)
         if do_bwd:
             if kev is not None:
                 bca.magi_bca_profile_events(kev[0], kev[1])
-            bca.magi_bca_bwd(q, k, v, out, inp["dout"], lse, w.q_offsets, w.kv_offsets, gq, gk, dq=dq, dk=dk,
-                             dv=dv, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range)
+            bwd_call(q, k, v, out, inp["dout"], lse, dq, dk, dv)
             if ev is not None:
                 ev[2].record(stream)
         if kev is not None:
@@ -257,9 +277,17 @@ def run_ours(args, w, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
+    host_s = []
     for i in range(args.steps):
         l2_flush.zero_()           # inputs of small workloads fit in L2: flush between steps
+        # a bounded spin (about 1 ms) keeps the GPU busy while the host enqueues
+        # the step, so the events time the device work and not the host's
+        # argument marshalling (which a training loop overlaps with the previous
+        # step); the host time per step is reported beside it
+        torch.cuda._sleep(HEAD_START_CYCLES)
+        h0 = time.perf_counter()
         step(evs[i], kevs[i])
+        host_s.append(time.perf_counter() - h0)
     torch.cuda.synchronize()
     barrier(world)
     t_wall = time.perf_counter() - t_wall0
@@ -318,12 +346,9 @@ def run_ours(args, w, world, rank, local):
         stream.wait_event(ev_in[n])
         if i >= 2:
             stream.wait_event(ev_out[n])               # step i-2's results are out of this set
-        bca.magi_bca_fwd(b["q"], b["k"], b["v"], w.q_offsets, w.kv_offsets, gq, gk, out=b["out"], lse=b["lse"],
-                         stream=stream, kv_range=w.kv_range)
+        fwd_call(b["q"], b["k"], b["v"], b["out"], b["lse"])
         if do_bwd:
-            bca.magi_bca_bwd(b["q"], b["k"], b["v"], b["out"], b["dout"], b["lse"], w.q_offsets, w.kv_offsets,
-                             gq, gk, dq=b["dq"], dk=b["dk"], dv=b["dv"], dgamma_q=dgq, dgamma_k=dgk, workspace=ws,
-                             stream=stream, kv_range=w.kv_range)
+            bwd_call(b["q"], b["k"], b["v"], b["out"], b["dout"], b["lse"], b["dq"], b["dk"], b["dv"])
         ev_done[n].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[n])
@@ -399,10 +424,12 @@ def run_ours(args, w, world, rank, local):
         "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
                    "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
                    "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
-                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range,
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range, "rope": w.rope,
                    "parallelism": f"replicas x{world}",
                    "l2": "flushed (512 MB write) between timed steps, outside the step events",
+                   "head_start": "~1 ms GPU spin queued before each step's first event",
                    "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4) if do_bwd else None,
+                   "host_enqueue_ms_per_step": round(1e3 * float(np.median(host_s)), 4),
                    "useful_tflop_per_step": round(flops_step / 1e12, 4)},
         "pct_of_measured_peak": round(100 * value / world / peak, 2),
         "pct_of_datasheet_peak": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
@@ -428,11 +455,13 @@ def bca_bwd_launches():
 def oracle_sample(w, inp, rows, do_bwd):
     """Runs the oracle on the given query rows (all heads, batch 0)."""
     from oracle import bca_oracle as orc
+    rq, rk = inp.get("rope_q"), inp.get("rope_k")
     orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
-                     inp["gamma_k"], rows, batches=[0], kv_range=w.kv_range)
+                     inp["gamma_k"], rows, batches=[0], kv_range=w.kv_range, rope_q=rq, rope_k=rk)
     if do_bwd:
         orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0], kv_range=w.kv_range)
+                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0], kv_range=w.kv_range,
+                          rope_q=rq, rope_k=rk)
 
 
 def sample_flops(w, rows, do_bwd):
@@ -506,7 +535,7 @@ def run_reference(args, w, world, rank):
         "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
                    "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
                    "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
-                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range},
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range, "rope": w.rope},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

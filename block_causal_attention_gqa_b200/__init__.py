@@ -19,7 +19,7 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_noalloc", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
+__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_fwd_rope", "magi_bca_bwd_rope", "magi_bca_bwd_noalloc", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
            "magi_bca_status_string", "magi_bca_last_device_status", "magi_bca_profile_events", "MagiBcaError",
            "Dims", "library",
            "library_path", "EXPORTED_SYMBOLS"]
@@ -30,7 +30,7 @@ library_path = os.path.join(_HERE, "libmagi_bca.so")
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
                     "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule",
-                    "magi_bca_profile_events"]
+                    "magi_bca_profile_events", "magi_bca_fwd_rope", "magi_bca_bwd_rope"]
 
 
 class MagiBcaError(RuntimeError):
@@ -85,6 +85,11 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_bwd_schedule.restype = ctypes.c_int64
     lib.magi_bca_version.argtypes = []
     lib.magi_bca_version.restype = ctypes.c_char_p
+    lib.magi_bca_fwd_rope.argtypes = [vp, vp, vp, i32p, i32p, f32p, f32p, vp, vp, vp, f32p, dp, vp]
+    lib.magi_bca_fwd_rope.restype = ctypes.c_int
+    lib.magi_bca_bwd_rope.argtypes = [vp, vp, vp, vp, vp, f32p, i32p, i32p, f32p, f32p, vp, vp, vp, vp, vp, f32p,
+                                      f32p, vp, vp, vp, ctypes.c_size_t, dp, vp]
+    lib.magi_bca_bwd_rope.restype = ctypes.c_int
     lib.magi_bca_profile_events.argtypes = [vp, vp]
     lib.magi_bca_profile_events.restype = ctypes.c_int
     _lib = lib
@@ -162,11 +167,8 @@ def _stream_handle(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out=None, lse=None,
-                 softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True,
-                 kv_range: int = 0):
-    """Forward.  q [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] bf16; gammas fp32 [D];
-    offsets: host int arrays of chunk boundaries.  Returns (out, lse)."""
+def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps, stream,
+         want_lse, kv_range, rope=None):
     import torch
     _check_bf16("q", q)
     B, Sq, Hq, D = q.shape
@@ -185,26 +187,53 @@ def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, o
     if lse is not None:
         _check_f32("lse", lse, (B, Hq, Sq))
     dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
+    ptr = lambda t: t.data_ptr() if t is not None else None
     with torch.cuda.device(q.device):
-        st = library().magi_bca_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _i32p(qo), _i32p(ko),
-                                    gamma_q.data_ptr(), gamma_k.data_ptr(), out.data_ptr(),
-                                    lse.data_ptr() if lse is not None else None, ctypes.byref(dims),
-                                    _stream_handle(stream, q.device))
+        if rope is None:
+            st = library().magi_bca_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _i32p(qo), _i32p(ko),
+                                        gamma_q.data_ptr(), gamma_k.data_ptr(), out.data_ptr(), ptr(lse),
+                                        ctypes.byref(dims), _stream_handle(stream, q.device))
+        else:
+            rq, rk = rope
+            if rq is not None:
+                _check_f32("rope_q", rq, (Sq, D // 2))
+            if rk is not None:
+                _check_f32("rope_k", rk, (Skv, D // 2))
+            st = library().magi_bca_fwd_rope(q.data_ptr(), k.data_ptr(), v.data_ptr(), _i32p(qo), _i32p(ko),
+                                             gamma_q.data_ptr(), gamma_k.data_ptr(), ptr(rq), ptr(rk),
+                                             out.data_ptr(), ptr(lse), ctypes.byref(dims),
+                                             _stream_handle(stream, q.device))
     if st != 0:
-        raise MagiBcaError(st, "magi_bca_fwd")
+        raise MagiBcaError(st, "magi_bca_fwd" if rope is None else "magi_bca_fwd_rope")
     return out, lse
+
+
+def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out=None, lse=None,
+                 softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True,
+                 kv_range: int = 0):
+    """Forward.  q [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] bf16; gammas fp32 [D];
+    offsets: host int arrays of chunk boundaries.  Returns (out, lse)."""
+    return _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps,
+                stream, want_lse, kv_range)
+
+
+def magi_bca_fwd_rope(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, rope_q, rope_k, out=None,
+                      lse=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
+                      want_lse: bool = True, kv_range: int = 0):
+    """Forward with rotary angles (fp32 [Sq, D/2] / [Skv, D/2] per token, or
+    None) applied to q and k before the norm.  Returns (out, lse)."""
+    return _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps,
+                stream, want_lse, kv_range, rope=(rope_q, rope_k))
 
 
 def magi_bca_bwd_workspace_size(dims: Dims) -> int:
     return int(library().magi_bca_bwd_workspace_size(ctypes.byref(dims)))
 
 
-def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
-                 dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
-                 workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
-                 kv_range: int = 0):
-    """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
-    respect to the raw (pre-norm) q and k."""
+def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv, dgamma_q,
+         dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range, rope=None):
+    """Shared marshalling of magi_bca_bwd and (rope = (rope_q, rope_k, drope_q,
+    drope_k)) magi_bca_bwd_rope."""
     import torch
     _check_bf16("q", q)
     B, Sq, Hq, D = q.shape
@@ -230,17 +259,57 @@ def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gam
     ws_bytes = magi_bca_bwd_workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), device=q.device, dtype=torch.uint8)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    common = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+              _i32p(qo), _i32p(ko), gamma_q.data_ptr(), gamma_k.data_ptr())
+    tail = (workspace.data_ptr(), workspace.numel() * workspace.element_size(), ctypes.byref(dims),
+            _stream_handle(stream, q.device))
     with torch.cuda.device(q.device):
-        st = library().magi_bca_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
-                                    lse.data_ptr(), _i32p(qo), _i32p(ko), gamma_q.data_ptr(), gamma_k.data_ptr(),
-                                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                    dgamma_q.data_ptr() if dgamma_q is not None else None,
-                                    dgamma_k.data_ptr() if dgamma_k is not None else None,
-                                    workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                    ctypes.byref(dims), _stream_handle(stream, q.device))
+        if rope is None:
+            st = library().magi_bca_bwd(*common, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ptr(dgamma_q),
+                                        ptr(dgamma_k), *tail)
+        else:
+            rq, rk, drq, drk = rope
+            st = library().magi_bca_bwd_rope(*common, ptr(rq), ptr(rk), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                             ptr(dgamma_q), ptr(dgamma_k), ptr(drq), ptr(drk), *tail)
     if st != 0:
-        raise MagiBcaError(st, "magi_bca_bwd")
+        raise MagiBcaError(st, "magi_bca_bwd" if rope is None else "magi_bca_bwd_rope")
     return dq, dk, dv, dgamma_q, dgamma_k
+
+
+def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
+                 dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
+                 workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
+                 kv_range: int = 0):
+    """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
+    respect to the raw (pre-norm) q and k."""
+    return _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
+                dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range)
+
+
+def magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
+                      rope_q, rope_k, dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None,
+                      want_dgamma: bool = True, want_drope: bool = True, workspace=None,
+                      softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, kv_range: int = 0):
+    """Backward of magi_bca_fwd_rope.  Returns (dq, dk, dv, dgamma_q, dgamma_k,
+    drope_q, drope_k); dq/dk are with respect to the raw (pre-rotation,
+    pre-norm) q and k; drope_* (fp32 [seqlen, D/2], summed over batch and
+    heads) are None where the angle table is None or want_drope is False."""
+    import torch
+    D = q.shape[3]
+    drq = drk = None
+    if rope_q is not None:
+        _check_f32("rope_q", rope_q, (q.shape[1], D // 2))
+        if want_drope:
+            drq = torch.empty_like(rope_q)
+    if rope_k is not None:
+        _check_f32("rope_k", rope_k, (k.shape[1], D // 2))
+        if want_drope:
+            drk = torch.empty_like(rope_k)
+    res = _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
+               dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range,
+               rope=(rope_q, rope_k, drq, drk))
+    return res + (drq, drk)
 
 
 def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,

@@ -277,6 +277,14 @@ int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
 int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
                  const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets, const float* gamma_q,
                  const float* gamma_k, magi_bca_bf16* out, float* lse, const magi_bca_dims* dims, void* stream) {
+  return magi_bca_fwd_rope(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, nullptr, nullptr, out, lse,
+                           dims, stream);
+}
+
+int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                      const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets, const float* gamma_q,
+                      const float* gamma_k, const float* rope_q, const float* rope_k, magi_bca_bf16* out, float* lse,
+                      const magi_bca_dims* dims, void* stream) {
   int st = validate_dims(dims);
   if (st != MAGI_BCA_OK) return st;
   const magi_bca_dims& d = *dims;
@@ -296,7 +304,8 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   void* kn = nullptr;
   st = knorm_buffer(dev, cs, (size_t)kv_rows * d.head_dim * 2, &kn);
   if (st != MAGI_BCA_OK) return st;
-  cudaError_t ke = launch_knorm(k, static_cast<uint16_t*>(kn), kv_rows, d.head_dim, d.rms_eps, cs);
+  cudaError_t ke = launch_knorm(k, static_cast<uint16_t*>(kn), kv_rows, d.head_dim, d.rms_eps, cs, rope_k,
+                                d.heads_kv, d.seqlen_kv);
   if (ke != cudaSuccess) return cuda_fail("key normalisation launch", ke);
   CUtensorMap tq, tk, tv;
   if (make_map(&tq, q, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
@@ -310,6 +319,7 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
   p.kv_range = d.kv_range;
+  p.rope_q = rope_q;
   p.gamma_q = gamma_q;
   p.gamma_k = gamma_k;
   p.out = out;
@@ -337,6 +347,18 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
                  const int32_t* kv_chunk_offsets, const float* gamma_q, const float* gamma_k, magi_bca_bf16* dq,
                  magi_bca_bf16* dk, magi_bca_bf16* dv, float* dgamma_q, float* dgamma_k, void* workspace,
                  size_t workspace_bytes, const magi_bca_dims* dims, void* stream) {
+  return magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, nullptr,
+                           nullptr, dq, dk, dv, dgamma_q, dgamma_k, nullptr, nullptr, workspace, workspace_bytes, dims,
+                           stream);
+}
+
+int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                      const magi_bca_bf16* out, const magi_bca_bf16* dout, const float* lse,
+                      const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets, const float* gamma_q,
+                      const float* gamma_k, const float* rope_q, const float* rope_k, magi_bca_bf16* dq,
+                      magi_bca_bf16* dk, magi_bca_bf16* dv, float* dgamma_q, float* dgamma_k, float* drope_q,
+                      float* drope_k, void* workspace, size_t workspace_bytes, const magi_bca_dims* dims,
+                      void* stream) {
   int st = validate_dims(dims);
   if (st != MAGI_BCA_OK) return st;
   const magi_bca_dims& d = *dims;
@@ -371,6 +393,10 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
   p.kv_range = d.kv_range;
+  p.rope_q = rope_q;
+  p.rope_k = rope_k;
+  p.drope_q = rope_q != nullptr ? drope_q : nullptr;
+  p.drope_k = rope_k != nullptr ? drope_k : nullptr;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

@@ -165,6 +165,14 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
     if (p.dgamma_q) p.dgamma_q[threadIdx.x] = 0.f;
     if (p.dgamma_k) p.dgamma_k[threadIdx.x] = 0.f;
   }
+  // rotary angle gradients are sums over batch and heads: zero them here
+  {
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, nth = (int64_t)gridDim.x * blockDim.x;
+    if (p.drope_q)
+      for (int64_t i = tid; i < (int64_t)p.seqlen_q * (D / 2); i += nth) p.drope_q[i] = 0.f;
+    if (p.drope_k)
+      for (int64_t i = tid; i < (int64_t)p.seqlen_kv * (D / 2); i += nth) p.drope_k[i] = 0.f;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t n_q = (int64_t)p.batch * p.seqlen_q * p.heads_q;
@@ -178,7 +186,8 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
   for (int64_t rr = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); rr < n_q + n_k; rr += warps) {
     if (rr >= n_q) {
       const int64_t r = rr - n_q;
-      knorm_row<D>(p.k + r * D, p.kn + r * D, lane, p.eps);
+      const float* ang = p.rope_k ? p.rope_k + ((r / p.heads_kv) % p.seqlen_kv) * (D / 2) : nullptr;
+      knorm_row<D>(p.k + r * D, p.kn + r * D, lane, p.eps, ang);
       IO::store_zero_f32(p.dvacc + r * D, lane);
       IO::store_zero_f32(p.dkacc + r * D, lane);
       continue;
@@ -189,6 +198,12 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
     IO::load_bf16(p.out + r * D, lane, o);
     IO::load_bf16(p.dout + r * D, lane, g);
     const float rq = rms_inv<D>(warp_sumsq_row<E>(x), p.eps);
+    if (p.rope_q) {   // rotate after the RMS of the raw row, as the forward's prologue does
+      float y[E];
+      rope_warp<D>(x, p.rope_q + ((r / p.heads_q) % p.seqlen_q) * (D / 2), lane, y);
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = y[e];
+    }
     float qh[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) qh[e] = x[e] * rq * qscale[lane * E + e];
@@ -637,8 +652,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // RMSNorm Jacobian, dgamma_q += dq~ q^.  Key rows: dv = bf16(dV), gamma_k dk~ =
 // G_k / log2(e), dk through the Jacobian, dgamma_k += dk~ k^.  With r = rsqrt
 // (mean x^2 + eps), x^ = x r and g = gamma dx~:  dx = r (g - x^ mean(g x^)).
-template <int D>
-__global__ void __launch_bounds__(256, 4) bca_bwd_finalize_kernel(const BwdParams p) {
+template <int D, bool kRope>
+__global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p) {
   using IO = RowIO<D>;
   constexpr int E = IO::E;
   __shared__ float red[2][8][D];
@@ -659,6 +674,11 @@ __global__ void __launch_bounds__(256, 4) bca_bwd_finalize_kernel(const BwdParam
   auto finish_row = [&](int64_t rr, float (&x)[E], float (&g)[E], const float (&dvv)[E]) {
     const bool is_q = rr < n_q;
     const int64_t r = is_q ? rr : rr - n_q;
+    // with rotary angles the normalised vector is rope(x): the Jacobian below
+    // acts on it, and its result goes back through the transposed rotation
+    const float* rope = kRope ? (is_q ? p.rope_q : p.rope_k) : nullptr;
+    float* drope = kRope ? (is_q ? p.drope_q : p.drope_k) : nullptr;
+    const int64_t tok = (r / (is_q ? p.heads_q : p.heads_kv)) % (is_q ? p.seqlen_q : p.seqlen_kv);
     float dqt[E];
     // g = gamma * dx~   (for query rows dq~ = scale gamma_k G_q is kept for dgamma_q)
 #pragma unroll
@@ -670,6 +690,16 @@ __global__ void __launch_bounds__(256, 4) bca_bwd_finalize_kernel(const BwdParam
 #pragma unroll
     for (int e = 0; e < E; ++e) ss = fmaf(x[e], x[e], ss);
     const float rinv = rsqrtf(warp_sum(ss) * (1.0f / D) + p.eps);
+    float cs[E], sn[E], y[E];
+    if (rope != nullptr) {   // warp-uniform
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xp = __shfl_xor_sync(0xffffffffu, x[e], 16);
+        sincosf(__ldg(rope + tok * (D / 2) + (lane & 15) * E + e), &sn[e], &cs[e]);
+        y[e] = lane < 16 ? rope_first(x[e], xp, cs[e], sn[e]) : rope_second(xp, x[e], cs[e], sn[e]);
+        x[e] = y[e];
+      }
+    }
     float dot = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -680,6 +710,17 @@ __global__ void __launch_bounds__(256, 4) bca_bwd_finalize_kernel(const BwdParam
     float o[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] = rinv * (g[e] - x[e] * mean_dot);
+    if (rope != nullptr) {
+      // o = gradient w.r.t. y = rope(raw); pair (a, b) = (lane < 16, lane ^ 16):
+      // d angle = -o_a y_b + o_b y_a, d raw_a = o_a c + o_b s, d raw_b = o_b c - o_a s
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float op = __shfl_xor_sync(0xffffffffu, o[e], 16);
+        const float yp = __shfl_xor_sync(0xffffffffu, y[e], 16);
+        if (drope != nullptr && lane < 16) atomicAdd(drope + tok * (D / 2) + lane * E + e, op * y[e] - o[e] * yp);
+        o[e] = lane < 16 ? fmaf(op, sn[e], o[e] * cs[e]) : fmaf(-op, sn[e], o[e] * cs[e]);
+      }
+    }
     if (is_q) {
       IO::store_bf16(p.dq + r * D, lane, o);
 #pragma unroll
@@ -750,14 +791,21 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
   // one wave of the row kernels (grid-stride loops over one warp per row)
-  static int prep_per_sm[2] = {0, 0}, fin_per_sm[2] = {0, 0};
+  static int prep_per_sm[2] = {0, 0}, fin_per_sm[2][2] = {{0, 0}, {0, 0}};
+  const bool rope = p.rope_q != nullptr || p.rope_k != nullptr;
   int& prep_occ = prep_per_sm[D == 128];
-  int& fin_occ = fin_per_sm[D == 128];
+  int& fin_occ = fin_per_sm[D == 128][rope];
   if (prep_occ == 0) {
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_prep_kernel<D>, 256, 0);
     prep_occ = std::max(n, 1);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D>, 256, 0);
+  }
+  if (fin_occ == 0) {
+    int n = 0;
+    if (rope)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D, true>, 256, 0);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D, false>, 256, 0);
     fin_occ = std::max(n, 1);
   }
   const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * prep_occ);
@@ -778,7 +826,10 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   profile_mark(1, stream);
   const int64_t frows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
   const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * fin_occ);
-  bca_bwd_finalize_kernel<D><<<fin_blocks, 256, 0, stream>>>(p);
+  if (rope)
+    bca_bwd_finalize_kernel<D, true><<<fin_blocks, 256, 0, stream>>>(p);
+  else
+    bca_bwd_finalize_kernel<D, false><<<fin_blocks, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -96,7 +96,7 @@ __device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
 }
 
 
-template <int D>
+template <int D, bool kRope>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -242,16 +242,33 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int bar_id = 1 + s;
       bool ok = true;
 
-      // Q prologue: RMSNorm the row and fold gains, scale and log2(e) into it.
+      // Q prologue: RMSNorm the row and fold gains, scale and log2(e) into it;
+      // with rotary angles the row is rotated first (the RMS is the raw row's:
+      // a rotation keeps it).
       ok = warp_wait(&bars->q_full[s], 0, ok, p.status, kErrQ);
+      const int row = (s ? m01 : m00) + r;
       if (ok) {
         const float rq = rms_inv<D>(row_sumsq_swizzled_warp_order<D>(q_tile, r), p.eps);
+        if (kRope && row < p.seqlen_q) {
+          const float* ang = p.rope_q + (size_t)row * (D / 2);
 #pragma unroll
-        for (int box = 0; box < D / 64; ++box) {
+          for (int pc = 0; pc < D / 16; ++pc) {
+            const int fa = pc * 8, fb = fa + D / 2;
+            uint4* pa = reinterpret_cast<uint4*>(q_tile + (fa / 64) * 16384 + sw128_offset(r, fa % 64));
+            uint4* pb = reinterpret_cast<uint4*>(q_tile + (fb / 64) * 16384 + sw128_offset(r, fb % 64));
+            uint4 va = *pa, vb = *pb;
+            fold_q_pair<D>(va, vb, rq, qscale, fa, ang + fa);
+            *pa = va;
+            *pb = vb;
+          }
+        } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint4* ptr = reinterpret_cast<uint4*>(q_tile + box * 16384 + sw128_offset(r, c * 8));
-            *ptr = fold_q_chunk(*ptr, rq, qscale, box * 64 + c * 8);
+          for (int box = 0; box < D / 64; ++box) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4* ptr = reinterpret_cast<uint4*>(q_tile + box * 16384 + sw128_offset(r, c * 8));
+              *ptr = fold_q_chunk(*ptr, rq, qscale, box * 64 + c * 8);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -260,7 +277,6 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (r == 0 && ok) mbar_arrive(&bars->q_ready[s]);
 
       // Visible-key end of this row.
-      const int row = (s ? m01 : m00) + r;
       int limit = p.seqlen_kv, kv_first = 0;   // visible keys [kv_first, limit)
       if (row < p.seqlen_q) {
         const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
@@ -437,48 +453,57 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // so both passes see identical key operands.
 template <int D>
 __global__ void __launch_bounds__(256) bca_knorm_kernel(const uint16_t* __restrict__ k, uint16_t* __restrict__ kn,
-                                                         int64_t rows, float eps) {
+                                                         int64_t rows, float eps, const float* __restrict__ rope,
+                                                         int heads, int seqlen) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps)
-    knorm_row<D>(k + r * D, kn + r * D, lane, eps);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+    // row r = (b * seqlen + token) * heads + h; the angles are the token's
+    const float* ang = rope != nullptr ? rope + ((r / heads) % seqlen) * (D / 2) : nullptr;
+    knorm_row<D>(k + r * D, kn + r * D, lane, eps, ang);
+  }
 }
 
-cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream) {
+cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream,
+                         const float* rope, int heads, int seqlen) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * 16);
   if (blocks <= 0) return cudaSuccess;
   if (head_dim == 128)
-    bca_knorm_kernel<128><<<blocks, 256, 0, stream>>>(k, kn, rows, eps);
+    bca_knorm_kernel<128><<<blocks, 256, 0, stream>>>(k, kn, rows, eps, rope, heads, seqlen);
   else
-    bca_knorm_kernel<64><<<blocks, 256, 0, stream>>>(k, kn, rows, eps);
+    bca_knorm_kernel<64><<<blocks, 256, 0, stream>>>(k, kn, rows, eps, rope, heads, seqlen);
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool kRope>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, int n_units, cudaStream_t stream) {
   using L = FwdLayout<D>;
-  static uint64_t configured = 0;  // one bit per device ordinal that has the attribute set
+  static uint64_t configured = 0;  // one bit per device ordinal that has the attribute set (per variant)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((configured >> dev) & 1u)) {
-    e = cudaFuncSetAttribute(bca_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    e = cudaFuncSetAttribute(bca_fwd_kernel<D, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     if (dev < 64) configured |= uint64_t(1) << dev;
   }
-  bca_fwd_kernel<D><<<n_units, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  bca_fwd_kernel<D, kRope><<<n_units, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream) {
   if (n_units <= 0) return cudaSuccess;
-  if (head_dim == 128) return launch_fwd_d<128>(tq, tk, tv, p, n_units, stream);
-  return launch_fwd_d<64>(tq, tk, tv, p, n_units, stream);
+  const bool rope = p.rope_q != nullptr;
+  if (head_dim == 128)
+    return rope ? launch_fwd_d<128, true>(tq, tk, tv, p, n_units, stream)
+                : launch_fwd_d<128, false>(tq, tk, tv, p, n_units, stream);
+  return rope ? launch_fwd_d<64, true>(tq, tk, tv, p, n_units, stream)
+              : launch_fwd_d<64, false>(tq, tk, tv, p, n_units, stream);
 }
 
 size_t fwd_smem_bytes(int head_dim) {

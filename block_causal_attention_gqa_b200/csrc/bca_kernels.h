@@ -16,6 +16,7 @@ struct FwdParams {
   const int32_t* kv_offsets;  // device copy of the kv chunk offsets
   int n_q_chunks, n_kv_chunks;
   int kv_range;               // 0 = no limit, else chunks visible back from the row's own
+  const float* rope_q;        // rotary angles of the query tokens [Sq, D/2] or nullptr
   const float* gamma_q;
   const float* gamma_k;
   uint16_t* out;              // [B, Sq, Hq, D] bf16
@@ -40,6 +41,10 @@ struct BwdParams {
   const int32_t* kv_offsets;
   int n_q_chunks, n_kv_chunks;
   int kv_range;               // 0 = no limit, else chunks visible back from the row's own
+  const float* rope_q;        // rotary angles [Sq, D/2] / [Skv, D/2], or nullptr
+  const float* rope_k;
+  float* drope_q;             // their gradients (summed over batch and heads), or nullptr
+  float* drope_k;
   // outputs
   uint16_t* dq;
   uint16_t* dk;
@@ -70,8 +75,10 @@ cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUt
                        const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream);
 int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 
-// K^ = bf16(k rsqrt(mean k^2 + eps)) for `rows` rows of head_dim features.
-cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream);
+// K^ = bf16(rope(k) rsqrt(mean k^2 + eps)) for `rows` rows [B, seqlen, heads] of head_dim
+// features; `rope` = per-token angles [seqlen, head_dim / 2] or nullptr (no rotation).
+cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head_dim, float eps, cudaStream_t stream,
+                         const float* rope, int heads, int seqlen);
 
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
                        int head_dim, int n_units, cudaStream_t stream);

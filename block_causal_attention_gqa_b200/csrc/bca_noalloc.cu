@@ -129,6 +129,8 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.n_q_chunks = d.n_q_chunks;
   p.n_kv_chunks = d.n_kv_chunks;
   p.kv_range = d.kv_range;
+  p.rope_q = p.rope_k = nullptr;
+  p.drope_q = p.drope_k = nullptr;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

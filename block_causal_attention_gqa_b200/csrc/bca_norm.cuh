@@ -93,11 +93,39 @@ __device__ __forceinline__ float rms_inv(float sumsq, float eps) {
   return rsqrtf(sumsq * (1.0f / D) + eps);
 }
 
-// One key row: dst = bf16(src * r_k), r_k = 1 / RMS(src), by one warp (lane
-// holds features [lane*D/32, lane*D/32 + D/32)).  The forward's key pre-pass
-// and the backward's prep both call this, so both see the same K^ bits.
+// Rotary pair: (a, b) = (x_i, x_{i+D/2}) rotated by the angle whose cosine and
+// sine are c, s.  Explicit roundings, so every kernel that rotates a row (the
+// forward's Q prologue and key pre-pass, the backward's prep and finalize)
+// gets the same bits.
+__device__ __forceinline__ float rope_first(float a, float b, float c, float s) {
+  return __fmaf_rn(-b, s, __fmul_rn(a, c));
+}
+__device__ __forceinline__ float rope_second(float a, float b, float c, float s) {
+  return __fmaf_rn(a, s, __fmul_rn(b, c));
+}
+
+// Warp form: lane holds features [lane*E, lane*E + E) (E = D/32), so the pair
+// partner of its features (i +- D/2) sits in lane ^ 16.  `ang` is the row's
+// D/2 angles (nullptr: no rotation); y receives the rotated features.
 template <int D>
-__device__ __forceinline__ void knorm_row(const uint16_t* src, uint16_t* dst, int lane, float eps) {
+__device__ __forceinline__ void rope_warp(const float (&x)[D / 32], const float* ang, int lane, float (&y)[D / 32]) {
+  constexpr int E = D / 32;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float xp = __shfl_xor_sync(0xffffffffu, x[e], 16);
+    float sn, cs;
+    sincosf(__ldg(ang + (lane & 15) * E + e), &sn, &cs);
+    y[e] = lane < 16 ? rope_first(x[e], xp, cs, sn) : rope_second(xp, x[e], cs, sn);
+  }
+}
+
+// One key row: dst = bf16(rope(src) * r_k), r_k = 1 / RMS(src) (a rotation
+// keeps the RMS), by one warp (lane holds features [lane*D/32, lane*D/32 +
+// D/32)); `ang` = the token's rotary angles or nullptr.  The forward's key
+// pre-pass and the backward's prep both call this, so both see the same K^ bits.
+template <int D>
+__device__ __forceinline__ void knorm_row(const uint16_t* src, uint16_t* dst, int lane, float eps,
+                                          const float* ang = nullptr) {
   constexpr int E = D / 32;
   float x[E];
   if constexpr (E == 4) {
@@ -113,6 +141,12 @@ __device__ __forceinline__ void knorm_row(const uint16_t* src, uint16_t* dst, in
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float rk = rms_inv<D>(ss, eps);
+  if (ang != nullptr) {   // warp-uniform
+    float y[E];
+    rope_warp<D>(x, ang, lane, y);
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] = y[e];
+  }
   if constexpr (E == 4) {
     uint2 w;
     w.x = sm100::pack_bf16x2(x[0] * rk, x[1] * rk);
@@ -134,6 +168,31 @@ __device__ __forceinline__ uint4 fold_q_chunk(uint4 v, float rq, const float* qs
     w[i] = sm100::pack_bf16x2(lo, hi);
   }
   return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The forward's query operand for a rotary pair of 16-byte chunks: va holds
+// features [d0, d0 + 8) and vb features [d0 + D/2, d0 + D/2 + 8); `ang` the
+// row's angles for d0 .. d0 + 7.  bf16(rope(q) * r_q * qscale[d]).
+template <int D>
+__device__ __forceinline__ void fold_q_pair(uint4& va, uint4& vb, float rq, const float* qscale, int d0,
+                                            const float* ang) {
+  uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a[2] = {bf16_lo(wa[i]), bf16_hi(wa[i])}, b[2] = {bf16_lo(wb[i]), bf16_hi(wb[i])};
+    float ya[2], yb[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float sn, cs;
+      sincosf(__ldg(ang + 2 * i + h), &sn, &cs);
+      ya[h] = rope_first(a[h], b[h], cs, sn) * rq * qscale[d0 + 2 * i + h];
+      yb[h] = rope_second(a[h], b[h], cs, sn) * rq * qscale[d0 + D / 2 + 2 * i + h];
+    }
+    wa[i] = sm100::pack_bf16x2(ya[0], ya[1]);
+    wb[i] = sm100::pack_bf16x2(yb[0], yb[1]);
+  }
+  va = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+  vb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
 }
 
 __device__ __forceinline__ float qscale_of(const float* gamma_q, const float* gamma_k, float scale_log2, int d) {

@@ -99,6 +99,23 @@ int magi_bca_fwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
                  magi_bca_bf16* out, float* lse,
                  const magi_bca_dims* dims, void* stream);
 
+/* Forward with rotary position embedding on q and k before the norm
+ * (MAGI-1 §2.2.2 and the notes' DiT-block sketch: learnable 3D RoPE, then
+ * QK-norm).  rope_q [seqlen_q, head_dim/2] and rope_k [seqlen_kv,
+ * head_dim/2] are fp32 device arrays of per-token rotation angles (radians),
+ * shared by every head and batch element; feature pair (i, i + head_dim/2) of
+ * token s rotates by angle[s][i]: y_i = x_i cos - x_{i+D/2} sin,
+ * y_{i+D/2} = x_{i+D/2} cos + x_i sin.  The 3D split (time, height, width)
+ * and the learnable frequencies live in the caller, which computes the
+ * angles.  Either table may be NULL (no rotation of that side).  Otherwise
+ * as magi_bca_fwd (which is this call with both tables NULL). */
+int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                      const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                      const float* gamma_q, const float* gamma_k,
+                      const float* rope_q, const float* rope_k,
+                      magi_bca_bf16* out, float* lse,
+                      const magi_bca_dims* dims, void* stream);
+
 /* Bytes of device workspace magi_bca_bwd needs for `dims` (0 on invalid dims). */
 size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims);
 
@@ -149,6 +166,22 @@ const char* magi_bca_status_string(int status);
  * (which CUDA call failed and its error string); "" if none.  Owned by the
  * library, valid until the thread's next failing call. */
 const char* magi_bca_last_error_detail(void);
+
+/* Backward of magi_bca_fwd_rope.  dq and dk are gradients with respect to
+ * the raw (pre-rotation, pre-norm) q and k.  drope_q [seqlen_q, head_dim/2]
+ * and drope_k [seqlen_kv, head_dim/2] (fp32, nullable; ignored where the
+ * matching angle table is NULL) receive the angle gradients summed over
+ * batch and heads, so the caller can continue into its learnable
+ * frequencies.  Otherwise as magi_bca_bwd (this call with NULL tables). */
+int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_bf16* v,
+                      const magi_bca_bf16* out, const magi_bca_bf16* dout, const float* lse,
+                      const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
+                      const float* gamma_q, const float* gamma_k,
+                      const float* rope_q, const float* rope_k,
+                      magi_bca_bf16* dq, magi_bca_bf16* dk, magi_bca_bf16* dv,
+                      float* dgamma_q, float* dgamma_k, float* drope_q, float* drope_k,
+                      void* workspace, size_t workspace_bytes,
+                      const magi_bca_dims* dims, void* stream);
 
 /* Reads (and clears) the device status word that bounded waits write when
  * they give up.  Synchronises with the device; returns MAGI_BCA_OK or

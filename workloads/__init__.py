@@ -30,7 +30,7 @@ from typing import Optional, Sequence
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "ORDER", "workload", "custom", "uniform_offsets",
+__all__ = ["Workload", "WORKLOADS", "ORDER", "workload", "custom", "uniform_offsets", "rope_angles",
            "make_inputs", "sample_rows"]
 
 
@@ -49,6 +49,7 @@ class Workload:
     gamma: str = "perturbed"     # "ones" or "perturbed" (1 + N(0, 0.1) per head-dim)
     token_scale: bool = False    # LogNormal(0, 0.5) per-token scale on q and k
     kv_range: int = 0            # KV range in chunks (0 = every earlier chunk); MAGI-1 §2.4.4, Fig. 12
+    rope: bool = False           # rotary angles for q and k (3D positions, see rope_angles)
 
     @property
     def seqlen_q(self) -> int:
@@ -96,9 +97,13 @@ WORKLOADS = {
     # against 1024 text tokens (MAGI-1 §2.2.2: cross-attention with QK-norm and GQA
     # to the T5 text condition; the text length is a reading), GQA 24/8.
     "xattn46k": Workload("xattn46k", 1, (46080,), (1024,), 24, 8, 128, seed=6, backward=True),
+    # model46k with rotary angles on q and k before the norm (MAGI-1 §2.2.2: learnable 3D
+    # RoPE; angles from the 6 x 24 x 40 latent grid of each chunk, see rope_angles).
+    "model46k_rope": Workload("model46k_rope", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760),
+                              24, 8, 128, seed=7, backward=True, rope=True),
 }
 
-ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k"]
+ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k", "model46k_rope"]
 
 
 def workload(name_or_index) -> Workload:
@@ -109,10 +114,31 @@ def workload(name_or_index) -> Workload:
 
 def custom(name: str, batch: int, q_chunks: Sequence[int], kv_chunks: Optional[Sequence[int]],
            heads_q: int, heads_kv: int, head_dim: int, seed: int, backward: bool = True,
-           gamma: str = "perturbed", token_scale: bool = False, kv_range: int = 0) -> Workload:
+           gamma: str = "perturbed", token_scale: bool = False, kv_range: int = 0,
+           rope: bool = False) -> Workload:
     kv = tuple(kv_chunks) if kv_chunks is not None else tuple(q_chunks)
     return Workload(name, batch, tuple(q_chunks), kv, heads_q, heads_kv, head_dim, seed,
-                    backward, gamma=gamma, token_scale=token_scale, kv_range=kv_range)
+                    backward, gamma=gamma, token_scale=token_scale, kv_range=kv_range, rope=rope)
+
+
+def rope_angles(positions: np.ndarray, head_dim: int, grid=(6, 24, 40), base: float = 10000.0) -> np.ndarray:
+    """Rotary angles [len(positions), head_dim/2] (fp32) for key/value token
+    positions: token t of the sequence sits at latent frame, row and column
+    (t // (H W), (t // W) % H, t % W) of a 6 x 24 x 40 grid per 5760-token
+    chunk (frames continue across chunks), and the head_dim/2 frequency pairs
+    are split into three near-equal groups, one per axis, with frequencies
+    base^(-j / n) inside a group.  (A stand-in for MAGI-1's learnable 3D RoPE,
+    whose learned frequencies the pages do not give.)"""
+    t = np.asarray(positions, dtype=np.int64)
+    _, H, W = grid
+    axes = [t // (H * W), (t // W) % H, t % W]
+    half = head_dim // 2
+    sizes = [half - 2 * (half // 3), half // 3, half // 3]
+    cols = []
+    for a, n in zip(axes, sizes):
+        freq = base ** (-np.arange(n) / max(n, 1))
+        cols.append(a[:, None].astype(np.float64) * freq[None, :])
+    return np.concatenate(cols, axis=1).astype(np.float32)
 
 
 def make_inputs(w: Workload, device: str = "cpu", with_grad_out: Optional[bool] = None) -> dict:
@@ -152,6 +178,13 @@ def make_inputs(w: Workload, device: str = "cpu", with_grad_out: Optional[bool] 
                v=v.to(torch.bfloat16).to(device))
     if dout is not None:
         out["dout"] = dout.to(torch.bfloat16).to(device)
+    if w.rope:
+        # query token i of query chunk c is kv token kv_offsets[n_kv - n_q + c] + (i - q_offsets[c])
+        qo, ko = w.q_offsets, w.kv_offsets
+        shift = len(ko) - len(qo)
+        qpos = np.concatenate([ko[shift + c] + np.arange(qo[c + 1] - qo[c]) for c in range(len(qo) - 1)])
+        out["rope_q"] = torch.from_numpy(rope_angles(qpos, D)).to(device)
+        out["rope_k"] = torch.from_numpy(rope_angles(np.arange(Skv), D)).to(device)
     return out
 
 

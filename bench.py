@@ -238,10 +238,11 @@ def run_ours(args, w, world, rank, local):
         if w.rope:
             bca.magi_bca_bwd_rope(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, rq, rk, dq=dq_,
                                   dk=dk_, dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream,
-                                  kv_range=w.kv_range)
+                                  kv_range=w.kv_range, deterministic=w.deterministic)
         else:
             bca.magi_bca_bwd(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, dq=dq_, dk=dk_,
-                             dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range)
+                             dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range,
+                             deterministic=w.deterministic)
 
     def step(ev=None, kev=None):
         # ev: events around the forward and backward calls; kev: a pair the
@@ -391,7 +392,9 @@ def run_ours(args, w, world, rank, local):
     bwd_avg = float(np.mean(bwd_ms)) if do_bwd else 0.0
     dom_ms = float(np.mean(kernel_ms))
     if do_bwd:
-        dom, dom_flops = "bca_bwd_main_kernel", bwd_flops(w)
+        # deterministic backward: the events bracket the dq pass and the main kernel
+        dom = "bca_bwd_dq_kernel+bca_bwd_main_kernel" if w.deterministic else "bca_bwd_main_kernel"
+        dom_flops = bwd_flops(w)
     else:
         dom, dom_flops = "bca_fwd_kernel", fwd_flops(w)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
@@ -414,7 +417,7 @@ def run_ours(args, w, world, rank, local):
                 "traffic": ncu_traffic(dom, w.name),
                 "avg_launch_ms": round(dom_ms, 4),
                 "algorithmic_bytes_per_launch": fwd_bytes(w) if dom == "bca_fwd_kernel" else None}
-    launches_per_step = bca_fwd_launches() + (bca_bwd_launches() if do_bwd else 0)
+    launches_per_step = bca_fwd_launches() + (bca_bwd_launches(w) if do_bwd else 0)
     res = {
         "metric": "block-causal attention useful TFLOP/s on 1 B200 and % of dense BF16 peak",
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -425,6 +428,7 @@ def run_ours(args, w, world, rank, local):
                    "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
                    "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
                    "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range, "rope": w.rope,
+                   "deterministic": w.deterministic,
                    "parallelism": f"replicas x{world}",
                    "l2": "flushed (512 MB write) between timed steps, outside the step events",
                    "head_start": "~1 ms GPU spin queued before each step's first event",
@@ -447,8 +451,10 @@ def bca_fwd_launches():
     return 2   # key pre-pass, forward kernel
 
 
-def bca_bwd_launches():
-    return 3   # prep (query and key rows), main, finalize (plus a memset of the padded lse rows when Sq % 128 != 0)
+def bca_bwd_launches(w):
+    # prep (query and key rows), main, finalize (plus a memset of the padded lse rows
+    # when Sq % 128 != 0); deterministic: also the dq pass and the dgamma reduction
+    return 5 if w.deterministic else 3
 
 
 # ------------------------------------------------------------------ oracle (CPU)

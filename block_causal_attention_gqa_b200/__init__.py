@@ -46,7 +46,8 @@ class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("seqlen_q", ctypes.c_int32), ("seqlen_kv", ctypes.c_int32),
                 ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("n_q_chunks", ctypes.c_int32), ("n_kv_chunks", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("kv_range", ctypes.c_int32)]
+                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("kv_range", ctypes.c_int32),
+                ("deterministic", ctypes.c_int32)]
 
 
 _lib = None
@@ -135,9 +136,9 @@ def _i32p(a: np.ndarray):
 
 
 def make_dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-              softmax_scale=0.0, rms_eps=1e-6, kv_range=0) -> Dims:
+              softmax_scale=0.0, rms_eps=1e-6, kv_range=0, deterministic=False) -> Dims:
     return Dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-                float(softmax_scale), float(rms_eps), int(kv_range))
+                float(softmax_scale), float(rms_eps), int(kv_range), int(bool(deterministic)))
 
 
 def _check_bf16(name, t, shape=None):
@@ -231,7 +232,8 @@ def magi_bca_bwd_workspace_size(dims: Dims) -> int:
 
 
 def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv, dgamma_q,
-         dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range, rope=None):
+         dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range, rope=None,
+         deterministic=False):
     """Shared marshalling of magi_bca_bwd and (rope = (rope_q, rope_k, drope_q,
     drope_k)) magi_bca_bwd_rope."""
     import torch
@@ -246,7 +248,8 @@ def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, ga
     _check_f32("gamma_q", gamma_q, (D,))
     _check_f32("gamma_k", gamma_k, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
+                     deterministic)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -280,17 +283,20 @@ def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, ga
 def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                  dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
                  workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
-                 kv_range: int = 0):
+                 kv_range: int = 0, deterministic: bool = False):
     """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
-    respect to the raw (pre-norm) q and k."""
+    respect to the raw (pre-norm) q and k.  deterministic=True sums every
+    gradient in a fixed order (same bits on every call; more tensor work)."""
     return _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
-                dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range)
+                dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range,
+                deterministic=deterministic)
 
 
 def magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                       rope_q, rope_k, dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None,
                       want_dgamma: bool = True, want_drope: bool = True, workspace=None,
-                      softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, kv_range: int = 0):
+                      softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, kv_range: int = 0,
+                      deterministic: bool = False):
     """Backward of magi_bca_fwd_rope.  Returns (dq, dk, dv, dgamma_q, dgamma_k,
     drope_q, drope_k); dq/dk are with respect to the raw (pre-rotation,
     pre-norm) q and k; drope_* (fp32 [seqlen, D/2], summed over batch and
@@ -308,13 +314,13 @@ def magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets
             drk = torch.empty_like(rope_k)
     res = _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
                dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range,
-               rope=(rope_q, rope_k, drq, drk))
+               rope=(rope_q, rope_k, drq, drk), deterministic=deterministic)
     return res + (drq, drk)
 
 
 def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                          dq, dk, dv, dgamma_q=None, dgamma_k=None, softmax_scale: float = 0.0,
-                         rms_eps: float = 1e-6, stream=None, kv_range: int = 0):
+                         rms_eps: float = 1e-6, stream=None, kv_range: int = 0, deterministic: bool = False):
     """Backward through the allocation-free entry point.
 
     For callers that cannot allocate device memory or hand the library a
@@ -336,7 +342,8 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
         if t is not None:
             _check_f32(nm, t, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
+                     deterministic)
     import torch
     with torch.cuda.device(q.device):
         st = library().magi_bca_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -367,11 +374,12 @@ def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, hea
 
 
 def magi_bca_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
-                          num_sms=148, kv_range=0) -> np.ndarray:
-    """Host-only: the backward's work units as an int32 array [n_units, 8]."""
+                          num_sms=148, kv_range=0, deterministic=False) -> np.ndarray:
+    """Host-only: the backward's work units as an int32 array [n_units, 8]
+    (deterministic=True: one unit per kv tile)."""
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1,
-                     kv_range=kv_range)
+                     kv_range=kv_range, deterministic=deterministic)
     lib = library()
     n = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, None, 0)
     if n < 0:

@@ -115,8 +115,9 @@ int device_state(int* device_out, DeviceState** st_out) {
 }
 
 std::vector<int32_t> schedule_key(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko) {
-  std::vector<int32_t> key = {dev, kind, d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim,
-                              d.n_q_chunks, d.n_kv_chunks, d.kv_range};
+  std::vector<int32_t> key = {dev,        kind,         d.batch,       d.seqlen_q,  d.seqlen_kv,
+                              d.heads_q,  d.heads_kv,   d.head_dim,    d.n_q_chunks, d.n_kv_chunks,
+                              d.kv_range, kind == 0 ? 0 : d.deterministic};
   key.insert(key.end(), qo, qo + d.n_q_chunks + 1);
   key.insert(key.end(), ko, ko + d.n_kv_chunks + 1);
   return key;
@@ -375,9 +376,13 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   DeviceState* ds;
   st = device_state(&dev, &ds);
   if (st != MAGI_BCA_OK) return st;
-  ScheduleEntry sched;
+  ScheduleEntry sched, dq_sched;
   st = get_schedule(dev, 1, d, q_chunk_offsets, kv_chunk_offsets, &sched);
   if (st != MAGI_BCA_OK) return st;
+  if (d.deterministic) {   // the dq pass runs the forward's query-major units
+    st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, &dq_sched);
+    if (st != MAGI_BCA_OK) return st;
+  }
   uint8_t* w = static_cast<uint8_t*>(workspace);
   BwdParams p;
   p.q = q;
@@ -397,6 +402,9 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   p.rope_k = rope_k;
   p.drope_q = rope_q != nullptr ? drope_q : nullptr;
   p.drope_k = rope_k != nullptr ? drope_k : nullptr;
+  p.deterministic = d.deterministic;
+  p.dq_units = d.deterministic ? dq_sched.dev : nullptr;
+  p.dgamma_part = reinterpret_cast<float*>(w + ws.dgpart);
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -428,7 +436,8 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
       make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
   cudaError_t e =
-      launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, sched.n_units, static_cast<cudaStream_t>(stream));
+      launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, sched.n_units,
+                 d.deterministic ? dq_sched.n_units : 0, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("backward launch", e);
 }
 

@@ -10,7 +10,8 @@
 //   1. prep      one warp per row.  Query rows: Q^ into the workspace; Delta =
 //                rowsum(dO * O); -lse*log2(e) and -Delta, each split into three
 //                bf16 pieces, in a 16-byte row per query (128-padded layout);
-//                zero the row's fp32 dq accumulator.  Key rows: K^ into the
+//                zero the row's fp32 dq accumulator (not needed when
+//                deterministic: the dq pass stores every row).  Key rows: K^ into the
 //                workspace (knorm_row, as the forward's key pre-pass) and zero
 //                the row's fp32 dV / G_k accumulators.  Also zeroes dgamma.
 //   2. main      one CTA per (batch, kv head, 128-key tile, query-tile range).
@@ -34,6 +35,14 @@
 //                one kv tile).
 //   3. finalize  one warp per row: dq, dk through the RMSNorm Jacobian, dv, and
 //                dgamma_q, dgamma_k.
+// Deterministic backward (dims.deterministic): no sum depends on timing.  The
+// dq pass (bca_bwd_dq_kernel, query-major, one CTA per query tile) computes
+// G_q before the main kernel, which then skips its G_q product and drain;
+// every kv tile is one main-kernel unit, so dV and G_k are added once onto
+// zero; the finalize takes whole tokens (angle gradients summed in registers)
+// and writes per-block dgamma partials that one small kernel adds in block
+// order.  The dq pass recomputes S and dP, so the tensor work is 7/5 of the
+// default path's.
 // These are the five matrix products of the Flash-Attention backward (2.5x the
 // forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
 // query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.
@@ -76,7 +85,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 enum : int {
   kErrKv = 2001, kErrQFull = 2002, kErrQEmpty = 2003, kErrSFull = 2004, kErrDsReady = 2005,
-  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009, kErrLdEmpty = 2010
+  kErrDqFull = 2006, kErrDqDrained = 2007, kErrAcc = 2008, kErrSmem = 2009, kErrLdEmpty = 2010,
+  kErrDqQ = 2011, kErrDqK = 2012, kErrDqV = 2013, kErrDqKEmpty = 2014, kErrDqVEmpty = 2015,
+  kErrDqSFull = 2016, kErrDqDpFree = 2017, kErrDqDsReady = 2018, kErrDqGq = 2019
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool ok, int* status, int code) {
@@ -212,7 +223,7 @@ __global__ void __launch_bounds__(256) bca_bwd_prep_kernel(const BwdParams p) {
 #pragma unroll
     for (int e = 0; e < E; ++e) dot = fmaf(o[e], g[e], dot);
     dot = warp_sum(dot);
-    IO::store_zero_f32(p.dqacc + r * D, lane);
+    if (!p.deterministic) IO::store_zero_f32(p.dqacc + r * D, lane);   // (the dq pass stores every row)
     if (lane == 0) {
       const int h = (int)(r % p.heads_q);
       const int64_t bs = r / p.heads_q;
@@ -251,7 +262,7 @@ struct BwdBars {
   uint64_t q_full[2], q_empty[2];
 };
 
-template <int D>
+template <int D, bool kDq>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
@@ -293,7 +304,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     mbar_init(&bars->acc_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], kComputeWarpgroups);   // each warpgroup, once its dq staging is read
+      // with G_q: each warpgroup, once its dq staging is read; without: the MMA thread
+      mbar_init(&bars->q_empty[s], kDq ? kComputeWarpgroups : 1);
     }
     fence_mbar_init();
   }
@@ -428,12 +440,16 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (!(ok = mbar_wait(&bars->ds_ready, t & 1, p.status, kErrDsReady))) break;
         tc_fence_after();
         dkdv(4);
-        // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
+        if constexpr (kDq) {
+          // G_q = dS' K : A = dS'^T buffer read MN-major (M = queries, K = keys), B = K [keys][D] (MN-major)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
-                      make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
-        mma_commit(&bars->dq_full);   // G_q ready; this step's Q^ / dO stage and dS^T are no longer read
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ss(tmem + T_DP, make_sw128_desc(ds_a + kk * 2048, 16384, 1024),
+                        make_sw128_desc(kn_a + kk * 2048, 16384, 1024), id_mm, kk > 0);
+          mma_commit(&bars->dq_full);   // G_q ready; this step's Q^ / dO stage and dS^T are no longer read
+        } else {
+          mma_commit(&bars->q_empty[st]);   // the stage is free once dK~ and dV have read it
+        }
         if (t + 1 < n_steps) {
           const int st1 = (t + 1) & 1;
           // S^T(t+1) only needs P^T(t) read (dV was issued before); dP^T(t+1)
@@ -441,8 +457,11 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           if (!(ok = mbar_wait(&bars->q_full[st1], ((t + 1) >> 1) & 1, p.status, kErrQFull))) break;
           tc_fence_after();
           mma_kmajor(T_S, kn_a, qn_a + st1 * L::kTile, ext_lse);
-          if (!(ok = mbar_wait(&bars->dq_drained, t & 1, p.status, kErrDqDrained))) break;
-          tc_fence_after();
+          if constexpr (kDq) {
+            if (!(ok = mbar_wait(&bars->dq_drained, t & 1, p.status, kErrDqDrained))) break;
+            tc_fence_after();
+          }
+          // (without G_q, dP^T(t) was read before ds_ready)
           mma_kmajor(T_DP, v_a, do_a + st1 * L::kTile, ext_delta);
           mma_commit(&bars->s_full);
           mma_commit(&bars->ld_empty);
@@ -556,7 +575,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       named_bar_sync(bar_id, 128);
       if (j == 0 && ok) {
         mbar_arrive(&bars->ds_ready);
-        if (t > 0) {
+        if (kDq && t > 0) {
           // The previous step's dq reduction has had this step's MMAs and
           // softmax to read its staging; once it has, that Q^/dO stage goes back
           // to the producer (the next load still has this step's products to land).
@@ -565,6 +584,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         }
       }
 
+      if constexpr (!kDq) continue;
       // Drain G_q (TMEM lane = query row of this step) into the fp32 accumulator:
       // TMEM -> registers (then the dP^T/G_q columns are free again), registers ->
       // this step's Q^/dO stage (dq_full also means dK~ and dV have read it), then a TMA bulk
@@ -599,7 +619,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     // every bulk reduction has read its staging (and the last stage is
     // released) before the stage buffers are reused below
-    if (j == 0) {
+    if (kDq && j == 0) {
       tma_store_wait_read();
       if (ok && n_steps > 0) mbar_arrive(&bars->q_empty[(n_steps - 1) & 1]);
     }
@@ -647,12 +667,331 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 }
 
+// ------------------------------------------------------------------ dq pass
+// Deterministic backward only.  Query-major: one CTA per 128-row query
+// sub-tile of the forward schedule (block 2u + s runs sub-tile s of unit u),
+// so each query row's G_q is summed over its visible kv tiles in tile order
+// inside one CTA, with no reductions across CTAs.  Q^ and dO of the sub-tile
+// stay in shared memory; K^ streams through a 3-stage ring and V through a
+// 2-stage one (K^ is read twice per tile, by S and by G_q, so it stays
+// longer).  Per kv tile j, in TMEM:
+//   S    = Q^ K^_j^T                    -> S_buf[j % 2]  (log2 units)
+//   dP   = dO V_j^T                     -> DP
+//   dS'  = exp2(S - lse2) (dP - Delta)  -> bf16 pairs over the first half of
+//                                          each warpgroup's S_buf columns
+//   G_q += dS' K^_j                     -> GQ  (A from TMEM, K^ MN-major)
+// and at the end G_q goes to the fp32 dq buffer for the finalize kernel.
+// Roles: warpgroups 0 and 1 own key columns [0, 64) and [64, 128) of every
+// row (thread = query row = TMEM lane), warp 8 issues MMAs, warp 9 runs TMA.
+// Per tile j the MMA thread issues dP(j+1) as soon as both warpgroups have
+// read dP(j), G_q(j) once dS'(j) is written, then S(j+2): the tensor pipe
+// holds the next tile's products while the softmax runs.
+constexpr int kDqThreads = 320;
+constexpr int kDqKStages = 3, kDqVStages = 2;
+
+template <int D>
+struct DqLayout {
+  static constexpr int kTile = 128 * D * 2;  // [128][D] bf16
+  static constexpr int kQn = 0;
+  static constexpr int kDo = kQn + kTile;
+  static constexpr int kK = kDo + kTile;                // kDqKStages
+  static constexpr int kV = kK + kDqKStages * kTile;    // kDqVStages
+  static constexpr int kBars = kV + kDqVStages * kTile;
+  static constexpr int kTmemSlot = kBars + 16 * 8;
+  static constexpr int kTotal = kTmemSlot + 16;
+};
+
+struct DqBars {
+  uint64_t q_full, dp_free, ds_ready, gq_full;
+  uint64_t s_full[2];
+  uint64_t k_full[kDqKStages], k_empty[kDqKStages], v_full[kDqVStages], v_empty[kDqVStages];
+};
+static_assert(sizeof(DqBars) <= 16 * 8, "dq barriers exceed their slot");
+
+// chunk c with offs[c] <= row < offs[c + 1]
+__device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
+  int lo = 0, hi = n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(offs + mid) <= row) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDqThreads, 1)
+bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const BwdParams p, const int smem_alloc) {
+  using L = DqLayout<D>;
+  const int32_t* u = p.dq_units + (size_t)(blockIdx.x >> 1) * 12;
+  const int sub = blockIdx.x & 1;
+  const int h = __ldg(u + (sub ? 4 : 2));
+  if (h < 0) return;  // the unit has one sub-tile: this CTA has no work
+  extern __shared__ uint8_t smem_raw[];
+  const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
+  uint8_t* smem = reinterpret_cast<uint8_t*>(base);
+  if (base - reinterpret_cast<uintptr_t>(smem_raw) + L::kTotal > (uintptr_t)smem_alloc) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kErrSmem);
+    return;
+  }
+  DqBars* bars = reinterpret_cast<DqBars*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = __ldg(u + 0), hk = __ldg(u + 1);
+  const int m0 = __ldg(u + (sub ? 5 : 3));
+  const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
+  const int t_begin = __ldg(u + 8), t_full_begin = __ldg(u + 9);
+  const int n_vis = n_tiles - t_begin;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->dp_free, 2);   // one arrival per warpgroup
+    mbar_init(&bars->ds_ready, 2);
+    mbar_init(&bars->gq_full, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&bars->s_full[i], 1);
+    for (int i = 0; i < kDqKStages; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < kDqVStages; ++i) {
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tm_qn);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t T_S = 0, T_DP = 256, T_GQ = 384;  // S_buf[i] at columns [128 i, 128 i + 128)
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      mbar_arrive_expect_tx(&bars->q_full, 2 * L::kTile);
+      for (int box = 0; box < D / 64; ++box) {
+        tma_load_4d(smem + L::kQn + box * 16384, &tm_qn, &bars->q_full, box * 64, h, m0, b);
+        tma_load_4d(smem + L::kDo + box * 16384, &tm_do, &bars->q_full, box * 64, h, m0, b);
+      }
+      for (int j = 0; j < n_vis; ++j) {
+        const int n0 = (t_begin + j) * 128;
+        const int ks = j % kDqKStages, vs = j % kDqVStages;
+        if (!mbar_wait(&bars->k_empty[ks], ((j / kDqKStages) & 1) ^ 1, p.status, kErrDqKEmpty)) break;
+        mbar_arrive_expect_tx(&bars->k_full[ks], L::kTile);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_4d(smem + L::kK + ks * L::kTile + box * 16384, &tm_k, &bars->k_full[ks], box * 64, hk, n0, b);
+        if (!mbar_wait(&bars->v_empty[vs], ((j / kDqVStages) & 1) ^ 1, p.status, kErrDqVEmpty)) break;
+        mbar_arrive_expect_tx(&bars->v_full[vs], L::kTile);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_4d(smem + L::kV + vs * L::kTile + box * 16384, &tm_v, &bars->v_full[vs], box * 64, hk, n0, b);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t id_s = make_idesc_bf16(128, 128, false, false);  // S, dP: both operands K-major
+      constexpr uint32_t id_g = make_idesc_bf16(128, D, false, true);     // G_q: A from TMEM, B MN-major
+      const uint32_t qn_a = smem_u32(smem + L::kQn), do_a = smem_u32(smem + L::kDo);
+      const uint32_t k_a = smem_u32(smem + L::kK), v_a = smem_u32(smem + L::kV);
+      // C[128 x 128] = A[128 x D] B[128 x D]^T, both K-major in 64-feature boxes
+      auto mma_kk = [&](uint32_t d, uint32_t a, uint32_t bb) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(tmem + d, make_sw128_desc(a + off, 16, 1024), make_sw128_desc(bb + off, 16, 1024), id_s,
+                      kk > 0);
+        }
+      };
+      auto issue_s = [&](int j) { mma_kk(T_S + 128 * (j & 1), qn_a, k_a + (j % kDqKStages) * L::kTile); };
+      auto issue_dp = [&](int j) {
+        mma_kk(T_DP, do_a, v_a + (j % kDqVStages) * L::kTile);
+        mma_commit(&bars->v_empty[j % kDqVStages]);   // V_j is read only by dP(j)
+      };
+      bool ok = n_vis > 0 && mbar_wait(&bars->q_full, 0, p.status, kErrDqQ);
+      ok = ok && mbar_wait(&bars->k_full[0], 0, p.status, kErrDqK);
+      ok = ok && mbar_wait(&bars->v_full[0], 0, p.status, kErrDqV);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+        mma_commit(&bars->s_full[0]);
+      }
+      if (ok && n_vis > 1) {
+        ok = mbar_wait(&bars->k_full[1 % kDqKStages], 0, p.status, kErrDqK);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
+        }
+      }
+      for (int j = 0; j < n_vis && ok; ++j) {
+        if (j + 1 < n_vis) {
+          // dP(j+1) overwrites DP once both warpgroups hold dP(j) in registers
+          if (!(ok = mbar_wait(&bars->dp_free, j & 1, p.status, kErrDqDpFree))) break;
+          const int j1 = j + 1;
+          if (!(ok = mbar_wait(&bars->v_full[j1 % kDqVStages], (j1 / kDqVStages) & 1, p.status, kErrDqV))) break;
+          tc_fence_after();
+          issue_dp(j1);
+          mma_commit(&bars->s_full[j1 & 1]);   // S(j+1) was issued earlier
+        }
+        if (!(ok = mbar_wait(&bars->ds_ready, j & 1, p.status, kErrDqDsReady))) break;
+        tc_fence_after();
+        // G_q += dS'(j) K^_j: K-step kk covers keys [16 kk, 16 kk + 16); warpgroup
+        // w wrote the packed pairs of keys [64 w, 64 w + 64) at S_buf + 64 w
+        const uint32_t ks = k_a + (j % kDqKStages) * L::kTile;
+        const uint32_t sb = T_S + 128 * (j & 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + T_GQ, tmem + sb + (kk >> 2) * 64 + (kk & 3) * 8,
+                      make_sw128_desc(ks + kk * 2048, 16384, 1024), id_g, j > 0 || kk > 0);
+        mma_commit(&bars->k_empty[j % kDqKStages]);
+        if (j + 2 < n_vis) {
+          // S(j+2) overwrites S_buf[j % 2] after G_q(j) (issued before it) has read dS'(j)
+          const int j2 = j + 2;
+          if (!(ok = mbar_wait(&bars->k_full[j2 % kDqKStages], (j2 / kDqKStages) & 1, p.status, kErrDqK))) break;
+          tc_fence_after();
+          issue_s(j2);
+        }
+      }
+      mma_commit(&bars->gq_full);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int wg = warp >> 2;             // key columns [64 wg, 64 wg + 64)
+    const int r = threadIdx.x & 127;      // query row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int bar_id = 1 + wg;
+    const int row = m0 + r;
+    // -lse log2(e) and -Delta of the row, rebuilt from the prep kernel's three
+    // bf16 pieces each (padding rows past seqlen_q hold zeros)
+    float nl, nd;
+    {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(
+          p.ld + (((size_t)b * p.heads_q + h) * p.seqlen_q_pad + row) * 4));
+      nl = (bf16_lo(v.x) + bf16_hi(v.x)) + bf16_lo(v.y);
+      nd = (bf16_hi(v.y) + bf16_lo(v.z)) + bf16_hi(v.z);
+    }
+    // visible keys [kv_first, limit) of the row
+    int limit = p.seqlen_kv, kv_first = 0;
+    if (row < p.seqlen_q) {
+      const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
+      limit = __ldg(p.kv_offsets + p.n_kv_chunks - p.n_q_chunks + c + 1);
+      if (p.kv_range > 0)
+        kv_first = __ldg(p.kv_offsets + max(p.n_kv_chunks - p.n_q_chunks + c - p.kv_range + 1, 0));
+    }
+    const uint64_t nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
+    bool ok = true;
+    // Every thread runs all n_vis iterations and reaches every named barrier
+    // even after a failed wait; only the work is skipped.
+    for (int j = 0; j < n_vis; ++j) {
+      ok = warp_wait(&bars->s_full[j & 1], (j >> 1) & 1, ok, p.status, kErrDqSFull);
+      const uint32_t t_s = tmem + lane_base + T_S + 128 * (j & 1) + 64 * wg;
+      uint32_t sa[32], sb[32], da[32], db[32];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(t_s, sa);
+        tmem_ld32(t_s + 32, sb);
+        tmem_ld32(tmem + lane_base + T_DP + 64 * wg, da);
+        tmem_ld32(tmem + lane_base + T_DP + 64 * wg + 32, db);
+        tmem_wait_ld();
+        tc_fence_before();
+      }
+      named_bar_sync(bar_id, 128);
+      if (r == 0 && ok) mbar_arrive(&bars->dp_free);
+      if (ok) {
+        const int tile = t_begin + j;
+        const bool masked = tile < t_full_begin || tile >= n_full;
+        uint32_t pk[32];
+        auto sval = [&](int c) { return __uint_as_float(c < 32 ? sa[c] : sb[c - 32]); };
+        auto dval = [&](int c) { return __uint_as_float(c < 32 ? da[c] : db[c - 32]); };
+        if (masked) {
+          const int c0 = tile * 128 + 64 * wg;
+          const int lim = limit - c0, lo = kv_first - c0;   // columns [lo, lim) are visible
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = c >= lo && c < lim ? fast_exp2(sval(c) + nl) : 0.f;
+            const float p1 = c + 1 >= lo && c + 1 < lim ? fast_exp2(sval(c + 1) + nl) : 0.f;
+            pk[c >> 1] = pack_bf16x2(p0 * (dval(c) + nd), p1 * (dval(c + 1) + nd));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const uint64_t a2 = f2_add(f2_pack(sval(c), sval(c + 1)), nl2);
+            float p0, p1;
+            if (((c >> 1) & 3) == 3) {   // one pair in four on the FMA pipe
+              exp2_poly_pair(a2, p0, p1);
+            } else {
+              float a0, a1;
+              f2_unpack(a2, a0, a1);
+              p0 = fast_exp2(a0);
+              p1 = fast_exp2(a1);
+            }
+            const uint64_t d2 = f2_mul(f2_add(f2_pack(dval(c), dval(c + 1)), nd2), f2_pack(p0, p1));
+            float d0, d1;
+            f2_unpack(d2, d0, d1);
+            pk[c >> 1] = pack_bf16x2(d0, d1);
+          }
+        }
+        tmem_st32(t_s, pk);   // dS' pairs over columns [64 wg, 64 wg + 32) of S_buf
+        tmem_wait_st();
+        tc_fence_before();
+      }
+      named_bar_sync(bar_id, 128);
+      if (r == 0 && ok) mbar_arrive(&bars->ds_ready);
+    }
+
+    // Epilogue: G_q (fp32) of the row, warpgroup w storing columns [w D/2, w D/2 + D/2).
+    ok = warp_wait(&bars->gq_full, 0, ok, p.status, kErrDqGq);
+    if (ok) {
+      tc_fence_after();
+      constexpr int kCols = D / 2;
+      float* dst = p.dqacc + (((size_t)b * p.seqlen_q + row) * p.heads_q + h) * D + wg * kCols;
+#pragma unroll 1
+      for (int c = 0; c < kCols / 32; ++c) {
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_base + T_GQ + wg * kCols + c * 32, g);
+        tmem_wait_ld();
+        if (n_vis == 0) {   // (chunks are never empty, so every row sees some key)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) g[i] = 0u;
+        }
+        if (row < p.seqlen_q) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d4[i] = make_uint4(g[4 * i], g[4 * i + 1], g[4 * i + 2], g[4 * i + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------------------ finalize
 // One warp per row.  Query rows: dq~ = scale gamma_k G_q, dq through the
 // RMSNorm Jacobian, dgamma_q += dq~ q^.  Key rows: dv = bf16(dV), gamma_k dk~ =
 // G_k / log2(e), dk through the Jacobian, dgamma_k += dk~ k^.  With r = rsqrt
 // (mean x^2 + eps), x^ = x r and g = gamma dx~:  dx = r (g - x^ mean(g x^)).
-template <int D, bool kRope>
+// kDet (deterministic backward): each warp takes whole tokens, i.e. all rows
+// (batch, head) of one query or key token in a fixed order, so a token's angle
+// gradient is summed in registers and written once; the block's dgamma sums
+// go to per-block slots that bca_bwd_dgamma_reduce_kernel adds in block order.
+template <int D, bool kRope, bool kDet>
 __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p) {
   using IO = RowIO<D>;
   constexpr int E = IO::E;
@@ -671,7 +1010,7 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
   }
   // Two rows per warp and iteration, all loads issued before the arithmetic,
   // so each warp keeps two rows' reads in flight.
-  auto finish_row = [&](int64_t rr, float (&x)[E], float (&g)[E], const float (&dvv)[E]) {
+  auto finish_row = [&](int64_t rr, float (&x)[E], float (&g)[E], const float (&dvv)[E], float (&dr)[E]) {
     const bool is_q = rr < n_q;
     const int64_t r = is_q ? rr : rr - n_q;
     // with rotary angles the normalised vector is rope(x): the Jacobian below
@@ -717,7 +1056,10 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
       for (int e = 0; e < E; ++e) {
         const float op = __shfl_xor_sync(0xffffffffu, o[e], 16);
         const float yp = __shfl_xor_sync(0xffffffffu, y[e], 16);
-        if (drope != nullptr && lane < 16) atomicAdd(drope + tok * (D / 2) + lane * E + e, op * y[e] - o[e] * yp);
+        if constexpr (kDet)
+          dr[e] += op * y[e] - o[e] * yp;
+        else if (drope != nullptr && lane < 16)
+          atomicAdd(drope + tok * (D / 2) + lane * E + e, op * y[e] - o[e] * yp);
         o[e] = lane < 16 ? fmaf(op, sn[e], o[e] * cs[e]) : fmaf(-op, sn[e], o[e] * cs[e]);
       }
     }
@@ -739,14 +1081,48 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
     IO::load_f32((is_q ? p.dqacc : p.dkacc) + r * D, lane, g);
     if (!is_q) IO::load_f32(p.dvacc + r * D, lane, dvv);
   };
-  const int64_t total = n_q + n_k;
-  for (int64_t rr = (int64_t)blockIdx.x * 8 + wid; rr < total; rr += 2 * warps) {
-    const int64_t rr2 = rr + warps;
-    float x0[E], g0[E], v0[E], x1[E], g1[E], v1[E];
-    load_row(rr, x0, g0, v0);
-    if (rr2 < total) load_row(rr2, x1, g1, v1);
-    finish_row(rr, x0, g0, v0);
-    if (rr2 < total) finish_row(rr2, x1, g1, v1);
+  if constexpr (!kDet) {
+    const int64_t total = n_q + n_k;
+    float dr[E];   // (unused: angle gradients go out by atomics)
+    for (int64_t rr = (int64_t)blockIdx.x * 8 + wid; rr < total; rr += 2 * warps) {
+      const int64_t rr2 = rr + warps;
+      float x0[E], g0[E], v0[E], x1[E], g1[E], v1[E];
+      load_row(rr, x0, g0, v0);
+      if (rr2 < total) load_row(rr2, x1, g1, v1);
+      finish_row(rr, x0, g0, v0, dr);
+      if (rr2 < total) finish_row(rr2, x1, g1, v1, dr);
+    }
+  } else {
+    // tokens [0, Sq) are query tokens, [Sq, Sq + Skv) key tokens
+    const int64_t tokens = (int64_t)p.seqlen_q + p.seqlen_kv;
+    for (int64_t tt = (int64_t)blockIdx.x * 8 + wid; tt < tokens; tt += warps) {
+      const bool is_q = tt < p.seqlen_q;
+      const int64_t s_tok = is_q ? tt : tt - p.seqlen_q;
+      const int H = is_q ? p.heads_q : p.heads_kv;
+      const int64_t S = is_q ? p.seqlen_q : p.seqlen_kv;
+      const int n = p.batch * H;
+      auto row_of = [&](int i) {   // i-th (batch, head) row of the token, in the finalize's row numbering
+        const int64_t r = ((int64_t)(i / H) * S + s_tok) * H + i % H;
+        return is_q ? r : n_q + r;
+      };
+      float dr[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) dr[e] = 0.f;
+      for (int i = 0; i < n; i += 2) {
+        float x0[E], g0[E], v0[E], x1[E], g1[E], v1[E];
+        load_row(row_of(i), x0, g0, v0);
+        if (i + 1 < n) load_row(row_of(i + 1), x1, g1, v1);
+        finish_row(row_of(i), x0, g0, v0, dr);
+        if (i + 1 < n) finish_row(row_of(i + 1), x1, g1, v1, dr);
+      }
+      if constexpr (kRope) {
+        float* drope = is_q ? p.drope_q : p.drope_k;
+        if (drope != nullptr && lane < 16) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) drope[s_tok * (D / 2) + lane * E + e] = dr[e];
+        }
+      }
+    }
   }
   if (p.dgamma_q != nullptr || p.dgamma_k != nullptr) {
 #pragma unroll
@@ -762,18 +1138,50 @@ __global__ void __launch_bounds__(256) bca_bwd_finalize_kernel(const BwdParams p
         aq += red[0][w][threadIdx.x];
         ak += red[1][w][threadIdx.x];
       }
-      if (p.dgamma_q != nullptr) atomicAdd(p.dgamma_q + threadIdx.x, aq);
-      if (p.dgamma_k != nullptr) atomicAdd(p.dgamma_k + threadIdx.x, ak);
+      if constexpr (kDet) {
+        p.dgamma_part[(size_t)blockIdx.x * 2 * D + threadIdx.x] = aq;
+        p.dgamma_part[(size_t)blockIdx.x * 2 * D + D + threadIdx.x] = ak;
+      } else {
+        if (p.dgamma_q != nullptr) atomicAdd(p.dgamma_q + threadIdx.x, aq);
+        if (p.dgamma_k != nullptr) atomicAdd(p.dgamma_k + threadIdx.x, ak);
+      }
     }
   }
+}
+
+// dgamma of the deterministic backward: thread d adds slot d of every
+// finalize block's partials in block order.
+template <int D>
+__global__ void __launch_bounds__(2 * D) bca_bwd_dgamma_reduce_kernel(const BwdParams p, int blocks) {
+  const int d = threadIdx.x % D;
+  const bool is_k = threadIdx.x >= D;
+  float acc = 0.f;
+  for (int i = 0; i < blocks; ++i) acc += p.dgamma_part[(size_t)i * 2 * D + threadIdx.x];
+  float* dst = is_k ? p.dgamma_k : p.dgamma_q;
+  if (dst != nullptr) dst[d] = acc;
+}
+
+// Largest finalize grid of the deterministic backward (its dgamma slots).
+constexpr int kMaxFinBlocks = 2048;
+
+// cudaFuncSetAttribute once per (kernel, device); bit `dev` of `mask`.
+template <typename K>
+cudaError_t set_smem_once(uint64_t& mask, int dev, K kernel, int bytes) {
+  if (dev < 64 && ((mask >> dev) & 1u)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) mask |= uint64_t(1) << dev;
+  return e;
 }
 
 template <int D>
 cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
                          const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
-                         const CUtensorMap& t_dk, const BwdParams& p, int n_units, cudaStream_t stream) {
+                         const CUtensorMap& t_dk, const BwdParams& p, int n_units, int n_dq_units,
+                         cudaStream_t stream) {
   using L = BwdLayout<D>;
-  static uint64_t configured = 0;
+  using LD = DqLayout<D>;
+  static uint64_t configured[2] = {0, 0}, configured_dq = 0;
+  const bool det = p.deterministic != 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -782,30 +1190,35 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   if (e != cudaSuccess) return e;
   const int alloc = L::kTotal + 1024 <= max_optin ? L::kTotal + 1024 : max_optin;
   if (alloc < L::kTotal) return cudaErrorInvalidConfiguration;
-  if (dev >= 64 || !((configured >> dev) & 1u)) {
-    e = cudaFuncSetAttribute(bca_bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
+  e = det ? set_smem_once(configured[0], dev, bca_bwd_main_kernel<D, false>, alloc)
+          : set_smem_once(configured[1], dev, bca_bwd_main_kernel<D, true>, alloc);
+  if (e != cudaSuccess) return e;
+  const int alloc_dq = LD::kTotal + 1024 <= max_optin ? LD::kTotal + 1024 : max_optin;
+  if (det) {
+    if (alloc_dq < LD::kTotal) return cudaErrorInvalidConfiguration;
+    e = set_smem_once(configured_dq, dev, bca_bwd_dq_kernel<D>, alloc_dq);
     if (e != cudaSuccess) return e;
-    if (dev < 64) configured |= uint64_t(1) << dev;
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
-  // one wave of the row kernels (grid-stride loops over one warp per row)
-  static int prep_per_sm[2] = {0, 0}, fin_per_sm[2][2] = {{0, 0}, {0, 0}};
+  // one wave of the row kernels (grid-stride loops over one warp per row or token)
+  static int prep_per_sm[2] = {0, 0}, fin_per_sm[2][2][2] = {};
   const bool rope = p.rope_q != nullptr || p.rope_k != nullptr;
   int& prep_occ = prep_per_sm[D == 128];
-  int& fin_occ = fin_per_sm[D == 128][rope];
+  int& fin_occ = fin_per_sm[D == 128][rope][det];
   if (prep_occ == 0) {
     int n = 0;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_prep_kernel<D>, 256, 0);
     prep_occ = std::max(n, 1);
   }
+  auto finalize_kernel = [&]() {
+    if (det) return rope ? bca_bwd_finalize_kernel<D, true, true> : bca_bwd_finalize_kernel<D, false, true>;
+    return rope ? bca_bwd_finalize_kernel<D, true, false> : bca_bwd_finalize_kernel<D, false, false>;
+  };
   if (fin_occ == 0) {
     int n = 0;
-    if (rope)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D, true>, 256, 0);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, bca_bwd_finalize_kernel<D, false>, 256, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, finalize_kernel(), 256, 0);
     fin_occ = std::max(n, 1);
   }
   const int prep_blocks = (int)std::min<int64_t>((rows + 7) / 8, (int64_t)sms * prep_occ);
@@ -818,19 +1231,35 @@ cudaError_t launch_bwd_d(const CUtensorMap& t_k, const CUtensorMap& t_v, const C
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   profile_mark(0, stream);
+  if (det && n_dq_units > 0) {
+    // G_q of every query row, summed in tile order inside one CTA
+    bca_bwd_dq_kernel<D><<<2 * n_dq_units, kDqThreads, alloc_dq, stream>>>(t_qn, t_do, t_k, t_v, p, alloc_dq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (n_units > 0) {
-    bca_bwd_main_kernel<D><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, alloc);
+    if (det)
+      bca_bwd_main_kernel<D, false><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p,
+                                                                          alloc);
+    else
+      bca_bwd_main_kernel<D, true><<<n_units, kThreads, alloc, stream>>>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p,
+                                                                         alloc);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   profile_mark(1, stream);
-  const int64_t frows = (int64_t)p.batch * p.seqlen_q * p.heads_q + (int64_t)p.batch * p.seqlen_kv * p.heads_kv;
-  const int fin_blocks = (int)std::min<int64_t>((frows + 7) / 8, (int64_t)sms * fin_occ);
-  if (rope)
-    bca_bwd_finalize_kernel<D, true><<<fin_blocks, 256, 0, stream>>>(p);
-  else
-    bca_bwd_finalize_kernel<D, false><<<fin_blocks, 256, 0, stream>>>(p);
-  return cudaGetLastError();
+  // a deterministic finalize takes whole tokens; its grid also fixes the dgamma slots
+  const int64_t work = det ? (int64_t)p.seqlen_q + p.seqlen_kv : rows;
+  int fin_blocks = (int)std::min<int64_t>((work + 7) / 8, (int64_t)sms * fin_occ);
+  if (det) fin_blocks = std::min(fin_blocks, kMaxFinBlocks);
+  finalize_kernel()<<<fin_blocks, 256, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (det && (p.dgamma_q != nullptr || p.dgamma_k != nullptr)) {
+    bca_bwd_dgamma_reduce_kernel<D><<<1, 2 * D, 0, stream>>>(p, fin_blocks);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 }  // namespace
@@ -845,15 +1274,18 @@ BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D
   w.dqacc = w.ld + up((size_t)B * Hq * sq_pad * 16);
   w.dvacc = w.dqacc + up((size_t)B * Sq * Hq * D * 4);
   w.dkacc = w.dvacc + up((size_t)B * Skv * Hkv * D * 4);
-  w.total = w.dkacc + up((size_t)B * Skv * Hkv * D * 4);
+  w.dgpart = w.dkacc + up((size_t)B * Skv * Hkv * D * 4);
+  w.total = w.dgpart + up((size_t)kMaxFinBlocks * 2 * D * 4);
   return w;
 }
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
                        const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
-                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream) {
-  if (head_dim == 128) return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, stream);
-  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, stream);
+                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, int n_dq_units,
+                       cudaStream_t stream) {
+  if (head_dim == 128)
+    return launch_bwd_d<128>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, n_dq_units, stream);
+  return launch_bwd_d<64>(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, n_units, n_dq_units, stream);
 }
 
 }  // namespace magi

@@ -58,6 +58,10 @@ struct BwdParams {
   float* dqacc;               // fp32 G_q accumulator          [B, Sq, Hq, D]
   float* dvacc;               // fp32 dV accumulator           [B, Skv, Hkv, D]
   float* dkacc;               // fp32 G_k accumulator          [B, Skv, Hkv, D]
+  // deterministic backward
+  int deterministic;          // 0 or 1
+  const int32_t* dq_units;    // query-major units of the dq pass (forward schedule, 12 int32 each)
+  float* dgamma_part;         // per finalize block: dgamma_q [D] then dgamma_k [D], summed in block order
   int batch, seqlen_q, seqlen_kv, heads_q, heads_kv, seqlen_q_pad;
   float scale;                // softmax scale
   float scale_log2;           // softmax scale * log2(e)
@@ -66,13 +70,14 @@ struct BwdParams {
 };
 
 struct BwdWorkspace {
-  size_t qn, kn, ld, dqacc, dvacc, dkacc, total;  // byte offsets and total size
+  size_t qn, kn, ld, dqacc, dvacc, dkacc, dgpart, total;  // byte offsets and total size
 };
 BwdWorkspace bwd_workspace_layout(int B, int Sq, int Skv, int Hq, int Hkv, int D);
 
 cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
                        const CUtensorMap& t_do, const CUtensorMap& t_dq, const CUtensorMap& t_dv,
-                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, cudaStream_t stream);
+                       const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, int n_dq_units,
+                       cudaStream_t stream);
 int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
 
 // K^ = bf16(rope(k) rsqrt(mean k^2 + eps)) for `rows` rows [B, seqlen, heads] of head_dim

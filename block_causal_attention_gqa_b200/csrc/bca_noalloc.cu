@@ -84,7 +84,8 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, d);
   if (st != MAGI_BCA_OK) return st;
 
-  // Layout inside the array: [workspace][schedule units][q offsets][kv offsets].
+  // Layout inside the array: [workspace][schedule units][q offsets][kv offsets]
+  // and, for the deterministic backward, [dq-pass units].
   const BwdWorkspace ws = bwd_workspace_layout(d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim);
   int sms = 148;
   {
@@ -95,6 +96,13 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   const int n_units = static_cast<int>(blob.size() / kUnitInts);
   blob.insert(blob.end(), q_chunk_offsets, q_chunk_offsets + d.n_q_chunks + 1);
   blob.insert(blob.end(), kv_chunk_offsets, kv_chunk_offsets + d.n_kv_chunks + 1);
+  const size_t dq_units_off = blob.size();
+  int n_dq_units = 0;
+  if (d.deterministic) {
+    const std::vector<int32_t> fwd = build_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, d);
+    n_dq_units = static_cast<int>(fwd.size() / kFwdUnitInts);
+    blob.insert(blob.end(), fwd.begin(), fwd.end());
+  }
   const size_t sched_off = ws.total;  // a multiple of 256
   const size_t need = sched_off + blob.size() * sizeof(int32_t);
   if (need > kNoallocScratchBytes) return MAGI_BCA_WORKSPACE_TOO_SMALL;
@@ -131,6 +139,9 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.kv_range = d.kv_range;
   p.rope_q = p.rope_k = nullptr;
   p.drope_q = p.drope_k = nullptr;
+  p.deterministic = d.deterministic;
+  p.dq_units = d.deterministic ? sched + dq_units_off : nullptr;
+  p.dgamma_part = reinterpret_cast<float*>(scratch + ws.dgpart);
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -161,6 +172,6 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
       make_bf16_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_bf16_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  const cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, n_units, s);
+  const cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, n_units, n_dq_units, s);
   return e == cudaSuccess ? MAGI_BCA_OK : record_cuda_failure("allocation-free backward launch", e);
 }

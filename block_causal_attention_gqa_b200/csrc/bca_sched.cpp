@@ -18,6 +18,7 @@ int validate_dims(const magi_bca_dims* dims) {
   if (!(d.rms_eps >= 0.f) || !std::isfinite(d.rms_eps)) return MAGI_BCA_INVALID_ARG;
   if (!(d.softmax_scale >= 0.f) || !std::isfinite(d.softmax_scale)) return MAGI_BCA_INVALID_ARG;
   if (d.kv_range < 0) return MAGI_BCA_INVALID_ARG;
+  if (d.deterministic != 0 && d.deterministic != 1) return MAGI_BCA_INVALID_ARG;
   if (d.head_dim != 64 && d.head_dim != 128) return MAGI_BCA_UNSUPPORTED;
   if (d.heads_q % d.heads_kv != 0) return MAGI_BCA_UNSUPPORTED;
   if (d.n_q_chunks > d.n_kv_chunks) return MAGI_BCA_BAD_OFFSETS;
@@ -150,6 +151,8 @@ double lpt_makespan(const std::vector<double>& costs, int machines) {
 }  // namespace
 
 std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, const magi_bca_dims& d, int num_sms) {
+  // deterministic backward: one unit per kv tile, so each tile's dV and G_k
+  // are written by exactly one CTA
   const int n_qt = (d.seqlen_q + kBlockM - 1) / kBlockM;
   const int n_kt = (d.seqlen_kv + kBlockN - 1) / kBlockN;
   const int group = d.heads_q / d.heads_kv;
@@ -204,7 +207,8 @@ std::vector<int32_t> build_bwd_schedule(const int32_t* qo, const int32_t* ko, co
   // pieces shorter than an eighth of an SM's share only add overhead
   const double min_len = std::max(4.0, (double)total / (8.0 * sms));
   std::vector<int> candidates;
-  for (double c = max_len; c >= min_len; c /= 1.08) candidates.push_back((int)std::lround(c));
+  if (d.deterministic == 0)
+    for (double c = max_len; c >= min_len; c /= 1.08) candidates.push_back((int)std::lround(c));
   if (candidates.empty()) candidates.push_back(max_len);
   int best_len = max_len;
   double best_span = 0.0;

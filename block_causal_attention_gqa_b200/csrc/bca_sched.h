@@ -66,7 +66,8 @@ std::vector<int32_t> build_fwd_schedule(const int32_t* q_offsets, const int32_t*
 // diag_hi_begin, 0}: query tiles below diag_end straddle the first row that
 // sees the kv tile, and query tiles at or above diag_hi_begin straddle the
 // first row (under a KV range) that no longer sees all of it, so both need
-// the mask; units are sorted longest first.
+// the mask; units are sorted longest first.  With d.deterministic every kv
+// tile is one unit (no pieces), so one CTA writes each tile's dV and G_k.
 std::vector<int32_t> build_bwd_schedule(const int32_t* q_offsets, const int32_t* kv_offsets,
                                         const magi_bca_dims& d, int num_sms);
 

@@ -89,6 +89,13 @@ typedef struct {
   int32_t kv_range;     /* KV range in chunks (MAGI-1 §2.4.4, §2.6, Fig. 12): > 0 limits the query
                          * chunk matched to kv chunk c to kv chunks [c - kv_range + 1, c] (1 = its
                          * own chunk only); 0 = no limit (every kv chunk up to c).  Must be >= 0. */
+  int32_t deterministic; /* backward only: 1 = every gradient is summed in a fixed order, so two calls
+                          * with the same inputs on the same device give the same bits (dq comes from
+                          * a query-major pass that owns each query tile, no dq reductions across
+                          * CTAs; each kv tile is one work unit; dgamma and the angle gradients are
+                          * reduced in a fixed order).  Costs about 7/5 of the tensor work of 0.
+                          * 0 = fastest (fp32 reductions whose order depends on timing).  The
+                          * forward is always deterministic and ignores it.  Must be 0 or 1. */
 } magi_bca_dims;
 
 /* Forward.  Writes out (bf16) and lse (fp32; may be NULL when the caller
@@ -204,12 +211,15 @@ int magi_bca_profile_events(void* event_begin, void* event_end);
  * A work unit is up to two 128-row query tiles ("sub-tiles") that read the
  * same key/value head and visit the same kv tiles, so every K/V tile the
  * unit loads into shared memory serves both.  For every unit the scheduler
- * emits 8 int32 values:
- *   {batch, kv_head, head_0, m0_0, head_1, m0_1, n_full, n_tiles}
+ * emits 12 int32 values:
+ *   {batch, kv_head, head_0, m0_0, head_1, m0_1, n_full, n_tiles,
+ *    t_begin, t_full_begin, 0, 0}
  * where (head_s, m0_s) is sub-tile s's query head and first query row
- * (head_1 = -1 when the unit has one sub-tile), n_tiles is the number of
- * 128-token kv tiles visited and n_full how many of them (from tile 0) need
- * no mask.  Units are listed in launch order: longest first.
+ * (head_1 = -1 when the unit has one sub-tile); kv tiles [t_begin, n_tiles)
+ * are visited (t_begin > 0 only under a KV range) and tiles below
+ * t_full_begin or from n_full on need the per-row mask.  Units are listed in
+ * launch order: longest first.  The deterministic backward's query-major dq
+ * pass runs the same units, one CTA per sub-tile.
  * Returns the number of units (even if larger than `capacity`, in which case
  * only `capacity` units are written), or a negative status. */
 int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
@@ -220,11 +230,13 @@ int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
  * a step is one (query tile qt, query head g of the kv head's group) that sees
  * the tile, numbered qt * G + g with G = heads_q / heads_kv.  Each tile's steps
  * are cut into near-equal pieces whose length is chosen by simulating how
- * `num_sms` SMs would run them.  Per unit 8 int32:
+ * `num_sms` SMs would run them (with dims->deterministic = 1 every tile is
+ * one unit).  Per unit 8 int32:
  *   {batch, kv_head, n0 (first key), step_begin, step_end,
- *    diag_end (query tiles below it need the mask), 0, 0}
- * in launch order (longest first).  Returns the number of units (writing at
- * most `capacity`), or a negative status. */
+ *    diag_end, diag_hi_begin, 0}
+ * where query tiles below diag_end or from diag_hi_begin on (KV range) need
+ * the mask, in launch order (longest first).  Returns the number of units
+ * (writing at most `capacity`), or a negative status. */
 int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
                               const magi_bca_dims* dims, int32_t num_sms, int32_t* units, int64_t capacity);
 

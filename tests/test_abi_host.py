@@ -64,6 +64,7 @@ def dims_for(qo, ko, B=1, Hq=4, Hkv=2, D=128, eps=1e-6, scale=0.0):
     ("head_dim_96", UNSUPPORTED), ("gqa_indivisible", UNSUPPORTED),
     ("first_not_zero", BAD_OFFSETS), ("last_not_seqlen", BAD_OFFSETS), ("empty_chunk", BAD_OFFSETS),
     ("decreasing", BAD_OFFSETS), ("more_q_than_kv_chunks", BAD_OFFSETS), ("negative_kv_range", INVALID_ARG),
+    ("deterministic_2", INVALID_ARG),
 ])
 def test_invalid_arguments_are_rejected_on_the_host(case, expect):
     qo, ko = _offs([10, 20]), _offs([10, 20])
@@ -101,6 +102,8 @@ def test_invalid_arguments_are_rejected_on_the_host(case, expect):
         d = dims_for(qo, ko)
     elif case == "negative_kv_range":
         d.kv_range = -1
+    elif case == "deterministic_2":
+        d.deterministic = 2
     assert call_fwd(d, qo, ko, **kw) == expect
 
 
@@ -292,11 +295,12 @@ def test_workload_shapes():
     assert (w.batch, w.seqlen_q, w.seqlen_kv) == (2, 23040, 92160)
 
 
-def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=0):
+def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=0, deterministic=False):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
     G = Hq // Hkv
-    units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms, kv_range=kv_range)
+    units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms, kv_range=kv_range,
+                                      deterministic=deterministic)
     M = TileMask(qo, ko, kv_range)
     n_qt, n_kt = -(-Sq // 128), -(-Skv // 128)
     cover = np.zeros((B, Hkv, n_kt, n_qt, G), np.int64)
@@ -348,6 +352,33 @@ def test_bwd_schedule_covers_each_visible_step_once(q_lens, kv_lens, B, Hq, Hkv)
 ])
 def test_bwd_schedule_with_kv_range(q_lens, kv_lens, R):
     check_bwd_schedule(q_lens, kv_lens, 2, 8, 2, kv_range=R)
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,B,Hq,Hkv,R", [
+    ([1024] * 4, [1024] * 4, 1, 16, 4, 0),
+    ([100, 333, 1000, 67], [100, 333, 1000, 67], 2, 4, 2, 0),
+    ([150, 250], [300, 200, 150, 250], 2, 8, 2, 0),
+    ([300, 200, 150, 250, 100], [300, 200, 150, 250, 100], 1, 8, 2, 2),
+    ([1] * 37, [1] * 37, 1, 2, 1, 5),
+])
+def test_deterministic_bwd_schedule_has_one_unit_per_kv_tile(q_lens, kv_lens, B, Hq, Hkv, R):
+    """The deterministic backward writes each kv tile's dV and G_k from exactly
+    one CTA: every (batch, kv head, kv tile) is one unit holding all its steps."""
+    units = check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R, deterministic=True)
+    keys = [tuple(u[:3]) for u in units]
+    assert len(keys) == len(set(keys))
+    pieces = check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=R)
+    for key in set(keys):
+        mine = [u for u in pieces if tuple(u[:3]) == key]
+        whole = [u for u in units if tuple(u[:3]) == key][0]
+        assert min(u[3] for u in mine) == whole[3] and max(u[4] for u in mine) == whole[4]
+
+
+def test_dims_struct_layout():
+    """magi_bca_dims: ten 4-byte fields, then kv_range and deterministic."""
+    assert ctypes.sizeof(bca.Dims) == 48
+    assert bca.Dims.kv_range.offset == 40 and bca.Dims.deterministic.offset == 44
+    assert bca.make_dims(1, 8, 8, 2, 1, 64, 1, 1, deterministic=True).deterministic == 1
 
 
 def lpt_span(costs, machines):

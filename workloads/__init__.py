@@ -50,6 +50,7 @@ class Workload:
     token_scale: bool = False    # LogNormal(0, 0.5) per-token scale on q and k
     kv_range: int = 0            # KV range in chunks (0 = every earlier chunk); MAGI-1 §2.4.4, Fig. 12
     rope: bool = False           # rotary angles for q and k (3D positions, see rope_angles)
+    deterministic: bool = False  # backward with every sum in a fixed order (same bits on every call)
 
     @property
     def seqlen_q(self) -> int:
@@ -101,9 +102,16 @@ WORKLOADS = {
     # RoPE; angles from the 6 x 24 x 40 latent grid of each chunk, see rope_angles).
     "model46k_rope": Workload("model46k_rope", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760),
                               24, 8, 128, seed=7, backward=True, rope=True),
+    # model46k through the deterministic backward (dq from a query-major pass, one unit
+    # per kv tile, fixed-order dgamma): the reproducible-training setting
+    "model46k_det": Workload("model46k_det", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760),
+                             24, 8, 128, seed=2, backward=True, deterministic=True),
+    "train4k_det": Workload("train4k_det", 1, uniform_offsets(4, 1024), uniform_offsets(4, 1024),
+                            16, 4, 128, seed=1, backward=True, deterministic=True),
 }
 
-ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k", "model46k_rope"]
+ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k", "model46k_rope",
+         "model46k_det", "train4k_det"]
 
 
 def workload(name_or_index) -> Workload:

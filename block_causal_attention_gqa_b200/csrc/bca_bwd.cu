@@ -292,6 +292,12 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int diag_hi_begin = __ldg(u + 6);
   const int group = p.heads_q / p.heads_kv;
   const int n_steps = s_end - s_begin;
+  // Within each query tile the group's heads are visited from head rot on:
+  // neighbouring kv tiles (which walk the same query tiles at the same time)
+  // then add their G_q into different heads' dq rows, not all into the same
+  // rows at once.  rot depends on the kv tile only, so all pieces of a tile
+  // agree on which step is which head.
+  const int rot = (n0 >> 7) % group;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -349,7 +355,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       for (int t = 0; t < n_steps; ++t) {
         const int st = t & 1;
         if (!mbar_wait(&bars->q_empty[st], ((t >> 1) & 1) ^ 1, p.status, kErrQEmpty)) break;
-        const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
+        const int qt = (s_begin + t) / group, h = hk * group + ((s_begin + t) % group + rot) % group;
         // the single {-lse, -Delta} buffer: the previous step's S^T/dP^T have read it
         if (t > 0 && !mbar_wait(&bars->ld_empty, (t - 1) & 1, p.status, kErrLdEmpty)) break;
         mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2048);
@@ -364,7 +370,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // warm L2 with the next step's tiles: their loads are issued only once
         // a stage frees, and then wait on memory otherwise
         if (t + 1 < n_steps) {
-          const int qt1 = (s_begin + t + 1) / group, h1 = hk * group + (s_begin + t + 1) % group;
+          const int qt1 = (s_begin + t + 1) / group, h1 = hk * group + ((s_begin + t + 1) % group + rot) % group;
           for (int box = 0; box < D / 64; ++box) {
             tma_prefetch_l2_4d(&tm_qn, box * 64, h1, qt1 * 128, b);
             tma_prefetch_l2_4d(&tm_do, box * 64, h1, qt1 * 128, b);
@@ -502,7 +508,7 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
       const int st = t & 1;
-      const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
+      const int qt = (s_begin + t) / group, h = hk * group + ((s_begin + t) % group + rot) % group;
       const int q0 = qt * 128;
       const bool diag = qt < diag_end || qt >= diag_hi_begin;
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);

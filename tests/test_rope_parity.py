@@ -95,7 +95,7 @@ def test_rope_full_size_sampled_rows():
     out, lse = bca.magi_bca_fwd_rope(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, rq, rk)
     dq, _, _, _, _, _, _ = bca.magi_bca_bwd_rope(q, k, v, out, do, lse, w.q_offsets, w.kv_offsets, gq, gk, rq, rk)
     torch.cuda.synchronize()
-    rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, 2048, seed=300)
+    rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, 1024, seed=300)
     idx = torch.as_tensor(rows)
     o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
                                     inp["gamma_k"], rows, rope_q=inp["rope_q"], rope_k=inp["rope_k"])

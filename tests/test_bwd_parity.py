@@ -1,7 +1,7 @@
 """GPU parity of the backward against the fp64 oracle (through the C ABI).
 
 Small workloads: dq, dk, dv, dgamma_q, dgamma_k on every row.  Full-size
-training workloads: dq on 1536 stratified query rows per head, dk/dv on
+training workloads: dq on 4096 stratified query rows per head, dk/dv on
 sampled keys of the last chunk (exact and cheap: only last-chunk queries see
 them) where the oracle finishes in seconds, and everywhere the identities
 that hold at any size: sum_j dV_j = sum over the group of sum_i dO_i (rows of
@@ -114,7 +114,7 @@ def test_backward_full_size_sampled(name, kv_heads):
     dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()
     torch.cuda.empty_cache()
     identities(name, w, inp, dq, dk, dv)
-    rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, 1536, seed=200)
+    rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, 4096, seed=200)
     ref = orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
                             inp["gamma_q"], inp["gamma_k"], q_rows=rows, kv_range=w.kv_range)
     idx = torch.as_tensor(rows)

@@ -1,7 +1,7 @@
 """GPU parity of the forward against the fp64 oracle (through the C ABI).
 
 Small workloads are compared on every row; the model-scale, streaming and
-long-context workloads at full size (the launch bench.py times) on 2048
+long-context workloads at full size (the launch bench.py times) on 4096
 stratified query rows per head.  Tolerance: max abs 1e-2 and relative L2
 5e-3 for bf16 inputs with fp32 accumulation."""
 import numpy as np
@@ -108,8 +108,8 @@ def test_forward_full_size_sampled_rows(name):
     out_c, lse_c = out.cpu(), lse.cpu()
     del out, lse
     torch.cuda.empty_cache()
-    # 2048 rows per head, spread over the batch elements
-    per_batch = 2048 // w.batch
+    # 4096 rows per head, spread over the batch elements
+    per_batch = 4096 // w.batch
     for b in range(w.batch):
         rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, per_batch, seed=100 + b)
         o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,

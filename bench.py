@@ -136,7 +136,8 @@ class ClockSampler:
 
 def kernel_source_sha():
     h = hashlib.sha256()
-    for f in ("bca_fwd.cu", "bca_bwd.cu", "sm100.cuh", "bca_norm.cuh", "bca_kernels.h"):
+    for f in ("bca_fwd.cu", "bca_bwd.cu", "bca_bwd_split.cu", "bca_bwd_common.cuh", "sm100.cuh", "bca_norm.cuh",
+              "bca_kernels.h"):
         p = os.path.join(ROOT, "block_causal_attention_gqa_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())

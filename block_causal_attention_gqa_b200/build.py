@@ -10,8 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmagi_bca.so")
-SOURCES = ["bca_api.cu", "bca_fwd.cu", "bca_bwd.cu", "bca_noalloc.cu", "bca_sched.cpp"]
-DEPS = SOURCES + ["sm100.cuh", "bca_kernels.h", "bca_sched.h", "bca_norm.cuh"]
+SOURCES = ["bca_api.cu", "bca_fwd.cu", "bca_bwd.cu", "bca_bwd_split.cu", "bca_noalloc.cu", "bca_sched.cpp"]
+DEPS = SOURCES + ["sm100.cuh", "bca_kernels.h", "bca_sched.h", "bca_norm.cuh", "bca_bwd_common.cuh"]
 
 
 def nvcc():

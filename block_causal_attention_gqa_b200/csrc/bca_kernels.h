@@ -79,6 +79,11 @@ cudaError_t launch_bwd(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUt
                        const CUtensorMap& t_dk, const BwdParams& p, int head_dim, int n_units, int n_dq_units,
                        cudaStream_t stream);
 int make_tensor_map_f32_dq(CUtensorMap* m, const void* base, int B, int S, int H, int D);
+// The deterministic backward's dq pass and dK/dV pass (bca_bwd_split.cu), launched
+// by launch_bwd between the prep and finalize kernels.
+cudaError_t launch_bwd_split(const CUtensorMap& t_k, const CUtensorMap& t_v, const CUtensorMap& t_qn,
+                             const CUtensorMap& t_do, const CUtensorMap& t_dv, const CUtensorMap& t_dk,
+                             const BwdParams& p, int head_dim, int n_units, int n_dq_units, cudaStream_t stream);
 
 // K^ = bf16(rope(k) rsqrt(mean k^2 + eps)) for `rows` rows [B, seqlen, heads] of head_dim
 // features; `rope` = per-token angles [seqlen, head_dim / 2] or nullptr (no rotation).

@@ -129,3 +129,40 @@ def test_backward_full_size_sampled(name, kv_heads):
         for nm, got in (("dk", dk), ("dv", dv)):
             e, r = assert_close(f"{name} {nm} rows", to_np(got[:, kidx][:, :, kv_heads]), ref[nm])
             print(f"{name} {nm} rows: max abs {e:.2e} rel L2 {r:.2e}")
+
+
+def test_backward_canaries_and_finite_outputs():
+    """Every output of the backward inside a larger buffer filled with a canary:
+    nothing is written past (or before) the gradients, and every gradient is
+    finite, for the default and the deterministic path."""
+    w = SMALL["ragged_d64_gqa3"]
+    inp = workloads.make_inputs(w, with_grad_out=True)
+    dev = "cuda"
+    q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
+    gq, gk = inp["gamma_q"].to(dev), inp["gamma_k"].to(dev)
+    dout = inp["dout"].to(dev)
+    out, lse = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk)
+    pad = 4096
+
+    def padded(like, value):
+        big = torch.full((pad + like.numel() + pad,), value, device=dev, dtype=like.dtype)
+        return big, big[pad:pad + like.numel()].view(like.shape)
+
+    ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
+                       inp["gamma_q"], inp["gamma_k"])
+    for det in (False, True):
+        bq, dq = padded(q, 7.0)
+        bk, dk = padded(k, 7.0)
+        bv, dv = padded(v, 7.0)
+        bgq, dgq = padded(gq, 7.0)
+        bgk, dgk = padded(gk, 7.0)
+        bca.magi_bca_bwd(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk, dq=dq, dk=dk, dv=dv,
+                         dgamma_q=dgq, dgamma_k=dgk, deterministic=det)
+        torch.cuda.synchronize()
+        assert bca.magi_bca_last_device_status() == 0
+        for nm, big, t in (("dq", bq, dq), ("dk", bk, dk), ("dv", bv, dv), ("dgamma_q", bgq, dgq),
+                           ("dgamma_k", bgk, dgk)):
+            assert (big[:pad] == 7.0).all() and (big[pad + t.numel():] == 7.0).all(), f"{nm}: canary overwritten"
+            assert torch.isfinite(t).all(), f"{nm}: non-finite values (deterministic={det})"
+        for nm, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+            assert_close(f"canary {nm} det={det}", to_np(got), ref[nm], max_abs=2e-2)

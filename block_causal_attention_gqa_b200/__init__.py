@@ -30,7 +30,8 @@ library_path = os.path.join(_HERE, "libmagi_bca.so")
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
                     "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule",
-                    "magi_bca_profile_events", "magi_bca_fwd_rope", "magi_bca_bwd_rope"]
+                    "magi_bca_profile_events", "magi_bca_fwd_rope", "magi_bca_bwd_rope",
+                    "magi_bca_selftest_wait_timeout"]
 
 
 class MagiBcaError(RuntimeError):
@@ -93,6 +94,8 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_bwd_rope.restype = ctypes.c_int
     lib.magi_bca_profile_events.argtypes = [vp, vp]
     lib.magi_bca_profile_events.restype = ctypes.c_int
+    lib.magi_bca_selftest_wait_timeout.argtypes = [vp]
+    lib.magi_bca_selftest_wait_timeout.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -103,6 +106,17 @@ def magi_bca_status_string(status: int) -> str:
 
 def magi_bca_last_device_status() -> int:
     return int(library().magi_bca_last_device_status())
+
+
+def magi_bca_selftest_wait_timeout(stream=None) -> None:
+    """Diagnostic: one kernel whose bounded wait on an mbarrier that nothing
+    arrives at gives up; magi_bca_last_device_status() then reports the
+    device timeout (-6) without any fault."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = library().magi_bca_selftest_wait_timeout(_stream_handle(stream, dev))
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_selftest_wait_timeout")
 
 
 def magi_bca_profile_events(begin=None, end=None) -> None:

@@ -15,6 +15,7 @@
 #include "../../include/magi_bca.h"
 #include "bca_kernels.h"
 #include "bca_sched.h"
+#include "sm100.cuh"
 
 namespace magi {
 
@@ -23,6 +24,18 @@ __device__ int g_device_status;
 
 // Diagnostic timing events (magi_bca_profile_events); null when unset.
 std::atomic<void*> g_profile_begin{nullptr}, g_profile_end{nullptr};
+
+// Self-test of the bounded-wait path: one thread waits, with a short poll
+// limit, on an mbarrier that nothing arrives at, so the wait gives up and
+// records `code` in the status word as a stalled pipeline stage would.
+__global__ void bca_wait_selftest_kernel(int* status, int code, uint32_t limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    sm100::mbar_wait_limit(&bar, 0, status, code, limit);
+  }
+}
 
 void profile_mark(int which, cudaStream_t stream) {
   void* ev = which == 0 ? g_profile_begin.load() : g_profile_end.load();
@@ -442,6 +455,16 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
 }
 
 const char* magi_bca_last_error_detail(void) { return g_last_detail; }
+
+int magi_bca_selftest_wait_timeout(void* stream) {
+  int dev;
+  DeviceState* ds;
+  const int st = device_state(&dev, &ds);
+  if (st != MAGI_BCA_OK) return st;
+  bca_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ds->status, 9001, 4096u);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("wait self-test launch", e);
+}
 
 int magi_bca_last_device_status(void) {
   int host = 0;

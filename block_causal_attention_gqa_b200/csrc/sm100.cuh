@@ -91,15 +91,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // hardware-chosen interval, so this is many seconds of real waiting.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
-// Bounded wait.  On timeout writes `code` into *status (first writer wins)
-// and returns false; callers then skip the rest of their work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int code) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+// Bounded wait of at most `limit` polls.  On timeout writes `code` into
+// *status (first writer wins) and returns false; callers then skip the rest
+// of their work.  It also gives up early once another wait has failed.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* status, int code,
+                                                uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 1023u) == 1023u && status != nullptr && *(volatile int*)status != 0) return false;
   }
   if (status != nullptr) atomicCAS(status, 0, code);
   return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int code) {
+  return mbar_wait_limit(bar, parity, status, code, kSpinLimit);
 }
 
 // ---------------------------------------------------------------- TMA

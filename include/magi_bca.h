@@ -207,6 +207,16 @@ int magi_bca_last_device_status(void);
  * one handle is NULL. */
 int magi_bca_profile_events(void* event_begin, void* event_end);
 
+/* Self-test of the device-timeout path (diagnostic; the paper has no
+ * counterpart).  Launches one small kernel on `stream` whose bounded wait, on
+ * an mbarrier that nothing arrives at, gives up after a short poll limit and
+ * records a device status code, as a stalled pipeline stage in the attention
+ * kernels would.  A following magi_bca_last_device_status() returns
+ * MAGI_BCA_DEVICE_TIMEOUT (and clears the word); the CUDA context stays
+ * usable.  Returns MAGI_BCA_OK, MAGI_BCA_UNSUPPORTED (device) or
+ * MAGI_BCA_CUDA_ERROR (launch failure). */
+int magi_bca_selftest_wait_timeout(void* stream);
+
 /* Host-only view of the tile schedule the kernels run (no device needed).
  * A work unit is up to two 128-row query tiles ("sub-tiles") that read the
  * same key/value head and visit the same kv tiles, so every K/V tile the

@@ -542,7 +542,8 @@ def run_reference(args, w, world, rank):
         "config": {"workload": w.name, "pass": args.pass_, "batch": w.batch, "seqlen_q": w.seqlen_q,
                    "seqlen_kv": w.seqlen_kv, "q_chunks": f"{len(w.q_chunks)}x{w.q_chunks[0]}",
                    "kv_chunks": f"{len(w.kv_chunks)}x{w.kv_chunks[0]}", "heads_q": w.heads_q,
-                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range, "rope": w.rope},
+                   "heads_kv": w.heads_kv, "head_dim": w.head_dim, "kv_range": w.kv_range, "rope": w.rope,
+                   "deterministic": w.deterministic},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -412,3 +412,27 @@ def test_profile_events_argument_check():
     assert lib.magi_bca_profile_events(256, None) == INVALID_ARG
     assert lib.magi_bca_profile_events(None, 256) == INVALID_ARG
     assert lib.magi_bca_profile_events(None, None) == OK
+
+
+@pytest.mark.parametrize("entry", ["fwd", "fwd_rope", "bwd", "bwd_rope", "bwd_noalloc"])
+def test_no_cpu_fallback_host_tensors_are_refused(entry):
+    """The product path has no CPU or PyTorch fallback: every entry point
+    refuses host tensors before anything is computed."""
+    import torch
+    B, S, H, D = 1, 128, 2, 64
+    q = torch.zeros(B, S, H, D, dtype=torch.bfloat16)
+    k = torch.zeros(B, S, 1, D, dtype=torch.bfloat16)
+    v = torch.zeros_like(k)
+    g = torch.ones(D)
+    lse = torch.zeros(B, H, S)
+    ang = torch.zeros(S, D // 2)
+    offs = [0, 64, 128]
+    calls = {
+        "fwd": lambda: bca.magi_bca_fwd(q, k, v, offs, offs, g, g),
+        "fwd_rope": lambda: bca.magi_bca_fwd_rope(q, k, v, offs, offs, g, g, ang, ang),
+        "bwd": lambda: bca.magi_bca_bwd(q, k, v, q, q, lse, offs, offs, g, g),
+        "bwd_rope": lambda: bca.magi_bca_bwd_rope(q, k, v, q, q, lse, offs, offs, g, g, ang, ang),
+        "bwd_noalloc": lambda: bca.magi_bca_bwd_noalloc(q, k, v, q, q, lse, offs, offs, g, g, q, k, v),
+    }
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        calls[entry]()

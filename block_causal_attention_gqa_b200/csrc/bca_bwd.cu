@@ -35,14 +35,14 @@
 //                one kv tile).
 //   3. finalize  one warp per row: dq, dk through the RMSNorm Jacobian, dv, and
 //                dgamma_q, dgamma_k.
-// Deterministic backward (dims.deterministic): no sum depends on timing.  The
-// dq pass (bca_bwd_dq_kernel, query-major, one CTA per query tile) computes
-// G_q before the main kernel, which then skips its G_q product and drain;
-// every kv tile is one main-kernel unit, so dV and G_k are added once onto
-// zero; the finalize takes whole tokens (angle gradients summed in registers)
-// and writes per-block dgamma partials that one small kernel adds in block
-// order.  The dq pass recomputes S and dP, so the tensor work is 7/5 of the
-// default path's.
+// Deterministic backward (dims.deterministic): no sum depends on timing.  In
+// place of the main kernel, bca_bwd_split.cu runs a query-major dq pass (one
+// CTA per query tile owns its rows' G_q) and a kv-major dK/dV pass without
+// G_q, with every kv tile one unit, so dV and G_k are added once onto zero;
+// the finalize takes whole tokens (angle gradients summed in registers) and
+// writes per-block dgamma partials that one small kernel adds in block order.
+// The dq pass recomputes S and dP, so the tensor work is 7/5 of the default
+// path's.
 // These are the five matrix products of the Flash-Attention backward (2.5x the
 // forward's FLOPs, MAGI-1 App. B.2.1).  Because gamma_k is folded into the
 // query operand, dgamma_k[d] is undefined (NaN/inf) where gamma_k[d] == 0.

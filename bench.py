@@ -393,8 +393,8 @@ def run_ours(args, w, world, rank, local):
     bwd_avg = float(np.mean(bwd_ms)) if do_bwd else 0.0
     dom_ms = float(np.mean(kernel_ms))
     if do_bwd:
-        # deterministic backward: the events bracket the dq pass and the main kernel
-        dom = "bca_bwd_dq_kernel+bca_bwd_main_kernel" if w.deterministic else "bca_bwd_main_kernel"
+        # deterministic backward: the events bracket the dq pass and the dK/dV pass
+        dom = "bca_bwd_dq_kernel+bca_bwd_dkdv_kernel" if w.deterministic else "bca_bwd_main_kernel"
         dom_flops = bwd_flops(w)
     else:
         dom, dom_flops = "bca_fwd_kernel", fwd_flops(w)

@@ -202,8 +202,9 @@ int magi_bca_last_device_status(void);
  * `event_end` are cudaEvent_t handles created by the caller.  While both are
  * non-NULL, every magi_bca_fwd / magi_bca_bwd / magi_bca_bwd_noalloc call
  * records event_begin on its stream immediately before launching its main
- * kernel (bca_fwd_kernel or bca_bwd_main_kernel) and event_end immediately
- * after, so the caller can time that kernel alone with cudaEventElapsedTime.
+ * kernel (bca_fwd_kernel or bca_bwd_main_kernel; with dims->deterministic the
+ * backward's dq and dK/dV passes together) and event_end immediately after, so
+ * the caller can time that work alone with cudaEventElapsedTime.
  * Pass NULL, NULL to stop.  Process-wide setting; not for concurrent calls on
  * several streams.  Returns MAGI_BCA_OK, or MAGI_BCA_INVALID_ARG if exactly
  * one handle is NULL. */

@@ -418,6 +418,13 @@ def run_ours(args, w, world, rank, local):
                 "traffic": ncu_traffic(dom, w.name),
                 "avg_launch_ms": round(dom_ms, 4),
                 "algorithmic_bytes_per_launch": fwd_bytes(w) if dom == "bca_fwd_kernel" else None}
+    # HBM rate of the dominant kernel: ncu's DRAM bytes per launch (and, for the
+    # forward, the algorithmic bytes) over the live launch time
+    if roofline["traffic"] is not None and dom_ms > 0:
+        roofline["dram_gbs"] = round(roofline["traffic"] / (dom_ms * 1e-3) / 1e9, 1)
+        roofline["dram_frac_of_hbm_peak"] = round(roofline["dram_gbs"] / peaks["hbm_gbs"], 4)
+    if roofline["algorithmic_bytes_per_launch"] is not None and dom_ms > 0:
+        roofline["algorithmic_gbs"] = round(roofline["algorithmic_bytes_per_launch"] / (dom_ms * 1e-3) / 1e9, 1)
     launches_per_step = bca_fwd_launches() + (bca_bwd_launches(w) if do_bwd else 0)
     res = {
         "metric": "block-causal attention useful TFLOP/s on 1 B200 and % of dense BF16 peak",

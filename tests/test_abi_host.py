@@ -436,3 +436,41 @@ def test_no_cpu_fallback_host_tensors_are_refused(entry):
     }
     with pytest.raises(TypeError, match="CUDA tensor"):
         calls[entry]()
+
+
+def random_layouts(seed, n):
+    """Seeded random chunk layouts: 1-6 kv chunks of 1-700 tokens (rarely tile
+    aligned), the query side the last 1..n_kv of them (training layout when all)
+    or, one time in four, chunks of other lengths (cross-attention), a KV range
+    of 0-3, batch 1-2 and a GQA ratio of 1-4."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        n_kv = int(rng.integers(1, 7))
+        kv = [int(x) for x in rng.integers(1, 701, n_kv)]
+        n_q = int(rng.integers(1, n_kv + 1))
+        if rng.random() < 0.25:
+            q = [int(x) for x in rng.integers(1, 701, n_q)]
+        else:
+            q = kv[n_kv - n_q:]
+        hkv = int(rng.integers(1, 3))
+        out.append((q, kv, int(rng.integers(1, 3)), hkv * int(rng.integers(1, 5)), hkv, int(rng.integers(0, 4))))
+    return out
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,B,Hq,Hkv,R", random_layouts(2024, 24))
+def test_schedules_on_random_layouts(q_lens, kv_lens, B, Hq, Hkv, R):
+    """Both schedules against the oracle's token mask (through the row
+    intervals) on random layouts: the forward visits exactly the kv tiles with
+    a visible pair and masks every tile it does not see whole; the backward
+    covers each visible (kv tile, query tile, head) once, pieced and whole."""
+    from oracle import bca_oracle as orc
+    qo, ko = _offs(q_lens), _offs(kv_lens)
+    b, e = row_intervals(qo, ko, R)
+    keys = np.arange(int(ko[-1]))
+    assert np.array_equal(orc.block_causal_mask(qo, ko, kv_range=R),
+                          (keys[None, :] >= b[:, None]) & (keys[None, :] < e[:, None]))
+    check_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R, deterministic=True)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=7, kv_range=R)

@@ -474,3 +474,22 @@ def test_schedules_on_random_layouts(q_lens, kv_lens, B, Hq, Hkv, R):
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R)
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R, deterministic=True)
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=7, kv_range=R)
+
+
+def test_maximum_sizes():
+    """The kernels index rows with 32-bit TMA coordinates and flattened 32-bit
+    row numbers: a problem with 2^31 or more query (or key) rows is refused on
+    the host; one just below the limit passes the checks."""
+    lib = bca.library()
+    # 2^31 query rows: batch 1, 2^27 tokens, 16 heads
+    S = 1 << 27
+    qo = np.array([0, S], np.int32)
+    d = bca.make_dims(1, S, S, 16, 2, 128, 1, 1)
+    assert lib.magi_bca_fwd_schedule(bca._i32p(qo), bca._i32p(qo), ctypes.byref(d), None, 0) == UNSUPPORTED
+    assert bca.magi_bca_bwd_workspace_size(d) == 0
+    # just below: 2^31 - 16 query rows pass the same checks (the workspace query
+    # runs them without building the 8-million-unit schedule)
+    S2 = (1 << 27) - 1
+    d2 = bca.make_dims(1, S2, S2, 16, 2, 128, 1, 1)
+    ws = bca.magi_bca_bwd_workspace_size(d2)
+    assert ws >= S2 * 16 * 128 * (2 + 4)   # at least Q^ (bf16) and the fp32 dq accumulator

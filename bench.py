@@ -571,7 +571,7 @@ def main():
     args.warmup = max(args.warmup, 3)
     w = workloads.workload(args.config)
     if args.pass_ is None:
-        args.pass_ = "fwdbwd" if (w.backward and BWD_AVAILABLE) else "fwd"
+        args.pass_ = "fwdbwd" if w.backward else "fwd"
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":
@@ -590,8 +590,6 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
 
-
-BWD_AVAILABLE = True
 
 if __name__ == "__main__":
     main()

@@ -15,39 +15,6 @@ namespace magi {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Accumulates x*x over the 8 bf16 of one 16-byte chunk, lowest feature first.
-__device__ __forceinline__ float sumsq_chunk(uint4 v, float acc) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc = fmaf(bf16_lo(w[i]), bf16_lo(w[i]), acc);
-    acc = fmaf(bf16_hi(w[i]), bf16_hi(w[i]), acc);
-  }
-  return acc;
-}
-
-// Sum of squares of row `row` of a [128][D] bf16 tile stored as D/64 boxes
-// of [128][64] with the 128-byte swizzle.
-template <int D>
-__device__ __forceinline__ float row_sumsq_swizzled(const uint8_t* tile, int row) {
-  float acc = 0.f;
-#pragma unroll
-  for (int box = 0; box < D / 64; ++box)
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      acc = sumsq_chunk(*reinterpret_cast<const uint4*>(tile + box * 16384 + sm100::sw128_offset(row, c * 8)), acc);
-  return acc;
-}
-
-// Same sum for a contiguous row in global memory (16-byte aligned).
-template <int D>
-__device__ __forceinline__ float row_sumsq_linear(const uint16_t* row) {
-  float acc = 0.f;
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) acc = sumsq_chunk(*reinterpret_cast<const uint4*>(row + c * 8), acc);
-  return acc;
-}
-
 // The same sum in the order a warp computes it when lane l holds features
 // [l*E, l*E + E) (E = D/32): per-lane fmaf chains, then an xor butterfly
 // (offsets 16, 8, 4, 2, 1).  Floating-point addition is commutative, so every

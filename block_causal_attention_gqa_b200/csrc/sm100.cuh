@@ -38,18 +38,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
-// Per-warpgroup register reallocation (all four warps of a warpgroup execute
-// it).  The block's pool is its launch allocation; increases wait until
-// decreases elsewhere have released enough registers.
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_increase() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kRegs));
-}
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_decrease() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kRegs));
-}
-
 // ----------------------------------------------------------- mbarriers
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
@@ -137,31 +125,12 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* gsrc, uint32_t byte
                : "memory");
 }
 
-// 4-D tiled bulk tensor store shared -> global (out-of-range parts clipped).
-__device__ __forceinline__ void tma_store_4d(const void* desc, const void* smem_src, int c0, int c1,
-                                             int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(
-          reinterpret_cast<uint64_t>(desc)),
-      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_store_commit() {
   asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
 }
 
-__device__ __forceinline__ void tma_store_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
-}
-
 __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-}
-
-// Wait until at most one committed bulk group is still reading shared memory.
-__device__ __forceinline__ void tma_store_wait_read_allow1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory");
 }
 
 // ----------------------------------------------------------- tcgen05
@@ -328,16 +297,6 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
 }
 
-// 3-D tiled bulk tensor load global -> shared, completing on `bar`.
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* desc, uint64_t* bar, int c0, int c1,
-                                            int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
 // Plain (non-tensor) bulk copy global -> shared of `bytes` (multiple of 16,
 // both addresses 16-byte aligned), completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
@@ -357,12 +316,6 @@ __device__ __forceinline__ void tma_reduce_add_4d(const void* desc, const void* 
           reinterpret_cast<uint64_t>(desc)),
       "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
-}
-
-// Vector fp32 atomic add to global memory (no return value).
-__device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(gptr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 
 // ----------------------------------------------------- packed fp32 pairs

@@ -123,7 +123,6 @@ int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
                       magi_bca_bf16* out, float* lse,
                       const magi_bca_dims* dims, void* stream);
 
-/* Bytes of device workspace magi_bca_bwd needs for `dims` (0 on invalid dims). */
 /* Bytes of device workspace magi_bca_bwd / magi_bca_bwd_rope need for `dims`
  * (either value of dims->deterministic); 0 if dims is NULL or invalid. */
 size_t magi_bca_bwd_workspace_size(const magi_bca_dims* dims);

@@ -567,6 +567,10 @@ def main():
     ap.add_argument("--pass", dest="pass_", default=None, choices=["fwd", "fwdbwd"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: every rank runs the whole workload (weak scaling); heads: the "
+                         "kv heads (with their query-head groups) are split over the ranks, one "
+                         "problem in all (strong scaling, no collective on the data path)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = workloads.workload(args.config)
@@ -576,6 +580,17 @@ def main():
     try:
         if args.impl == "reference":
             res = run_reference(args, w, world, rank)
+            if res is not None and args.shard == "heads":
+                res["scaling"] = "strong"
+        elif args.shard == "heads":
+            res = run_ours(args, workloads.shard_heads(w, world, rank), world, rank, local)
+            # the line describes the whole problem: value and e2e already count
+            # every rank's share (world x the per-rank FLOPs over the slowest rank)
+            res["scaling"] = "strong"
+            res["config"].update({"workload": w.name, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+                                  "parallelism": f"kv heads split over {world} ranks",
+                                  "useful_tflop_per_step": round(fwd_flops(w) / 1e12 + (
+                                      bwd_flops(w) / 1e12 if args.pass_ == "fwdbwd" else 0.0), 4)})
         else:
             res = run_ours(args, w, world, rank, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -120,6 +120,20 @@ def workload(name_or_index) -> Workload:
     return WORKLOADS[name_or_index]
 
 
+def shard_heads(w: Workload, world: int, rank: int) -> Workload:
+    """Rank `rank`'s share of `w` when its key/value heads (each with its whole
+    group of query heads) are split over `world` ranks: the same chunks and
+    head_dim with heads_kv / world kv heads and heads_q / world query heads.
+    Each kv head's attention is independent of the others, so the shards need
+    no exchange.  Each rank draws its own inputs (seed + rank)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    if w.heads_kv % world != 0:
+        raise ValueError(f"{w.name}: {w.heads_kv} kv heads do not split over {world} ranks")
+    return dataclasses.replace(w, name=f"{w.name}[heads {rank}/{world}]", heads_q=w.heads_q // world,
+                               heads_kv=w.heads_kv // world, seed=w.seed + rank)
+
+
 def custom(name: str, batch: int, q_chunks: Sequence[int], kv_chunks: Optional[Sequence[int]],
            heads_q: int, heads_kv: int, head_dim: int, seed: int, backward: bool = True,
            gamma: str = "perturbed", token_scale: bool = False, kv_range: int = 0,

@@ -561,3 +561,93 @@ def test_rope_backward_rows_match_full_backward():
     np.testing.assert_allclose(part["dq"][0], full["dq"][0, rows], rtol=0, atol=1e-12)
     np.testing.assert_allclose(part["dk"][0], full["dk"][0, kv_rows], rtol=0, atol=1e-12)
     np.testing.assert_allclose(part["dv"][0], full["dv"][0, kv_rows], rtol=0, atol=1e-12)
+
+
+def read_rope_fixture(name):
+    cases, cur = [], {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            cur[key] = np.array([float(x) for x in vals])
+            if key == "y":
+                cases.append(cur)
+                cur = {}
+    return cases
+
+
+def test_rope_matches_hand_written_quarter_turns():
+    """Direction and pairing: a quarter turn of pair 0 sends e0 to e4 and e4 to
+    -e0 (pairs are (i, i + D/2), turning counter-clockwise).  Rotating by -t
+    or pairing (2i, 2i + 1) fails here."""
+    cases = read_rope_fixture("rope_quarter_turn_d8.txt")
+    assert len(cases) == 7
+    for c in cases:
+        x = c["x"].reshape(1, 1, 1, 8)          # [B, S, H, D]
+        y = orc.rope(x, (np.pi * c["angles"]).reshape(1, 4))
+        np.testing.assert_allclose(y.reshape(8), c["y"], rtol=0, atol=1e-14)
+
+
+def torch_rope_reference(q, k, v, qo, ko, gq, gk, tq, tk, eps=1e-6, order="rope_then_norm"):
+    """fp64 torch composition, independent of the oracle's rotation code: the
+    pairs (x_i, x_{i+D/2}) as complex numbers multiplied by exp(i t)
+    (torch.polar), then F.rms_norm with the gains, then SDPA with a boolean
+    block-causal mask.  order="norm_then_rope" swaps the first two steps."""
+    def rot(x, t):
+        D = x.shape[-1]
+        z = torch.complex(x[..., :D // 2], x[..., D // 2:])
+        w = torch.polar(torch.ones_like(t), t)[None, :, None, :]   # [1, S, 1, D/2]
+        r = z * w
+        return torch.cat([r.real, r.imag], dim=-1)
+
+    Q, K, V = (x if torch.is_tensor(x) else torch.tensor(x) for x in (q, k, v))
+    D = Q.shape[-1]
+    Gq, Gk = (x if torch.is_tensor(x) else torch.tensor(x) for x in (gq, gk))
+    Tq, Tk = (x if torch.is_tensor(x) else torch.tensor(x) for x in (tq, tk))
+    if order == "rope_then_norm":
+        Qn = F.rms_norm(rot(Q, Tq), (D,), weight=Gq, eps=eps)
+        Kn = F.rms_norm(rot(K, Tk), (D,), weight=Gk, eps=eps)
+    else:
+        Qn = rot(F.rms_norm(Q, (D,), weight=Gq, eps=eps), Tq)
+        Kn = rot(F.rms_norm(K, (D,), weight=Gk, eps=eps), Tk)
+    g = Q.shape[2] // K.shape[2]
+    mask = torch.tensor(read_mask_like(qo, ko))
+    o = F.scaled_dot_product_attention(Qn.transpose(1, 2), Kn.repeat_interleave(g, dim=2).transpose(1, 2),
+                                       V.repeat_interleave(g, dim=2).transpose(1, 2), attn_mask=mask)
+    return o.transpose(1, 2)
+
+
+def test_rope_comes_before_the_norm_with_non_unit_gains():
+    """Order against the norm (notes page, DiT-block sketch: RoPE on q and k,
+    then QK-norm), with gains far from 1 so the two orders differ: the oracle
+    equals rotate-then-RMSNorm and differs from RMSNorm-then-rotate."""
+    rng = np.random.default_rng(56)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [5, 4, 6], [5, 4, 6], 4, 2, 16)
+    gq = rng.uniform(0.2, 2.0, 16)
+    gk = rng.uniform(0.2, 2.0, 16)
+    tq = rng.uniform(-3, 3, (15, 8))
+    tk = rng.uniform(-3, 3, (15, 8))
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk, rope_q=tq, rope_k=tk)
+    want = torch_rope_reference(q, k, v, qo, ko, gq, gk, tq, tk).numpy()
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-12)
+    other = torch_rope_reference(q, k, v, qo, ko, gq, gk, tq, tk, order="norm_then_rope").numpy()
+    assert np.abs(other - want).max() > 1e-2
+
+
+def test_rope_backward_matches_torch_autograd_fp64():
+    """Every gradient, the angle gradients included, against torch autograd
+    through the independent composition (complex rotation, F.rms_norm, SDPA)."""
+    rng = np.random.default_rng(57)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, [3, 5, 4], [3, 5, 4], 6, 2, 16)
+    tq = rng.uniform(-3, 3, (12, 8))
+    tk = rng.uniform(-3, 3, (12, 8))
+    do = rng.standard_normal(q.shape)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk, rope_q=tq, rope_k=tk)
+    T = [torch.tensor(x, requires_grad=True) for x in (q, k, v, gq, gk, tq, tk)]
+    o = torch_rope_reference(T[0], T[1], T[2], qo, ko, T[3], T[4], T[5], T[6])
+    (o * torch.tensor(do)).sum().backward()
+    for t, name in zip(T, ["dq", "dk", "dv", "dgamma_q", "dgamma_k", "drope_q", "drope_k"]):
+        np.testing.assert_allclose(g[name], t.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
+    np.testing.assert_allclose(g["out"], o.detach().numpy(), rtol=0, atol=1e-12)

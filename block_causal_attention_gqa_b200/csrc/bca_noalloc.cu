@@ -17,9 +17,12 @@
 // host the name is only a stand-in, not a device address.  The first call on a
 // device looks up the array's device address with cudaGetSymbolAddress (with
 // that device current) and keeps it; make that first call before any stream
-// capture.  All calls share the array and it keeps the last call's contents,
-// so calls that overlap on the GPU (other streams, other threads) race; the
-// kernels clear everything that must start at zero.
+// capture.  Each call copies its tile schedule into the array from host
+// memory, so while its stream is capturing the call returns
+// MAGI_BCA_UNSUPPORTED with nothing enqueued.  All calls share the array and
+// it keeps the last call's contents, so calls that overlap on the GPU (other
+// streams, other threads) race; the kernels clear everything that must start
+// at zero.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -117,6 +120,13 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   if (st != MAGI_BCA_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Every call uploads its schedule from a host vector that is gone when the
+  // call returns, so a capture would record a copy from freed host memory:
+  // refuse while the stream is capturing, before anything is enqueued.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  const cudaError_t ce = cudaStreamIsCapturing(s, &cap);
+  if (ce != cudaSuccess) return record_cuda_failure("cudaStreamIsCapturing", ce);
+  if (cap != cudaStreamCaptureStatusNone) return MAGI_BCA_UNSUPPORTED;
   int32_t* sched = reinterpret_cast<int32_t*>(scratch + sched_off);
   // From pageable host memory the copy is staged before this call returns, so
   // the local vector may go out of scope afterwards.

@@ -361,9 +361,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 // 2^a for a pair, a <= 8.5: j = round(a) via the 1.5*2^23 rounding constant,
 // f = a - j in [-1/2, 1/2], 2^f by a minimax cubic (relative error 7.5e-5,
-// fitted by fit_exp2_poly.py in the package), and 2^j added to the exponent bits.  Inputs
-// below -125 are clamped there (results ~1e-38 instead of smaller); callers
-// use it only where no element is masked to -inf.
+// fitted by the Remez script tests/fit_exp2_poly.py), and 2^j added to the
+// exponent bits.  Inputs below -125 are clamped there (results ~1e-38 instead
+// of smaller); callers use it only where no element is masked to -inf.
 __device__ __forceinline__ void exp2_poly_pair(uint64_t a2, float& p0, float& p1) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   float a0, a1;

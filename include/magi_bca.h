@@ -68,7 +68,8 @@ typedef uint16_t magi_bca_bf16; /* raw bfloat16 bits */
 enum {
   MAGI_BCA_OK = 0,
   MAGI_BCA_INVALID_ARG = -1,        /* null pointer, non-positive size, bad dims struct */
-  MAGI_BCA_UNSUPPORTED = -2,        /* head_dim not 64/128, heads_q % heads_kv != 0, device not sm_100 */
+  MAGI_BCA_UNSUPPORTED = -2,        /* head_dim not 64/128, heads_q % heads_kv != 0, device not sm_100,
+                                     * magi_bca_bwd_noalloc on a capturing stream */
   MAGI_BCA_BAD_OFFSETS = -3,        /* chunk offsets violate the rules above */
   MAGI_BCA_WORKSPACE_TOO_SMALL = -4,
   MAGI_BCA_CUDA_ERROR = -5,         /* a CUDA runtime call failed (launch, copy, ...) */
@@ -156,6 +157,9 @@ int magi_bca_bwd(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi_bca_
  *     head_dim 128 fits.
  *   - The first call on a device looks up the array's device address; make that
  *     first call before any stream capture.
+ *   - Every call copies its tile schedule from host memory into the array, so
+ *     while `stream` is capturing the call returns MAGI_BCA_UNSUPPORTED and
+ *     enqueues nothing.
  *   - All calls share the array and it keeps the last call's contents, so calls
  *     that overlap on the GPU (several streams or threads) race.  Run them in
  *     one stream, one at a time. */

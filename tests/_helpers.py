@@ -20,14 +20,18 @@ def rel_l2(got, want):
 BF16_HALF_ULP_REL = 2.0 ** -8
 
 
-def assert_close(name, got, want, max_abs=MAX_ABS, rel=REL_L2):
+def assert_close(name, got, want, max_abs=MAX_ABS, rel=REL_L2, bf16=True):
+    """Max abs and relative L2 against the oracle.  bf16=True for the bf16
+    outputs (out, dq, dk, dv): the max-abs bound applies beyond their own
+    rounding.  bf16=False for fp32 outputs (lse): plain |got - want| <= max_abs."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape, f"{name}: shape {got.shape} vs {want.shape}"
     assert np.isfinite(got).all(), f"{name}: non-finite values"
     diff = np.abs(got - want)
     err = float(diff.max()) if got.size else 0.0
-    excess = float(np.max(diff - BF16_HALF_ULP_REL * np.abs(want))) if got.size else 0.0
+    slack = BF16_HALF_ULP_REL if bf16 else 0.0
+    excess = float(np.max(diff - slack * np.abs(want))) if got.size else 0.0
     r = rel_l2(got, want)
     assert excess <= max_abs and r <= rel, (f"{name}: max abs {err:.3e} (beyond bf16 rounding {excess:.3e} "
                                             f"<= {max_abs}), rel L2 {r:.3e} (<= {rel})")
@@ -38,3 +42,20 @@ def to_np(t):
     if t.dtype == torch.bfloat16:
         t = t.float()
     return t.detach().cpu().numpy().astype(np.float64)
+
+
+def assert_lse_close(name, got, want):
+    """lse is an fp32 output: the stated bound with no bf16 allowance."""
+    return assert_close(name, got, want, bf16=False)
+
+
+# Gradient max-abs bounds.  Every case is held to the stated 1e-2 except the
+# ones named here, each with the largest element error that a CPU model of the
+# kernels' own bf16 rounding points (tests/numerics_model.py: the same
+# roundings, otherwise exact arithmetic) already reaches on it, and the GPU's.
+# Relative L2 stays 5e-3 for all of them.
+GRAD_MAX_ABS = {}
+
+
+def grad_bound(name):
+    return GRAD_MAX_ABS.get(name, MAX_ABS)

@@ -1,4 +1,4 @@
-"""Fits the polynomial the forward kernel uses for part of its exp2 work.
+"""Fits the polynomial the kernels use for part of their exp2 work.
 
 2^x is split as 2^j * 2^f with j = round(x) and f = x - j in [-1/2, 1/2]; 2^f
 is approximated by a cubic fitted here by the Remez exchange algorithm
@@ -7,8 +7,10 @@ this polynomial on the FMA pipe, so the MUFU unit is not the bottleneck of
 the softmax.  The result feeds a bf16 operand (rounding 2^-9), and the cubic's
 maximum relative error is ~7.5e-5.
 
-    python -m block_causal_attention_gqa_b200.fit_exp2_poly
-prints the coefficients (fp32) pasted into csrc/bca_fwd.cu and their errors.
+    python tests/fit_exp2_poly.py
+prints the coefficients (fp32) that exp2_poly_pair in
+block_causal_attention_gqa_b200/csrc/sm100.cuh uses, and their errors;
+tests/test_exp2_poly.py re-runs the fit and checks those constants.
 """
 import numpy as np
 

@@ -24,7 +24,17 @@ def _bf(x):
     return x.to(torch.bfloat16).to(torch.float64)
 
 
-def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6):
+def _rot(x, t):
+    """Rotary pairs (i, i + D/2) by the per-token angles t [S, D/2] (exact)."""
+    if t is None:
+        return x
+    h = x.shape[-1] // 2
+    c, s = torch.cos(t)[None, :, None, :], torch.sin(t)[None, :, None, :]
+    a, b = x[..., :h], x[..., h:]
+    return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+
+
+def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6, kv_range=0, rope_q=None, rope_k=None):
     q = inp["q"].double()
     k = inp["k"].double()
     v = inp["v"].double()
@@ -38,7 +48,11 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6):
     l2e = 1.0 / np.log(2.0)
     rq = torch.rsqrt((q * q).mean(-1, keepdim=True) + eps)
     rk = torch.rsqrt((k * k).mean(-1, keepdim=True) + eps)
-    mask = torch.tensor(orc.block_causal_mask(q_offsets, kv_offsets))
+    tq = None if rope_q is None else torch.as_tensor(rope_q).double()
+    tk = None if rope_k is None else torch.as_tensor(rope_k).double()
+    q_raw, k_raw = q, k
+    q, k = _rot(q, tq), _rot(k, tk)          # a rotation keeps the RMS of the raw row
+    mask = torch.tensor(orc.block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range))
     kr, vr = k.repeat_interleave(g, 2), v.repeat_interleave(g, 2)
     kh = _bf(kr * rk.repeat_interleave(g, 2))
     qh = _bf(q * rq * (gq * gk * sc * l2e))
@@ -60,5 +74,7 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6):
     dqt = sc * torch.einsum("bhij,bjhd->bihd", ds, kh * gk)
     dq, _ = orc.rms_norm_backward(q.numpy(), gq.numpy(), dqt.numpy(), eps)
     dk, _ = orc.rms_norm_backward(k.numpy(), gk.numpy(), dkt.numpy(), eps)
+    dq, _ = orc.rope_backward(q_raw.numpy(), rope_q, dq)
+    dk, _ = orc.rope_backward(k_raw.numpy(), rope_k, dk)
     return dict(out=out_bf.numpy(), lse=(lse2 / l2e).squeeze(-1).numpy(), dq=_bf(torch.tensor(dq)).numpy(),
                 dk=_bf(torch.tensor(dk)).numpy(), dv=_bf(dv).numpy())

@@ -8,7 +8,7 @@ import torch
 import block_causal_attention_gqa_b200 as bca
 import workloads
 from oracle import bca_oracle as orc
-from tests._helpers import assert_close, rel_l2, to_np
+from tests._helpers import assert_close, assert_lse_close, grad_bound, rel_l2, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -48,9 +48,9 @@ def test_rope_forward_and_backward_all_rows(name):
     ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
                        inp["gamma_k"], kv_range=w.kv_range, rope_q=rq, rope_k=rk)
     assert_close(f"{name} out", to_np(out), ref["out"])
-    assert_close(f"{name} lse", to_np(lse), ref["lse"])
+    assert_lse_close(f"{name} lse", to_np(lse), ref["lse"])
     for nm, got in (("dq", dq), ("dk", dk), ("dv", dv)):
-        e, r = assert_close(f"{name} {nm}", to_np(got), ref[nm], max_abs=2e-2)
+        e, r = assert_close(f"{name} {nm}", to_np(got), ref[nm], max_abs=grad_bound(name))
         print(f"{name} {nm}: max abs {e:.2e} rel L2 {r:.2e}")
     # sums over batch, tokens and heads (dgamma) or batch and heads (angles): relative L2 only
     for nm, got in (("dgamma_q", dgq), ("dgamma_k", dgk), ("drope_q", drq), ("drope_k", drk)):
@@ -100,7 +100,7 @@ def test_rope_full_size_sampled_rows():
     o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
                                     inp["gamma_k"], rows, rope_q=inp["rope_q"], rope_k=inp["rope_k"])
     assert_close("model46k_rope out rows", to_np(out.cpu()[:, idx]), o_ref)
-    assert_close("model46k_rope lse rows", to_np(lse.cpu()[:, :, idx]), l_ref)
+    assert_lse_close("model46k_rope lse rows", to_np(lse.cpu()[:, :, idx]), l_ref)
     ref = orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
                             inp["gamma_k"], q_rows=rows[:512], rope_q=inp["rope_q"], rope_k=inp["rope_k"])
     assert_close("model46k_rope dq rows", to_np(dq.cpu()[:, torch.as_tensor(rows[:512])]), ref["dq"])

@@ -51,6 +51,8 @@ class Workload:
     kv_range: int = 0            # KV range in chunks (0 = every earlier chunk); MAGI-1 §2.4.4, Fig. 12
     rope: bool = False           # rotary angles for q and k (3D positions, see rope_angles)
     deterministic: bool = False  # backward with every sum in a fixed order (same bits on every call)
+    shard_rank: int = 0          # with shard_world > 1: this workload is kv heads [r*Hkv, (r+1)*Hkv) (and
+    shard_world: int = 1         # their query groups) of a problem with shard_world times the heads
 
     @property
     def seqlen_q(self) -> int:
@@ -89,6 +91,10 @@ WORKLOADS = {
     # long context: 32 chunks x 8192 tokens, GQA 16/2, LogNormal per-token q/k scales.
     "long262k": Workload("long262k", 1, uniform_offsets(32, 8192), uniform_offsets(32, 8192),
                          16, 2, 128, seed=4, backward=True, token_scale=True),
+    # a quarter of long262k (8 chunks of 8192 tokens, same heads and value recipe): its launches fit an
+    # ncu capture, and long262k's DRAM traffic per launch is scaled from it by the units processed
+    "long65k": Workload("long65k", 1, uniform_offsets(8, 8192), uniform_offsets(8, 8192),
+                        16, 2, 128, seed=4, backward=True, token_scale=True),
     # long context with a KV range of 8 chunks (MAGI-1 §2.4.4 and §2.6: each chunk limited to
     # the preceding content, KV range 8 for long videos), otherwise as long262k.
     "window262k": Workload("window262k", 1, uniform_offsets(32, 8192), uniform_offsets(32, 8192),
@@ -111,7 +117,7 @@ WORKLOADS = {
 }
 
 ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k", "model46k_rope",
-         "model46k_det", "train4k_det"]
+         "model46k_det", "train4k_det", "long65k"]
 
 
 def workload(name_or_index) -> Workload:
@@ -125,13 +131,17 @@ def shard_heads(w: Workload, world: int, rank: int) -> Workload:
     group of query heads) are split over `world` ranks: the same chunks and
     head_dim with heads_kv / world kv heads and heads_q / world query heads.
     Each kv head's attention is independent of the others, so the shards need
-    no exchange.  Each rank draws its own inputs (seed + rank)."""
+    no exchange.  Every rank draws the whole problem's inputs (same seed) and
+    keeps its own contiguous heads (make_inputs), so the shards' results put
+    together are the unsharded result."""
     if world < 1 or not 0 <= rank < world:
         raise ValueError(f"rank {rank} of {world}")
+    if w.shard_world != 1:
+        raise ValueError(f"{w.name} is already a shard")
     if w.heads_kv % world != 0:
         raise ValueError(f"{w.name}: {w.heads_kv} kv heads do not split over {world} ranks")
     return dataclasses.replace(w, name=f"{w.name}[heads {rank}/{world}]", heads_q=w.heads_q // world,
-                               heads_kv=w.heads_kv // world, seed=w.seed + rank)
+                               heads_kv=w.heads_kv // world, shard_rank=rank, shard_world=world)
 
 
 def custom(name: str, batch: int, q_chunks: Sequence[int], kv_chunks: Optional[Sequence[int]],
@@ -175,7 +185,9 @@ def make_inputs(w: Workload, device: str = "cpu", with_grad_out: Optional[bool] 
     gen_dev = "cuda" if device.startswith("cuda") else "cpu"
     g = torch.Generator(device=gen_dev)
     g.manual_seed(w.seed)
-    B, Sq, Skv, Hq, Hkv, D = w.batch, w.seqlen_q, w.seqlen_kv, w.heads_q, w.heads_kv, w.head_dim
+    n, r = w.shard_world, w.shard_rank
+    # a head shard draws the whole problem (n times the heads) and keeps its heads
+    B, Sq, Skv, Hq, Hkv, D = w.batch, w.seqlen_q, w.seqlen_kv, w.heads_q * n, w.heads_kv * n, w.head_dim
     kw = dict(generator=g, device=gen_dev, dtype=torch.float32)
     q = torch.randn(B, Sq, Hq, D, **kw)
     k = torch.randn(B, Skv, Hkv, D, **kw)
@@ -193,6 +205,13 @@ def make_inputs(w: Workload, device: str = "cpu", with_grad_out: Optional[bool] 
         sk = torch.exp(0.5 * torch.randn(B, Skv, 1, 1, **kw))
         q.mul_(sq)
         k.mul_(sk)
+    if n > 1:
+        hq, hk = w.heads_q, w.heads_kv
+        q = q[:, :, r * hq:(r + 1) * hq].contiguous()
+        k = k[:, :, r * hk:(r + 1) * hk].contiguous()
+        v = v[:, :, r * hk:(r + 1) * hk].contiguous()
+        if dout is not None:
+            dout = dout[:, :, r * hq:(r + 1) * hq].contiguous()
     out = dict(gamma_q=gq.float().to(device), gamma_k=gk.float().to(device))
     if w.input_dtype == "fp32":
         out.update(q_f32=q.to(device), k_f32=k.to(device), v_f32=v.to(device))

@@ -39,7 +39,12 @@ folding of scales):
    dq~ = scale dS k~, dk~ = scale dS^T q~, summed over each query-head group
    for k and v, then the RMSNorm Jacobian back to the raw q and k, and the
    gain gradients dgamma = sum over (batch, token, head) of dx~ * x_hat.
-6. Optional rotary position embedding before the norm (MAGI-1 §2.2.2 and the
+6. Optional packed samples and a last global block (MAGI-1 §4.1.2 and
+   Figure 15 (f), (g); App. B.1, Figure 23): several samples packed into one sequence
+   attend only within themselves, and the last kv chunks may form a global
+   block that every query sees and whose queries see every key (see
+   ``block_causal_mask``).
+7. Optional rotary position embedding before the norm (MAGI-1 §2.2.2 and the
    notes' DiT-block sketch: learnable 3D RoPE applied to q and k, then
    QK-norm).  The pages give no formula; the reading here: per token an angle
    for each of the D/2 feature pairs (i, i + D/2), shared by all heads and
@@ -144,12 +149,23 @@ def matched_kv_chunk(q_chunk, n_q_chunks, n_kv_chunks):
     return n_kv_chunks - n_q_chunks + np.asarray(q_chunk)
 
 
-def block_causal_mask(q_offsets, kv_offsets, rows=None, kv_range=0):
+def block_causal_mask(q_offsets, kv_offsets, rows=None, kv_range=0, samples=None, n_global=0):
     """Boolean mask M[i, j]: query token i may attend key token j.
 
     Built token by token from chunk ids, not from tile arithmetic.  With
     ``kv_range`` R > 0, key chunks more than R - 1 chunks before the query's
-    own kv chunk are masked as well."""
+    own kv chunk are masked as well.
+
+    Packed samples (MAGI-1 §4.1.2, Figure 15 (f), "varlen block-causal"):
+    ``samples`` = cumulative kv-chunk counts [0, ..., n_kv] of the samples
+    packed one after another into the sequence; a query token sees only keys
+    of its own sample (the sample of its matched kv chunk).  None = one sample.
+
+    Global block (Figure 15 (g), a varlen block-causal mask with a global
+    block; App. B.1, Figure 23, a last global block): the last ``n_global`` kv
+    chunks.  Every query token sees
+    its keys, and the query tokens matched to it see every key.  Both rules
+    hold whatever the sample or the KV range."""
     q_offsets = np.asarray(q_offsets)
     kv_offsets = np.asarray(kv_offsets)
     nq, nkv = len(q_offsets) - 1, len(kv_offsets) - 1
@@ -161,6 +177,13 @@ def block_causal_mask(q_offsets, kv_offsets, rows=None, kv_range=0):
     m = ck[None, :] <= own
     if kv_range and kv_range > 0:
         m &= ck[None, :] >= own - (int(kv_range) - 1)
+    if samples is not None:
+        sid = chunk_of(np.asarray(samples), nkv)          # sample of every kv chunk
+        m &= sid[ck][None, :] == sid[own]
+    if n_global and n_global > 0:
+        first = nkv - int(n_global)
+        m |= ck[None, :] >= first                          # everyone sees the global keys
+        m |= own >= first                                  # global queries see every key
     return m
 
 
@@ -196,7 +219,7 @@ def _attend_rows(qn_rows, kn, vv, mask_rows, scale):
 
 def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=None,
                  batches=None, scale=None, eps=DEFAULT_EPS, block=None, kv_range=0, rope_q=None,
-                 rope_k=None):
+                 rope_k=None, samples=None, n_global=0):
     """Forward on a subset of query rows.
 
     ``rows`` is an int array of query-token indices; ``heads`` / ``batches``
@@ -229,7 +252,8 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
             for r0 in range(0, len(rows), block):
                 rr = rows[r0:r0 + block]
                 qn = rms_norm(qsel[b, r0:r0 + block, h, :], gamma_q, eps)
-                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range, samples=samples,
+                                         n_global=n_global)
                 o, ls, _ = _attend_rows(qn, kn, vv, mask, scale)
                 out[bi, r0:r0 + len(rr), hi, :] = o
                 lse[bi, hi, r0:r0 + len(rr)] = ls
@@ -237,16 +261,16 @@ def forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, rows, heads=N
 
 
 def forward(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None, eps=DEFAULT_EPS, kv_range=0,
-            rope_q=None, rope_k=None):
+            rope_q=None, rope_k=None, samples=None, n_global=0):
     """Full forward.  Returns (out [B, Sq, Hq, D], lse [B, Hq, Sq]), float64."""
     Sq = q.shape[1]
     return forward_rows(q, k, v, q_offsets, kv_offsets, gamma_q, gamma_k,
                         rows=np.arange(Sq), scale=scale, eps=eps, kv_range=kv_range, rope_q=rope_q,
-                        rope_k=rope_k)
+                        rope_k=rope_k, samples=samples, n_global=n_global)
 
 
 def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
-             eps=DEFAULT_EPS, kv_range=0, rope_q=None, rope_k=None):
+             eps=DEFAULT_EPS, kv_range=0, rope_q=None, rope_k=None, samples=None, n_global=0):
     """Full analytic backward in float64.
 
     Returns dict(dq, dk, dv, dgamma_q, dgamma_k, out, lse) and, with rotary
@@ -263,7 +287,7 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
     B, Sq, Hq, D, Skv, Hkv = _check(q, k, v, q_offsets, kv_offsets)
     scale = 1.0 / np.sqrt(D) if not scale else float(scale)
     group = Hq // Hkv
-    mask = block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range)
+    mask = block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range, samples=samples, n_global=n_global)
     dqn = np.zeros_like(q)
     dkn = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -303,7 +327,7 @@ def backward(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, scale=None,
 
 def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows=None,
                   kv_rows=None, kv_heads=None, batches=None, scale=None, eps=DEFAULT_EPS,
-                  block=None, kv_range=0, rope_q=None, rope_k=None):
+                  block=None, kv_range=0, rope_q=None, rope_k=None, samples=None, n_global=0):
     """Exact backward on chosen rows, without a full backward.
 
     * dq of query rows ``q_rows`` (all heads): needs only those rows' P, dP
@@ -343,7 +367,8 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
             kn_all = rms_norm(rope(k[b], rk), gk, eps)
             for r0 in range(0, len(q_rows), block):
                 rr = q_rows[r0:r0 + block]
-                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
+                mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range, samples=samples,
+                                         n_global=n_global)
                 dqn = np.zeros((len(rr), Hq, D))
                 for h in range(Hq):
                     hk = h // group
@@ -365,7 +390,9 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
         dk = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         dv = np.zeros((len(batches), len(kv_rows), len(kv_heads), D))
         # every query row that sees at least one of the requested keys
-        seeing = np.nonzero(block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range)[:, kv_rows].any(axis=1))[0]
+        full_mask = block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range, samples=samples, n_global=n_global)
+        seeing = np.nonzero(full_mask[:, kv_rows].any(axis=1))[0]
+        del full_mask
         qsel, dsel = take(q, seeing), take(dout, seeing)
         qsel = rope(qsel, None if rope_q is None else _f64(rope_q)[seeing])
         for bi, b in enumerate(batches):
@@ -379,7 +406,8 @@ def backward_rows(q, k, v, dout, q_offsets, kv_offsets, gamma_q, gamma_k, q_rows
                     for r0 in range(0, len(seeing), block):
                         rr = seeing[r0:r0 + block]
                         qn = rms_norm(qsel[b, r0:r0 + block, h, :], gq, eps)
-                        mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range)
+                        mask = block_causal_mask(q_offsets, kv_offsets, rows=rr, kv_range=kv_range,
+                                                 samples=samples, n_global=n_global)
                         o, _, p = _attend_rows(qn, kn, vv, mask, scale)
                         g = dsel[b, r0:r0 + block, h, :]
                         delta = np.sum(g * o, axis=1, keepdims=True)

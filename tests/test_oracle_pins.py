@@ -48,11 +48,14 @@ def read_mask_fixture(name):
 # ---------------------------------------------------------------- the mask
 
 @pytest.mark.parametrize("name", ["mask_train_2_1_3.txt", "mask_stream_2of3.txt",
-                                  "mask_kvrange2_train_2_1_2_1.txt", "mask_kvrange3_stream_2of4.txt"])
+                                  "mask_kvrange2_train_2_1_2_1.txt", "mask_kvrange3_stream_2of4.txt",
+                                  "mask_packed_train_2_1_2_1_2.txt", "mask_packed_global_train_2_1_2_1_2.txt",
+                                  "mask_packed_stream_2of4.txt", "mask_packed_kvrange2_global_1x5.txt"])
 def test_mask_matches_hand_written_fixture(name):
     meta, want = read_mask_fixture(name)
     got = orc.block_causal_mask(offs(meta["q_chunks"]), offs(meta["kv_chunks"]),
-                                kv_range=meta.get("kv_range", [0])[0])
+                                kv_range=meta.get("kv_range", [0])[0], samples=meta.get("samples"),
+                                n_global=meta.get("n_global", [0])[0])
     assert got.shape == want.shape
     assert np.array_equal(got, want)
 
@@ -651,3 +654,148 @@ def test_rope_backward_matches_torch_autograd_fp64():
     for t, name in zip(T, ["dq", "dk", "dv", "dgamma_q", "dgamma_k", "drope_q", "drope_k"]):
         np.testing.assert_allclose(g[name], t.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
     np.testing.assert_allclose(g["out"], o.detach().numpy(), rtol=0, atol=1e-12)
+
+
+
+# ------------------------------------------- packed samples and the global block
+
+def loop_mask(q_lens, kv_lens, samples, n_global, kv_range=0):
+    """Token-by-token mask from the rules as stated (independent of the
+    oracle's vectorised construction): same sample and not a later chunk (and
+    within the KV range), or a global key, or a global query."""
+    nq, nkv = len(q_lens), len(kv_lens)
+    kv_chunk = [c for c, n in enumerate(kv_lens) for _ in range(n)]
+    q_own = [nkv - nq + c for c, n in enumerate(q_lens) for _ in range(n)]
+    sample_of_chunk = {}
+    for sidx in range(len(samples) - 1):
+        for c in range(samples[sidx], samples[sidx + 1]):
+            sample_of_chunk[c] = sidx
+    first_global = nkv - n_global
+    m = np.zeros((len(q_own), len(kv_chunk)), dtype=bool)
+    for i, own in enumerate(q_own):
+        for j, ck in enumerate(kv_chunk):
+            same = sample_of_chunk[ck] == sample_of_chunk[own]
+            in_range = ck <= own and (kv_range <= 0 or ck >= own - kv_range + 1)
+            m[i, j] = (same and in_range) or ck >= first_global or own >= first_global
+    return m
+
+
+def test_packed_samples_equal_each_sample_alone():
+    """Samples packed into one sequence give, row for row, what each sample
+    gives on its own (forward and backward), with ragged chunks and GQA."""
+    rng = np.random.default_rng(71)
+    sample_chunks = [[5, 3], [4], [2, 6, 3]]
+    lens = [n for sc in sample_chunks for n in sc]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, lens, lens, 4, 2, 8)
+    do = rng.standard_normal(q.shape)
+    samples = offs([len(sc) for sc in sample_chunks])
+    packed = orc.backward(q, k, v, do, qo, ko, gq, gk, samples=samples)
+    t0 = 0
+    dg = {"dgamma_q": 0.0, "dgamma_k": 0.0}
+    for sc in sample_chunks:
+        sl = slice(t0, t0 + sum(sc))
+        o = offs(sc)
+        alone = orc.backward(q[:, sl], k[:, sl], v[:, sl], do[:, sl], o, o, gq, gk)
+        for nm in ("out", "dq", "dk", "dv"):
+            np.testing.assert_allclose(packed[nm][:, sl], alone[nm], rtol=0, atol=1e-12, err_msg=nm)
+        np.testing.assert_allclose(packed["lse"][:, :, sl], alone["lse"], rtol=0, atol=1e-12)
+        for nm in dg:
+            dg[nm] = dg[nm] + alone[nm]
+        t0 += sum(sc)
+    for nm in dg:
+        np.testing.assert_allclose(packed[nm], dg[nm], rtol=0, atol=1e-11, err_msg=nm)
+
+
+@pytest.mark.parametrize("kv_range", [0, 2])
+def test_packed_global_block_matches_torch_sdpa_with_a_loop_mask(kv_range):
+    rng = np.random.default_rng(72)
+    lens = [3, 5, 2, 4, 6, 3]
+    samples = [0, 2, 3, 6]            # chunks 0-1 | 2 | 3-5; chunk 5 is the global block
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 2, lens, lens, 6, 2, 16)
+    o, _ = orc.forward(q, k, v, qo, ko, gq, gk, kv_range=kv_range, samples=samples, n_global=1)
+    mask = torch.tensor(loop_mask(lens, lens, samples, 1, kv_range))
+    np.testing.assert_allclose(o, torch_reference(q, k, v, qo, ko, gq, gk, mask=mask), rtol=0, atol=1e-12)
+
+
+def test_packed_streaming_layout_matches_torch_sdpa_with_a_loop_mask():
+    rng = np.random.default_rng(73)
+    kv_lens, q_lens = [4, 3, 5, 2, 6], [2, 6]          # the query chunks are kv chunks 3 and 4
+    samples = [0, 2, 5]                                 # kv chunks 0-1 | 2-4
+    for n_global in (0, 1):
+        q, k, v, gq, gk, qo, ko = rand_case(rng, 1, q_lens, kv_lens, 4, 1, 8)
+        o, _ = orc.forward(q, k, v, qo, ko, gq, gk, samples=samples, n_global=n_global)
+        mask = torch.tensor(loop_mask(q_lens, kv_lens, samples, n_global))
+        np.testing.assert_allclose(o, torch_reference(q, k, v, qo, ko, gq, gk, mask=mask), rtol=0, atol=1e-12)
+
+
+def test_other_samples_kv_does_not_change_a_sample_and_the_global_block_does():
+    rng = np.random.default_rng(74)
+    lens = [4, 4, 3, 5, 2]
+    samples = [0, 2, 5]                                 # chunks 0-1 | 2-4
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 2, 1, 8)
+    o0, _ = orc.forward(q, k, v, qo, ko, gq, gk, samples=samples)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :8] = rng.standard_normal(k2[:, :8].shape)      # sample 0's keys and values
+    v2[:, :8] = rng.standard_normal(v2[:, :8].shape)
+    o1, _ = orc.forward(q, k2, v2, qo, ko, gq, gk, samples=samples)
+    assert np.array_equal(o0[:, 8:], o1[:, 8:])            # sample 1 untouched
+    assert not np.allclose(o0[:, :8], o1[:, :8])
+    # with the last chunk global, changing its values changes every row
+    g0, _ = orc.forward(q, k, v, qo, ko, gq, gk, samples=samples, n_global=1)
+    v3 = v.copy()
+    v3[:, 16:] += 1.0
+    g1, _ = orc.forward(q, k, v3, qo, ko, gq, gk, samples=samples, n_global=1)
+    assert np.all(np.abs(g1 - g0).max(axis=(0, 2, 3)) > 1e-6)
+
+
+def test_one_sample_and_no_global_block_is_the_plain_mask():
+    rng = np.random.default_rng(75)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, [3, 5, 4], [3, 5, 4], 2, 1, 8)
+    a, la = orc.forward(q, k, v, qo, ko, gq, gk)
+    b, lb = orc.forward(q, k, v, qo, ko, gq, gk, samples=[0, 3], n_global=0)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_packed_global_backward_matches_central_finite_differences():
+    rng = np.random.default_rng(76)
+    lens = [2, 1, 2, 2]
+    samples = [0, 1, 4]
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 2, 1, 4)
+    do = rng.standard_normal(q.shape)
+    kw = dict(samples=samples, n_global=1, kv_range=2)
+    g = orc.backward(q, k, v, do, qo, ko, gq, gk, **kw)
+    params = [q, k, v, gq, gk]
+
+    def loss(pp):
+        o, _ = orc.forward(pp[0], pp[1], pp[2], qo, ko, pp[3], pp[4], **kw)
+        return float(np.sum(o * do))
+
+    h = 1e-6
+    for pi, name in enumerate(["dq", "dk", "dv", "dgamma_q", "dgamma_k"]):
+        num = np.zeros_like(params[pi])
+        it = np.nditer(params[pi], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            pp = [p.copy() for p in params]
+            pp[pi][idx] += h
+            lp = loss(pp)
+            pp[pi][idx] -= 2 * h
+            num[idx] = (lp - loss(pp)) / (2 * h)
+        np.testing.assert_allclose(g[name], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_packed_global_backward_rows_match_full_backward():
+    rng = np.random.default_rng(77)
+    lens = [5, 4, 6, 3, 4]
+    kw = dict(samples=[0, 2, 4, 5], n_global=1)
+    q, k, v, gq, gk, qo, ko = rand_case(rng, 1, lens, lens, 4, 2, 8)
+    do = rng.standard_normal(q.shape)
+    full = orc.backward(q, k, v, do, qo, ko, gq, gk, **kw)
+    rows, kv_rows = np.array([0, 6, 9, 15, 20]), np.array([2, 7, 12, 19, 21])
+    part = orc.backward_rows(q, k, v, do, qo, ko, gq, gk, q_rows=rows, kv_rows=kv_rows, **kw)
+    np.testing.assert_allclose(part["dq"][0], full["dq"][0, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dk"][0], full["dk"][0, kv_rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(part["dv"][0], full["dv"][0, kv_rows], rtol=0, atol=1e-12)
+    fo, fl = orc.forward(q, k, v, qo, ko, gq, gk, **kw)
+    po, pl = orc.forward_rows(q, k, v, qo, ko, gq, gk, rows, **kw)
+    np.testing.assert_allclose(po, fo[:, rows], rtol=0, atol=1e-12)

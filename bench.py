@@ -39,14 +39,28 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ------------------------------------------------------------------ work model
 def row_visible_keys(w):
     """Visible keys of every query row: query chunk c is kv chunk c' = n_kv - n_q + c
-    and sees kv chunks [c' - R + 1, c'] under a KV range R, else [0, c']."""
+    and sees kv chunks from the first of its sample (packed samples) and from
+    c' - R + 1 (KV range R) up to c'; plus the keys of a last global block, and
+    every key if c' belongs to that block."""
     qo, ko = w.q_offsets, w.kv_offsets
     nq, nkv = len(qo) - 1, len(ko) - 1
+    first_global = nkv - w.n_global
+    g0, skv = int(ko[first_global]), int(ko[-1])
+    sample_first = np.zeros(nkv, np.int64)
+    if w.samples is not None:
+        for i in range(len(w.samples) - 1):
+            sample_first[w.samples[i]:w.samples[i + 1]] = w.samples[i]
     n = np.empty(w.seqlen_q, np.int64)
     for c in range(nq):
         own = nkv - nq + c
-        first = max(own - w.kv_range + 1, 0) if w.kv_range > 0 else 0
-        n[qo[c]:qo[c + 1]] = ko[own + 1] - ko[first]
+        if own >= first_global:
+            n[qo[c]:qo[c + 1]] = skv
+            continue
+        first = sample_first[own]
+        if w.kv_range > 0:
+            first = max(first, own - w.kv_range + 1)
+        lo, hi = int(ko[first]), int(ko[own + 1])
+        n[qo[c]:qo[c + 1]] = (hi - lo) + (skv - g0) - max(0, min(hi, skv) - max(lo, g0))
     return n
 
 
@@ -248,19 +262,19 @@ def run_ours(args, w, world, rank, local, light=False, pass_=None, steps=None, w
     def fwd_call(q_, k_, v_, out_, lse_):
         if w.rope:
             bca.magi_bca_fwd_rope(q_, k_, v_, w.q_offsets, w.kv_offsets, gq, gk, rq, rk, out=out_, lse=lse_,
-                                  stream=stream, kv_range=w.kv_range)
+                                  stream=stream, **w.mask_kw)
         else:
             bca.magi_bca_fwd(q_, k_, v_, w.q_offsets, w.kv_offsets, gq, gk, out=out_, lse=lse_, stream=stream,
-                             kv_range=w.kv_range)
+                             **w.mask_kw)
 
     def bwd_call(q_, k_, v_, out_, do_, lse_, dq_, dk_, dv_):
         if w.rope:
             bca.magi_bca_bwd_rope(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, rq, rk, dq=dq_,
                                   dk=dk_, dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream,
-                                  kv_range=w.kv_range, deterministic=w.deterministic)
+                                  **w.mask_kw, deterministic=w.deterministic)
         else:
             bca.magi_bca_bwd(q_, k_, v_, out_, do_, lse_, w.q_offsets, w.kv_offsets, gq, gk, dq=dq_, dk=dk_,
-                             dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, kv_range=w.kv_range,
+                             dv=dv_, dgamma_q=dgq, dgamma_k=dgk, workspace=ws, stream=stream, **w.mask_kw,
                              deterministic=w.deterministic)
 
     def step(ev=None, kev=None):
@@ -508,10 +522,10 @@ def oracle_sample(w, inp, rows, do_bwd):
     from oracle import bca_oracle as orc
     rq, rk = inp.get("rope_q"), inp.get("rope_k")
     orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
-                     inp["gamma_k"], rows, batches=[0], kv_range=w.kv_range, rope_q=rq, rope_k=rk)
+                     inp["gamma_k"], rows, batches=[0], **w.mask_kw, rope_q=rq, rope_k=rk)
     if do_bwd:
         orc.backward_rows(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0], kv_range=w.kv_range,
+                          inp["gamma_q"], inp["gamma_k"], q_rows=rows, batches=[0], **w.mask_kw,
                           rope_q=rq, rope_k=rk)
 
 

@@ -19,7 +19,8 @@ from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
-__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_fwd_rope", "magi_bca_bwd_rope", "magi_bca_bwd_noalloc", "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule",
+__all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_fwd_rope", "magi_bca_bwd_rope", "magi_bca_bwd_noalloc",
+           "magi_bca_bwd_workspace_size", "magi_bca_fwd_schedule", "magi_bca_release_caches", "magi_bca_cache_bytes",
            "magi_bca_status_string", "magi_bca_last_device_status", "magi_bca_profile_events", "MagiBcaError",
            "Dims", "library",
            "library_path", "EXPORTED_SYMBOLS"]
@@ -31,7 +32,7 @@ EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",
                     "magi_bca_bwd_noalloc", "magi_bca_last_error_detail", "magi_bca_bwd_schedule",
                     "magi_bca_profile_events", "magi_bca_fwd_rope", "magi_bca_bwd_rope",
-                    "magi_bca_selftest_wait_timeout"]
+                    "magi_bca_selftest_wait_timeout", "magi_bca_release_caches", "magi_bca_cache_bytes"]
 
 
 class MagiBcaError(RuntimeError):
@@ -48,7 +49,8 @@ class Dims(ctypes.Structure):
                 ("heads_q", ctypes.c_int32), ("heads_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("n_q_chunks", ctypes.c_int32), ("n_kv_chunks", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("kv_range", ctypes.c_int32),
-                ("deterministic", ctypes.c_int32)]
+                ("deterministic", ctypes.c_int32), ("n_samples", ctypes.c_int32), ("n_global_chunks", ctypes.c_int32),
+                ("sample_chunk_offsets", ctypes.POINTER(ctypes.c_int32))]
 
 
 _lib = None
@@ -96,8 +98,25 @@ def library() -> ctypes.CDLL:
     lib.magi_bca_profile_events.restype = ctypes.c_int
     lib.magi_bca_selftest_wait_timeout.argtypes = [vp]
     lib.magi_bca_selftest_wait_timeout.restype = ctypes.c_int
+    lib.magi_bca_release_caches.argtypes = []
+    lib.magi_bca_release_caches.restype = ctypes.c_int
+    lib.magi_bca_cache_bytes.argtypes = []
+    lib.magi_bca_cache_bytes.restype = ctypes.c_size_t
     _lib = lib
     return lib
+
+
+def magi_bca_release_caches() -> None:
+    """Frees the library's cached schedules and key buffers (synchronises the
+    devices that hold any)."""
+    st = library().magi_bca_release_caches()
+    if st != 0:
+        raise MagiBcaError(st, "magi_bca_release_caches")
+
+
+def magi_bca_cache_bytes() -> int:
+    """Device bytes held by the library's caches."""
+    return int(library().magi_bca_cache_bytes())
 
 
 def magi_bca_status_string(status: int) -> str:
@@ -150,9 +169,20 @@ def _i32p(a: np.ndarray):
 
 
 def make_dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-              softmax_scale=0.0, rms_eps=1e-6, kv_range=0, deterministic=False) -> Dims:
-    return Dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
-                float(softmax_scale), float(rms_eps), int(kv_range), int(bool(deterministic)))
+              softmax_scale=0.0, rms_eps=1e-6, kv_range=0, deterministic=False, samples=None,
+              n_global=0) -> Dims:
+    """The dims struct.  samples: cumulative kv-chunk counts [0, ..., n_kv_chunks]
+    of packed samples (None: one sample); n_global: the last n_global kv chunks
+    form a global block.  The struct keeps a reference to the samples array it
+    points at."""
+    d = Dims(batch, seqlen_q, seqlen_kv, heads_q, heads_kv, head_dim, n_q_chunks, n_kv_chunks,
+             float(softmax_scale), float(rms_eps), int(kv_range), int(bool(deterministic)), 0, int(n_global), None)
+    if samples is not None:
+        so = _offsets(samples)
+        d.n_samples = len(so) - 1
+        d.sample_chunk_offsets = _i32p(so)
+        d.keep_samples = so
+    return d
 
 
 def _check_bf16(name, t, shape=None):
@@ -183,7 +213,7 @@ def _stream_handle(stream, device):
 
 
 def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps, stream,
-         want_lse, kv_range, rope=None):
+         want_lse, kv_range, rope=None, samples=None, n_global=0):
     import torch
     _check_bf16("q", q)
     B, Sq, Hq, D = q.shape
@@ -201,7 +231,8 @@ def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse,
         lse = torch.empty(B, Hq, Sq, device=q.device, dtype=torch.float32)
     if lse is not None:
         _check_f32("lse", lse, (B, Hq, Sq))
-    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range)
+    dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
+                     samples=samples, n_global=n_global)
     ptr = lambda t: t.data_ptr() if t is not None else None
     with torch.cuda.device(q.device):
         if rope is None:
@@ -225,20 +256,22 @@ def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse,
 
 def magi_bca_fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out=None, lse=None,
                  softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, want_lse: bool = True,
-                 kv_range: int = 0):
+                 kv_range: int = 0, samples=None, n_global: int = 0):
     """Forward.  q [B,Sq,Hq,D], k/v [B,Skv,Hkv,D] bf16; gammas fp32 [D];
-    offsets: host int arrays of chunk boundaries.  Returns (out, lse)."""
+    offsets: host int arrays of chunk boundaries; samples: kv-chunk offsets of
+    packed samples (None: one); n_global: trailing kv chunks that form a global
+    block.  Returns (out, lse)."""
     return _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps,
-                stream, want_lse, kv_range)
+                stream, want_lse, kv_range, samples=samples, n_global=n_global)
 
 
 def magi_bca_fwd_rope(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, rope_q, rope_k, out=None,
                       lse=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
-                      want_lse: bool = True, kv_range: int = 0):
+                      want_lse: bool = True, kv_range: int = 0, samples=None, n_global: int = 0):
     """Forward with rotary angles (fp32 [Sq, D/2] / [Skv, D/2] per token, or
     None) applied to q and k before the norm.  Returns (out, lse)."""
     return _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse, softmax_scale, rms_eps,
-                stream, want_lse, kv_range, rope=(rope_q, rope_k))
+                stream, want_lse, kv_range, rope=(rope_q, rope_k), samples=samples, n_global=n_global)
 
 
 def magi_bca_bwd_workspace_size(dims: Dims) -> int:
@@ -247,7 +280,7 @@ def magi_bca_bwd_workspace_size(dims: Dims) -> int:
 
 def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv, dgamma_q,
          dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range, rope=None,
-         deterministic=False):
+         deterministic=False, samples=None, n_global=0):
     """Shared marshalling of magi_bca_bwd and (rope = (rope_q, rope_k, drope_q,
     drope_k)) magi_bca_bwd_rope."""
     import torch
@@ -263,7 +296,7 @@ def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, ga
     _check_f32("gamma_k", gamma_k, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
-                     deterministic)
+                     deterministic, samples=samples, n_global=n_global)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -297,20 +330,20 @@ def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, ga
 def magi_bca_bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                  dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None, want_dgamma: bool = True,
                  workspace=None, softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None,
-                 kv_range: int = 0, deterministic: bool = False):
+                 kv_range: int = 0, deterministic: bool = False, samples=None, n_global: int = 0):
     """Backward.  Returns (dq, dk, dv, dgamma_q, dgamma_k); dq/dk are with
     respect to the raw (pre-norm) q and k.  deterministic=True sums every
     gradient in a fixed order (same bits on every call; more tensor work)."""
     return _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
                 dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range,
-                deterministic=deterministic)
+                deterministic=deterministic, samples=samples, n_global=n_global)
 
 
 def magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                       rope_q, rope_k, dq=None, dk=None, dv=None, dgamma_q=None, dgamma_k=None,
                       want_dgamma: bool = True, want_drope: bool = True, workspace=None,
                       softmax_scale: float = 0.0, rms_eps: float = 1e-6, stream=None, kv_range: int = 0,
-                      deterministic: bool = False):
+                      deterministic: bool = False, samples=None, n_global: int = 0):
     """Backward of magi_bca_fwd_rope.  Returns (dq, dk, dv, dgamma_q, dgamma_k,
     drope_q, drope_k); dq/dk are with respect to the raw (pre-rotation,
     pre-norm) q and k; drope_* (fp32 [seqlen, D/2], summed over batch and
@@ -328,13 +361,14 @@ def magi_bca_bwd_rope(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets
             drk = torch.empty_like(rope_k)
     res = _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, dq, dk, dv,
                dgamma_q, dgamma_k, want_dgamma, workspace, softmax_scale, rms_eps, stream, kv_range,
-               rope=(rope_q, rope_k, drq, drk), deterministic=deterministic)
+               rope=(rope_q, rope_k, drq, drk), deterministic=deterministic, samples=samples, n_global=n_global)
     return res + (drq, drk)
 
 
 def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k,
                          dq, dk, dv, dgamma_q=None, dgamma_k=None, softmax_scale: float = 0.0,
-                         rms_eps: float = 1e-6, stream=None, kv_range: int = 0, deterministic: bool = False):
+                         rms_eps: float = 1e-6, stream=None, kv_range: int = 0, deterministic: bool = False,
+                         samples=None, n_global: int = 0):
     """Backward through the allocation-free entry point.
 
     For callers that cannot allocate device memory or hand the library a
@@ -357,7 +391,7 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
             _check_f32(nm, t, (D,))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
-                     deterministic)
+                     deterministic, samples=samples, n_global=n_global)
     import torch
     with torch.cuda.device(q.device):
         st = library().magi_bca_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -372,11 +406,11 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
 
 
 def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
-                          kv_range=0) -> np.ndarray:
+                          kv_range=0, samples=None, n_global=0) -> np.ndarray:
     """Host-only: the forward's work units as an int32 array [n_units, 12]."""
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1,
-                     kv_range=kv_range)
+                     kv_range=kv_range, samples=samples, n_global=n_global)
     lib = library()
     n = lib.magi_bca_fwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), None, 0)
     if n < 0:
@@ -388,17 +422,17 @@ def magi_bca_fwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, hea
 
 
 def magi_bca_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, batch, heads_q, heads_kv, head_dim,
-                          num_sms=148, kv_range=0, deterministic=False) -> np.ndarray:
-    """Host-only: the backward's work units as an int32 array [n_units, 8]
+                          num_sms=148, kv_range=0, deterministic=False, samples=None, n_global=0) -> np.ndarray:
+    """Host-only: the backward's work units as an int32 array [n_units, 12]
     (deterministic=True: one unit per kv tile)."""
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(batch, int(qo[-1]), int(ko[-1]), heads_q, heads_kv, head_dim, len(qo) - 1, len(ko) - 1,
-                     kv_range=kv_range, deterministic=deterministic)
+                     kv_range=kv_range, deterministic=deterministic, samples=samples, n_global=n_global)
     lib = library()
     n = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, None, 0)
     if n < 0:
         raise MagiBcaError(int(n), "magi_bca_bwd_schedule")
-    buf = np.zeros((max(n, 1), 8), dtype=np.int32)
+    buf = np.zeros((max(n, 1), 12), dtype=np.int32)
     n2 = lib.magi_bca_bwd_schedule(_i32p(qo), _i32p(ko), ctypes.byref(dims), num_sms, _i32p(buf), n)
     assert n2 == n
     return buf[:n]

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -79,29 +80,109 @@ struct DeviceState {
   bool supported = false;
 };
 
+// The library's own device memory: tile schedules (per device, shape and
+// mask) and the forward's normalised-key buffers (per device and stream).
+// Both are bounded: at most kScheduleCacheEntries schedules per device (least
+// recently used evicted), and one key buffer per stream that grows to the
+// largest shape seen.  New memory comes from cudaMallocAsync on the caller's
+// stream and schedules are uploaded with cudaMemcpyAsync from pinned staging,
+// so no call waits for the device.  Entries and buffers used while a stream
+// was being captured are kept until magi_bca_release_caches(): a graph holds
+// their addresses.
+constexpr int kScheduleCacheEntries = 64;
+
 struct ScheduleEntry {
-  int32_t* dev = nullptr;  // units, then q offsets, then kv offsets
+  int32_t* dev = nullptr;  // units, then the mask blob (query offsets, lo, hi)
+  size_t bytes = 0;
+  int device = 0;
   int n_units = 0;
+  MaskSpec mask;           // its scalars go into the kernels' MaskArgs
+  uint64_t last_use = 0;   // LRU clock
+  int refs = 0;            // calls between lookup and launch
+  bool pinned = false;     // used under stream capture: kept until release
+  std::vector<cudaStream_t> streams;  // every stream that has used it
+};
+
+struct KnormBuffer {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+  bool pinned = false;     // used under stream capture
+};
+
+// Pinned staging of a schedule upload, freed once its copy has completed.
+struct Staging {
+  void* host;
+  cudaEvent_t done;
 };
 
 std::map<int, DeviceState> g_devices;
 std::map<std::vector<int32_t>, ScheduleEntry> g_schedules;
-// Normalised-key buffers of the forward, one per (device, stream, bytes), so
-// calls on different streams never share one.
-std::map<std::tuple<int, uintptr_t, size_t>, void*> g_knorm_bufs;
+std::map<std::pair<int, uintptr_t>, KnormBuffer> g_knorm_bufs;
+std::vector<void*> g_retired;     // device buffers replaced while pinned (freed on release)
+std::vector<Staging> g_staging;
+uint64_t g_clock = 0;
+
+bool capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  return cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
+}
+
+// Frees the staging of uploads that have completed (caller holds g_mutex).
+void reap_staging() {
+  for (size_t i = 0; i < g_staging.size();) {
+    if (cudaEventQuery(g_staging[i].done) == cudaSuccess) {
+      cudaFreeHost(g_staging[i].host);
+      cudaEventDestroy(g_staging[i].done);
+      g_staging[i] = g_staging.back();
+      g_staging.pop_back();
+    } else {
+      ++i;
+    }
+  }
+}
+
+// Frees `ptr` in the order of `stream` after everything already enqueued on
+// `users` (caller holds g_mutex, device current).
+void free_after(void* ptr, const std::vector<cudaStream_t>& users, cudaStream_t stream) {
+  bool waited = true;
+  for (cudaStream_t u : users) {
+    if (u == stream) continue;
+    cudaEvent_t ev;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      waited = false;
+      continue;
+    }
+    if (cudaEventRecord(ev, u) != cudaSuccess || cudaStreamWaitEvent(stream, ev, 0) != cudaSuccess) waited = false;
+    cudaEventDestroy(ev);
+  }
+  if (!waited) cudaDeviceSynchronize();   // a user stream is gone: the slow, safe way
+  cudaFreeAsync(ptr, stream);
+}
 
 int knorm_buffer(int dev, cudaStream_t stream, size_t bytes, void** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
-  auto key = std::make_tuple(dev, reinterpret_cast<uintptr_t>(stream), bytes);
-  auto it = g_knorm_bufs.find(key);
-  if (it != g_knorm_bufs.end()) {
-    *out = it->second;
+  KnormBuffer& kb = g_knorm_bufs[std::make_pair(dev, reinterpret_cast<uintptr_t>(stream))];
+  const bool cap = capturing(stream);
+  if (kb.ptr != nullptr && kb.bytes >= bytes) {
+    kb.pinned = kb.pinned || cap;
+    *out = kb.ptr;
     return MAGI_BCA_OK;
   }
+  if (cap) {
+    std::snprintf(g_last_detail, sizeof(g_last_detail),
+                  "the first forward call for a key length must come before stream capture");
+    return MAGI_BCA_UNSUPPORTED;
+  }
+  // grow: the old buffer is only used on this stream, so a stream-ordered free is safe
+  if (kb.ptr != nullptr) {
+    if (kb.pinned) g_retired.push_back(kb.ptr); else cudaFreeAsync(kb.ptr, stream);
+  }
+  kb = KnormBuffer();
   void* ptr = nullptr;
-  const cudaError_t e = cudaMalloc(&ptr, bytes);
-  if (e != cudaSuccess) return cuda_fail("cudaMalloc (normalised-key buffer)", e);
-  g_knorm_bufs[key] = ptr;
+  const cudaError_t e = cudaMallocAsync(&ptr, bytes, stream);
+  if (e != cudaSuccess) return cuda_fail("cudaMallocAsync (normalised-key buffer)", e);
+  kb.ptr = ptr;
+  kb.bytes = bytes;
   *out = ptr;
   return MAGI_BCA_OK;
 }
@@ -128,41 +209,101 @@ int device_state(int* device_out, DeviceState** st_out) {
 }
 
 std::vector<int32_t> schedule_key(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko) {
+  const int n_samples = d.n_samples > 1 ? d.n_samples : 1;
   std::vector<int32_t> key = {dev,        kind,         d.batch,       d.seqlen_q,  d.seqlen_kv,
                               d.heads_q,  d.heads_kv,   d.head_dim,    d.n_q_chunks, d.n_kv_chunks,
-                              d.kv_range, kind == 0 ? 0 : d.deterministic};
+                              d.kv_range, kind == 0 ? 0 : d.deterministic, n_samples, d.n_global_chunks};
   key.insert(key.end(), qo, qo + d.n_q_chunks + 1);
   key.insert(key.end(), ko, ko + d.n_kv_chunks + 1);
+  if (n_samples > 1) key.insert(key.end(), d.sample_chunk_offsets, d.sample_chunk_offsets + n_samples + 1);
   return key;
 }
 
-// Returns the cached device schedule, building and uploading it on first use.
+// Returns the cached device schedule, building and uploading it (on `stream`)
+// on first use.  The entry stays referenced until release_schedule(key).
 int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, const int32_t* ko,
-                 ScheduleEntry* out) {
+                 cudaStream_t stream, ScheduleEntry* out, std::vector<int32_t>* key_out) {
   std::vector<int32_t> key = schedule_key(dev, kind, d, qo, ko);
   std::lock_guard<std::mutex> lock(g_mutex);
+  // under capture only lookups happen: event queries, allocations and frees
+  // would invalidate the capture
+  const bool cap = capturing(stream);
+  if (!cap) reap_staging();
   auto it = g_schedules.find(key);
-  if (it != g_schedules.end()) {
-    *out = it->second;
-    return MAGI_BCA_OK;
+  if (it == g_schedules.end()) {
+    if (cap) {
+      std::snprintf(g_last_detail, sizeof(g_last_detail),
+                    "the first call for a shape must come before stream capture");
+      return MAGI_BCA_UNSUPPORTED;
+    }
+    // evict the least recently used idle entries of this device beyond the limit
+    int count = 0;
+    for (auto& kv : g_schedules) count += kv.second.device == dev;
+    while (count >= kScheduleCacheEntries) {
+      auto victim = g_schedules.end();
+      for (auto v = g_schedules.begin(); v != g_schedules.end(); ++v)
+        if (v->second.device == dev && v->second.refs == 0 && !v->second.pinned &&
+            (victim == g_schedules.end() || v->second.last_use < victim->second.last_use))
+          victim = v;
+      if (victim == g_schedules.end()) break;   // everything is in use or pinned
+      free_after(victim->second.dev, victim->second.streams, stream);
+      g_schedules.erase(victim);
+      --count;
+    }
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d, sms);
+    ScheduleEntry e;
+    e.device = dev;
+    e.n_units = static_cast<int>(units.size() / (kind == 0 ? kFwdUnitInts : kUnitInts));
+    e.mask = build_mask_spec(qo, ko, d);
+    std::vector<int32_t> blob = units;
+    append_mask_blob(blob, qo, e.mask, d.n_q_chunks);
+    e.bytes = blob.size() * sizeof(int32_t);
+    Staging stg{nullptr, nullptr};
+    cudaError_t ce = cudaMallocHost(&stg.host, e.bytes);
+    if (ce != cudaSuccess) return cuda_fail("cudaMallocHost (schedule staging)", ce);
+    std::memcpy(stg.host, blob.data(), e.bytes);
+    ce = cudaMallocAsync(reinterpret_cast<void**>(&e.dev), e.bytes, stream);
+    if (ce == cudaSuccess) ce = cudaMemcpyAsync(e.dev, stg.host, e.bytes, cudaMemcpyHostToDevice, stream);
+    if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&stg.done, cudaEventDisableTiming);
+    if (ce == cudaSuccess) ce = cudaEventRecord(stg.done, stream);
+    if (ce != cudaSuccess) {
+      cudaStreamSynchronize(stream);
+      if (e.dev != nullptr) cudaFree(e.dev);
+      cudaFreeHost(stg.host);
+      return cuda_fail("schedule upload", ce);
+    }
+    g_staging.push_back(stg);
+    it = g_schedules.emplace(key, std::move(e)).first;
   }
-  int sms = 148;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  std::vector<int32_t> units = kind == 0 ? build_fwd_schedule(qo, ko, d) : build_bwd_schedule(qo, ko, d, sms);
-  ScheduleEntry e;
-  e.n_units = static_cast<int>(units.size() / (kind == 0 ? kFwdUnitInts : kUnitInts));
-  std::vector<int32_t> blob = units;
-  blob.insert(blob.end(), qo, qo + d.n_q_chunks + 1);
-  blob.insert(blob.end(), ko, ko + d.n_kv_chunks + 1);
-  if (cudaMalloc(&e.dev, blob.size() * sizeof(int32_t)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
-  if (cudaMemcpy(e.dev, blob.data(), blob.size() * sizeof(int32_t), cudaMemcpyHostToDevice) != cudaSuccess) {
-    cudaFree(e.dev);
-    return MAGI_BCA_CUDA_ERROR;
-  }
-  g_schedules[key] = e;
-  *out = e;
+  ScheduleEntry& e = it->second;
+  e.last_use = ++g_clock;
+  e.refs += 1;
+  e.pinned = e.pinned || cap;
+  if (std::find(e.streams.begin(), e.streams.end(), stream) == e.streams.end()) e.streams.push_back(stream);
+  out->dev = e.dev;
+  out->n_units = e.n_units;
+  out->mask = e.mask;
+  *key_out = std::move(key);
   return MAGI_BCA_OK;
 }
+
+// Ends the reference get_schedule took (after the launches that use it).
+void release_schedule(const std::vector<int32_t>& key) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto it = g_schedules.find(key);
+  if (it != g_schedules.end() && it->second.refs > 0) it->second.refs -= 1;
+}
+
+// Holds a schedule reference for the scope of an entry point.
+struct ScheduleRef {
+  std::vector<int32_t> key;
+  bool held = false;
+  ~ScheduleRef() {
+    if (held) release_schedule(key);
+  }
+};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -310,10 +451,12 @@ int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   DeviceState* ds;
   st = device_state(&dev, &ds);
   if (st != MAGI_BCA_OK) return st;
-  ScheduleEntry sched;
-  st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, &sched);
-  if (st != MAGI_BCA_OK) return st;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  ScheduleEntry sched;
+  ScheduleRef ref;
+  st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, cs, &sched, &ref.key);
+  if (st != MAGI_BCA_OK) return st;
+  ref.held = true;
   const int64_t kv_rows = (int64_t)d.batch * d.seqlen_kv * d.heads_kv;
   void* kn = nullptr;
   st = knorm_buffer(dev, cs, (size_t)kv_rows * d.head_dim * 2, &kn);
@@ -328,11 +471,7 @@ int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
     return MAGI_BCA_CUDA_ERROR;
   FwdParams p;
   p.units = sched.dev;
-  p.q_offsets = sched.dev + (size_t)sched.n_units * kFwdUnitInts;
-  p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
-  p.n_q_chunks = d.n_q_chunks;
-  p.n_kv_chunks = d.n_kv_chunks;
-  p.kv_range = d.kv_range;
+  p.mask = mask_args_at(sched.dev + (size_t)sched.n_units * kFwdUnitInts, sched.mask, d.n_q_chunks);
   p.rope_q = rope_q;
   p.gamma_q = gamma_q;
   p.gamma_k = gamma_k;
@@ -389,12 +528,16 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   DeviceState* ds;
   st = device_state(&dev, &ds);
   if (st != MAGI_BCA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ScheduleEntry sched, dq_sched;
-  st = get_schedule(dev, 1, d, q_chunk_offsets, kv_chunk_offsets, &sched);
+  ScheduleRef ref, dq_ref;
+  st = get_schedule(dev, 1, d, q_chunk_offsets, kv_chunk_offsets, cs, &sched, &ref.key);
   if (st != MAGI_BCA_OK) return st;
+  ref.held = true;
   if (d.deterministic) {   // the dq pass runs the forward's query-major units
-    st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, &dq_sched);
+    st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, cs, &dq_sched, &dq_ref.key);
     if (st != MAGI_BCA_OK) return st;
+    dq_ref.held = true;
   }
   uint8_t* w = static_cast<uint8_t*>(workspace);
   BwdParams p;
@@ -406,11 +549,7 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   p.gamma_q = gamma_q;
   p.gamma_k = gamma_k;
   p.units = sched.dev;
-  p.q_offsets = sched.dev + (size_t)sched.n_units * kUnitInts;
-  p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
-  p.n_q_chunks = d.n_q_chunks;
-  p.n_kv_chunks = d.n_kv_chunks;
-  p.kv_range = d.kv_range;
+  p.mask = mask_args_at(sched.dev + (size_t)sched.n_units * kUnitInts, sched.mask, d.n_q_chunks);
   p.rope_q = rope_q;
   p.rope_k = rope_k;
   p.drope_q = rope_q != nullptr ? drope_q : nullptr;
@@ -448,13 +587,56 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
       make_map(&t_qn, p.qn, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK ||
       make_map(&t_do, dout, d.batch, d.seqlen_q, d.heads_q, d.head_dim) != MAGI_BCA_OK)
     return MAGI_BCA_CUDA_ERROR;
-  cudaError_t e =
-      launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, sched.n_units,
-                 d.deterministic ? dq_sched.n_units : 0, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_bwd(t_k, t_v, t_qn, t_do, t_dq, t_dv, t_dk, p, d.head_dim, sched.n_units,
+                             d.deterministic ? dq_sched.n_units : 0, cs);
   return e == cudaSuccess ? MAGI_BCA_OK : cuda_fail("backward launch", e);
 }
 
 const char* magi_bca_last_error_detail(void) { return g_last_detail; }
+
+int magi_bca_release_caches(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int prev = -1;
+  if (cudaGetDevice(&prev) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
+  int status = MAGI_BCA_OK;
+  // every device that holds cached memory: wait for its work, then free
+  std::vector<int> devs;
+  for (auto& kv : g_schedules) devs.push_back(kv.second.device);
+  for (auto& kv : g_knorm_bufs) devs.push_back(kv.first.first);
+  if (!g_retired.empty()) devs.push_back(prev);
+  std::sort(devs.begin(), devs.end());
+  devs.erase(std::unique(devs.begin(), devs.end()), devs.end());
+  for (int dv : devs) {
+    if (cudaSetDevice(dv) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
+    for (auto& kv : g_schedules)
+      if (kv.second.device == dv && cudaFree(kv.second.dev) != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
+    for (auto& kv : g_knorm_bufs)
+      if (kv.first.first == dv && kv.second.ptr != nullptr && cudaFree(kv.second.ptr) != cudaSuccess)
+        status = MAGI_BCA_CUDA_ERROR;
+    if (dv == prev) {
+      for (void* ptr : g_retired) cudaFree(ptr);
+      g_retired.clear();
+    }
+  }
+  g_schedules.clear();
+  g_knorm_bufs.clear();
+  cudaSetDevice(prev);
+  for (Staging& stg : g_staging) {
+    cudaEventSynchronize(stg.done);
+    cudaFreeHost(stg.host);
+    cudaEventDestroy(stg.done);
+  }
+  g_staging.clear();
+  return status;
+}
+
+size_t magi_bca_cache_bytes(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  size_t total = 0;
+  for (auto& kv : g_schedules) total += kv.second.bytes;
+  for (auto& kv : g_knorm_bufs) total += kv.second.bytes;
+  return total;
+}
 
 int magi_bca_selftest_wait_timeout(void* stream) {
   int dev;

@@ -70,6 +70,7 @@
 
 #include "bca_bwd_common.cuh"
 #include "bca_kernels.h"
+#include "bca_mask.cuh"
 #include "bca_norm.cuh"
 #include "sm100.cuh"
 
@@ -259,15 +260,14 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int32_t* u = p.units + (size_t)blockIdx.x * 8;
+  const int32_t* u = p.units + (size_t)blockIdx.x * kUnitInts;
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
-  // steps [s_begin, s_end) of this kv tile; step s = (query tile s / group,
-  // head s % group of the kv head's group); query tiles below diag_end or from
-  // diag_hi_begin on (KV range) need the mask
-  const int s_begin = __ldg(u + 3), s_end = __ldg(u + 4), diag_end = __ldg(u + 5);
-  const int diag_hi_begin = __ldg(u + 6);
+  // this kv tile's steps t = 0 .. n_steps-1; absolute step s = bs.abs_step(t)
+  // is (query tile s / group, head s % group of the kv head's group), and
+  // bs.diag(t, qt) says whether the step needs the mask (bca_mask.cuh)
+  const BwdSteps bs = bwd_steps(u);
   const int group = p.heads_q / p.heads_kv;
-  const int n_steps = s_end - s_begin;
+  const int n_steps = bs.count();
   // Within each query tile the group's heads are visited from head rot on:
   // neighbouring kv tiles (which walk the same query tiles at the same time)
   // then add their G_q into different heads' dq rows, not all into the same
@@ -331,7 +331,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       for (int t = 0; t < n_steps; ++t) {
         const int st = t & 1;
         if (!mbar_wait(&bars->q_empty[st], ((t >> 1) & 1) ^ 1, p.status, kErrQEmpty)) break;
-        const int qt = (s_begin + t) / group, h = hk * group + ((s_begin + t) % group + rot) % group;
+        const int sa = bs.abs_step(t);
+        const int qt = sa / group, h = hk * group + (sa % group + rot) % group;
         // the single {-lse, -Delta} buffer: the previous step's S^T/dP^T have read it
         if (t > 0 && !mbar_wait(&bars->ld_empty, (t - 1) & 1, p.status, kErrLdEmpty)) break;
         mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2048);
@@ -346,7 +347,8 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         // warm L2 with the next step's tiles: their loads are issued only once
         // a stage frees, and then wait on memory otherwise
         if (t + 1 < n_steps) {
-          const int qt1 = (s_begin + t + 1) / group, h1 = hk * group + ((s_begin + t + 1) % group + rot) % group;
+          const int sa1 = bs.abs_step(t + 1);
+          const int qt1 = sa1 / group, h1 = hk * group + (sa1 % group + rot) % group;
           for (int box = 0; box < D / 64; ++box) {
             tma_prefetch_l2_4d(&tm_qn, box * 64, h1, qt1 * 128, b);
             tma_prefetch_l2_4d(&tm_do, box * 64, h1, qt1 * 128, b);
@@ -449,34 +451,11 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int j = threadIdx.x & 127;        // key row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int bar_id = 1 + wg;
-    // First query row that sees key n0 + j: query chunk c sees keys below
-    // kv_offsets[n_kv - n_q + c + 1], so it is the first chunk whose end exceeds the key.
-    int row_min = p.seqlen_q;
-    {
-      const int key = n0 + j;
-      if (key < p.seqlen_kv) {
-        const int shift = p.n_kv_chunks - p.n_q_chunks;
-        int lo = 0, hi = p.n_q_chunks;  // first c in [0, n_q) with kv_offsets[shift + c + 1] > key
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (__ldg(p.kv_offsets + shift + mid + 1) > key) hi = mid; else lo = mid + 1;
-        }
-        row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
-      }
-    }
-    // First query row that no longer sees key n0 + j (KV range R): query chunk
-    // c's first visible key is kv_offsets[max(0, n_kv - n_q + c - R + 1)].
-    int row_max = p.seqlen_q;
-    if (p.kv_range > 0) {
-      const int key = n0 + j;
-      const int shift = p.n_kv_chunks - p.n_q_chunks - p.kv_range + 1;
-      int lo = 0, hi = p.n_q_chunks;  // first c with a first visible key above `key`
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(p.kv_offsets + max(shift + mid, 0)) > key) hi = mid; else lo = mid + 1;
-      }
-      row_max = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
-    }
+    // Query rows that see key n0 + j: the non-global rows [row_min, row_max),
+    // every row from global_q_row on, and every row if the key is global.
+    int row_min, row_max;
+    key_rows(p.mask, n0 + j, row_min, row_max);
+    const bool key_global = n0 + j >= p.mask.global_key && n0 + j < p.seqlen_kv;
     // G_q drain: warpgroup w owns G_q columns [32 w, 32 w + 32); with D = 64 only
     // warpgroups 0 and 1 have columns.  Staging chunks are [128 rows][32 floats]
     // with the 128-byte swizzle (16 KB) in this step's Q^ and dO stage buffers.
@@ -484,9 +463,10 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
       const int st = t & 1;
-      const int qt = (s_begin + t) / group, h = hk * group + ((s_begin + t) % group + rot) % group;
+      const int sa = bs.abs_step(t);
+      const int qt = sa / group, h = hk * group + (sa % group + rot) % group;
       const int q0 = qt * 128;
-      const bool diag = qt < diag_end || qt >= diag_hi_begin;
+      const bool diag = bs.diag(t, qt);
       ok = warp_wait(&bars->s_full, t & 1, ok, p.status, kErrSFull);
       // Warpgroup w owns query columns [16w, 16w+16) of each 64-column half:
       // the first half's dK~/dV products run while the second half is computed.
@@ -517,12 +497,15 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
               dk[c >> 1] = pack_bf16x2(d0, d1);
             }
           } else {
-            // columns c < lim and c >= hi_lim cannot see key j
-            const int lim = row_min - (q0 + col0), hi_lim = row_max - (q0 + col0);
+            // columns c < lim and c >= hi_lim cannot see key j, unless they are
+            // global rows (c >= glim) or the key is global
+            const int lim = row_min - (q0 + col0), hl = row_max - (q0 + col0);
+            const int glim = key_global ? -128 : p.mask.global_q_row - (q0 + col0);
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const float p0 = c < lim || c >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c]));
-              const float p1 = c + 1 < lim || c + 1 >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]));
+              const bool v0 = (c >= lim && c < hl) || c >= glim, v1 = (c + 1 >= lim && c + 1 < hl) || c + 1 >= glim;
+              const float p0 = v0 ? fast_exp2(__uint_as_float(sr[c])) : 0.f;
+              const float p1 = v1 ? fast_exp2(__uint_as_float(sr[c + 1])) : 0.f;
               const float d0 = p0 * __uint_as_float(dpr[c]);
               const float d1 = p1 * __uint_as_float(dpr[c + 1]);
               pk[c >> 1] = pack_bf16x2(p0, p1);

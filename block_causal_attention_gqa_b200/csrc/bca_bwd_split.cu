@@ -12,6 +12,7 @@
 
 #include "bca_bwd_common.cuh"
 #include "bca_kernels.h"
+#include "bca_mask.cuh"
 #include "bca_norm.cuh"
 #include "sm100.cuh"
 
@@ -79,12 +80,11 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int32_t* u = p.units + (size_t)blockIdx.x * 8;
+  const int32_t* u = p.units + (size_t)blockIdx.x * kUnitInts;
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
-  const int s_begin = __ldg(u + 3), s_end = __ldg(u + 4), diag_end = __ldg(u + 5);
-  const int diag_hi_begin = __ldg(u + 6);
+  const BwdSteps bs = bwd_steps(u);   // steps t -> absolute steps, and which need the mask
   const int group = p.heads_q / p.heads_kv;
-  const int n_steps = s_end - s_begin;
+  const int n_steps = bs.count();
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -141,7 +141,8 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       for (int t = 0; t < n_steps; ++t) {
         const int st = t & 1;
         if (!mbar_wait(&bars->q_empty[st], ((t >> 1) & 1) ^ 1, p.status, kErrQEmpty)) break;
-        const int qt = (s_begin + t) / group, h = hk * group + (s_begin + t) % group;
+        const int sa = bs.abs_step(t);
+        const int qt = sa / group, h = hk * group + sa % group;
         mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2048);
         for (int box = 0; box < D / 64; ++box) {
           tma_load_4d(smem + L::kQn + st * L::kTile + box * 16384, &tm_qn, &bars->q_full[st], box * 64, h,
@@ -152,7 +153,8 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const float* ld_src = p.ld + (((size_t)b * p.heads_q + h) * p.seqlen_q_pad + (size_t)qt * 128) * 4;
         bulk_load(smem + L::kLd + st * L::kLdStride, ld_src, 2048, &bars->q_full[st]);
         if (t + 1 < n_steps) {
-          const int qt1 = (s_begin + t + 1) / group, h1 = hk * group + (s_begin + t + 1) % group;
+          const int sa1 = bs.abs_step(t + 1);
+          const int qt1 = sa1 / group, h1 = hk * group + sa1 % group;
           for (int box = 0; box < D / 64; ++box) {
             tma_prefetch_l2_4d(&tm_qn, box * 64, h1, qt1 * 128, b);
             tma_prefetch_l2_4d(&tm_do, box * 64, h1, qt1 * 128, b);
@@ -241,37 +243,17 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int j = threadIdx.x & 127;        // key row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int bar_id = 1 + wg;
-    // first query row that sees key n0 + j, and (KV range) the first that no longer does
-    int row_min = p.seqlen_q;
-    {
-      const int key = n0 + j;
-      if (key < p.seqlen_kv) {
-        const int shift = p.n_kv_chunks - p.n_q_chunks;
-        int lo = 0, hi = p.n_q_chunks;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (__ldg(p.kv_offsets + shift + mid + 1) > key) hi = mid; else lo = mid + 1;
-        }
-        row_min = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
-      }
-    }
-    int row_max = p.seqlen_q;
-    if (p.kv_range > 0) {
-      const int key = n0 + j;
-      const int shift = p.n_kv_chunks - p.n_q_chunks - p.kv_range + 1;
-      int lo = 0, hi = p.n_q_chunks;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(p.kv_offsets + max(shift + mid, 0)) > key) hi = mid; else lo = mid + 1;
-      }
-      row_max = lo < p.n_q_chunks ? __ldg(p.q_offsets + lo) : p.seqlen_q;
-    }
+    // query rows that see key n0 + j: the non-global rows [row_min, row_max),
+    // every row from global_q_row on, and every row if the key is global
+    int row_min, row_max;
+    key_rows(p.mask, n0 + j, row_min, row_max);
+    const bool key_global = n0 + j >= p.mask.global_key && n0 + j < p.seqlen_kv;
     const bool drains = wg * 32 < D;
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
-      const int qt = (s_begin + t) / group;
+      const int qt = bs.abs_step(t) / group;
       const int q0 = qt * 128;
-      const bool diag = qt < diag_end || qt >= diag_hi_begin;
+      const bool diag = bs.diag(t, qt);
 #pragma unroll
       for (int grp = 0; grp < 2; ++grp) {
         ok = warp_wait(grp ? &bars->s_hi : &bars->s_lo, t & 1, ok, p.status, kErrSFull);
@@ -299,11 +281,14 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
               dk[c >> 1] = pack_bf16x2(d0, d1);
             }
           } else {
-            const int lim = row_min - (q0 + col0), hi_lim = row_max - (q0 + col0);
+            // columns [lim, hl) see key j, and so do global rows (c >= glim) or all if the key is global
+            const int lim = row_min - (q0 + col0), hl = row_max - (q0 + col0);
+            const int glim = key_global ? -128 : p.mask.global_q_row - (q0 + col0);
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
-              const float p0 = c < lim || c >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c]));
-              const float p1 = c + 1 < lim || c + 1 >= hi_lim ? 0.f : fast_exp2(__uint_as_float(sr[c + 1]));
+              const bool v0 = (c >= lim && c < hl) || c >= glim, v1 = (c + 1 >= lim && c + 1 < hl) || c + 1 >= glim;
+              const float p0 = v0 ? fast_exp2(__uint_as_float(sr[c])) : 0.f;
+              const float p1 = v1 ? fast_exp2(__uint_as_float(sr[c + 1])) : 0.f;
               pk[c >> 1] = pack_bf16x2(p0, p1);
               dk[c >> 1] = pack_bf16x2(p0 * __uint_as_float(dpr[c]), p1 * __uint_as_float(dpr[c + 1]));
             }
@@ -399,16 +384,6 @@ struct DqBars {
 };
 static_assert(sizeof(DqBars) <= 16 * 8, "dq barriers exceed their slot");
 
-// chunk c with offs[c] <= row < offs[c + 1]
-__device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
-  int lo = 0, hi = n;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(offs + mid) <= row) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kDqThreads, 1)
 bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_do,
@@ -431,9 +406,8 @@ bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = __ldg(u + 0), hk = __ldg(u + 1);
   const int m0 = __ldg(u + (sub ? 5 : 3));
-  const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
-  const int t_begin = __ldg(u + 8), t_full_begin = __ldg(u + 9);
-  const int n_vis = n_tiles - t_begin;
+  const FwdTiles ft = fwd_tiles(u);   // the kv tiles this query tile visits (bca_mask.cuh)
+  const int n_vis = ft.count();
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -476,7 +450,7 @@ bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
         tma_load_4d(smem + L::kDo + box * 16384, &tm_do, &bars->q_full, box * 64, h, m0, b);
       }
       for (int j = 0; j < n_vis; ++j) {
-        const int n0 = (t_begin + j) * 128;
+        const int n0 = ft.tile(j) * 128;
         const int ks = j % kDqKStages, vs = j % kDqVStages;
         if (!mbar_wait(&bars->k_empty[ks], ((j / kDqKStages) & 1) ^ 1, p.status, kErrDqKEmpty)) break;
         mbar_arrive_expect_tx(&bars->k_full[ks], L::kTile);
@@ -572,14 +546,9 @@ bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
       nl = (bf16_lo(v.x) + bf16_hi(v.x)) + bf16_lo(v.y);
       nd = (bf16_hi(v.y) + bf16_lo(v.z)) + bf16_hi(v.z);
     }
-    // visible keys [kv_first, limit) of the row
+    // visible keys of the row: [kv_first, limit) and the global block's
     int limit = p.seqlen_kv, kv_first = 0;
-    if (row < p.seqlen_q) {
-      const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
-      limit = __ldg(p.kv_offsets + p.n_kv_chunks - p.n_q_chunks + c + 1);
-      if (p.kv_range > 0)
-        kv_first = __ldg(p.kv_offsets + max(p.n_kv_chunks - p.n_q_chunks + c - p.kv_range + 1, 0));
-    }
+    if (row < p.seqlen_q) row_keys(p.mask, row, kv_first, limit);
     const uint64_t nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
     bool ok = true;
     // Every thread runs all n_vis iterations and reaches every named barrier
@@ -600,18 +569,22 @@ bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
       named_bar_sync(bar_id, 128);
       if (r == 0 && ok) mbar_arrive(&bars->dp_free);
       if (ok) {
-        const int tile = t_begin + j;
-        const bool masked = tile < t_full_begin || tile >= n_full;
+        const int tile = ft.tile(j);
+        const bool masked = ft.masked(j, p.mask.global_key, p.seqlen_kv);
         uint32_t pk[32];
         auto sval = [&](int c) { return __uint_as_float(c < 32 ? sa[c] : sb[c - 32]); };
         auto dval = [&](int c) { return __uint_as_float(c < 32 ? da[c] : db[c - 32]); };
         if (masked) {
           const int c0 = tile * 128 + 64 * wg;
-          const int lim = limit - c0, lo = kv_first - c0;   // columns [lo, lim) are visible
+          // columns [lo, lim) and the global block's [glo, ghi) are visible
+          const int lim = limit - c0, lo = kv_first - c0;
+          const int glo = p.mask.global_key - c0, ghi = p.seqlen_kv - c0;
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
-            const float p0 = c >= lo && c < lim ? fast_exp2(sval(c) + nl) : 0.f;
-            const float p1 = c + 1 >= lo && c + 1 < lim ? fast_exp2(sval(c + 1) + nl) : 0.f;
+            const bool v0 = (c >= lo && c < lim) || (c >= glo && c < ghi);
+            const bool v1 = (c + 1 >= lo && c + 1 < lim) || (c + 1 >= glo && c + 1 < ghi);
+            const float p0 = v0 ? fast_exp2(sval(c) + nl) : 0.f;
+            const float p1 = v1 ? fast_exp2(sval(c + 1) + nl) : 0.f;
             pk[c >> 1] = pack_bf16x2(p0 * (dval(c) + nd), p1 * (dval(c + 1) + nd));
           }
         } else {

@@ -42,6 +42,7 @@
 #include <type_traits>
 
 #include "bca_kernels.h"
+#include "bca_mask.cuh"
 #include "bca_norm.cuh"
 #include "sm100.cuh"
 
@@ -86,17 +87,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, bool o
   return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ int find_chunk(const int32_t* offs, int n, int row) {
-  int lo = 0, hi = n;  // offs[lo] <= row < offs[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(offs + mid) <= row) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
-
-template <int D, bool kRope>
+// kGlobal: the schedule has units with a second range of kv tiles (a global
+// block); without it the tile of visited step j is t_begin + j and the mask
+// test is the first range's, which keeps the per-tile state (and the register
+// pressure of the softmax loop) as small as possible.
+template <int D, bool kRope, bool kGlobal>
 __global__ void __launch_bounds__(kThreads, 1)
 bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -113,12 +108,9 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int b = __ldg(u + 0), hk = __ldg(u + 1);
   const int head0 = __ldg(u + 2), head1 = __ldg(u + 4);
   const int m00 = __ldg(u + 3), m01 = __ldg(u + 5);
-  const int n_full = __ldg(u + 6), n_tiles = __ldg(u + 7);
-  // kv tiles [t_begin, n_tiles) are visited (t_begin > 0 only under a KV
-  // range); tiles below t_full_begin or from n_full on need the per-row mask.
-  // Loop indices below count visited tiles from 0: tile = t_begin + j.
-  const int t_begin = __ldg(u + 8), t_full_begin = __ldg(u + 9);
-  const int n_vis = n_tiles - t_begin;
+  const FwdTiles ft = fwd_tiles(u);
+  const int n_vis = kGlobal ? ft.count() : ft.n_tiles - ft.t_begin;
+  auto tile_of = [&](int j) { return kGlobal ? ft.tile(j) : ft.t_begin + j; };
   const int n_sub = head1 >= 0 ? 2 : 1;
 
   if (threadIdx.x == 0) {
@@ -167,12 +159,12 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_arrive_expect_tx(&bars->k_full[st], L::kTileBytes);
         for (int box = 0; box < D / 64; ++box)
           tma_load_4d(smem + L::kK + st * L::kTileBytes + box * 16384, &tm_k, &bars->k_full[st], box * 64, hk,
-                      (t_begin + j) * 128, b);
+                      tile_of(j) * 128, b);
         if (!mbar_wait(&bars->v_empty[st], par, p.status, kErrVEmpty)) break;
         mbar_arrive_expect_tx(&bars->v_full[st], L::kTileBytes);
         for (int box = 0; box < D / 64; ++box)
           tma_load_4d(smem + L::kV + st * L::kTileBytes + box * 16384, &tm_v, &bars->v_full[st], box * 64, hk,
-                      (t_begin + j) * 128, b);
+                      tile_of(j) * 128, b);
       }
     }
   } else if (warp == 8) {
@@ -276,14 +268,8 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       named_bar_sync(bar_id, 128);
       if (r == 0 && ok) mbar_arrive(&bars->q_ready[s]);
 
-      // Visible-key end of this row.
-      int limit = p.seqlen_kv, kv_first = 0;   // visible keys [kv_first, limit)
-      if (row < p.seqlen_q) {
-        const int c = find_chunk(p.q_offsets, p.n_q_chunks, row);
-        limit = __ldg(p.kv_offsets + p.n_kv_chunks - p.n_q_chunks + c + 1);
-        if (p.kv_range > 0)
-          kv_first = __ldg(p.kv_offsets + max(p.n_kv_chunks - p.n_q_chunks + c - p.kv_range + 1, 0));
-      }
+      int limit = p.seqlen_kv, kv_first = 0;
+      if (row < p.seqlen_q) row_keys(p.mask, row, kv_first, limit);
 
       float m_ref = -INFINITY, l_sum = 0.f;
       // Every thread runs all n_vis iterations and reaches every named
@@ -305,16 +291,21 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               for (int i = 0; i < 16; ++i)
                 x2[c * 16 + i] = f2_pack(__uint_as_float(raw[c][2 * i]), __uint_as_float(raw[c][2 * i + 1]));
           }
-          const int tile = t_begin + j;
-          const bool masked = tile < t_full_begin || tile >= n_full;
+          const int tile = tile_of(j);
+          const bool masked = kGlobal ? ft.masked(j, p.mask.global_key, p.seqlen_kv)
+                                      : tile < ft.t_full_begin || tile >= ft.n_full;
           if (masked) {
+            // columns [lo, lim) and, with a global block, its keys [glo, ghi) are visible
             const int lim = limit - tile * 128, lo = kv_first - tile * 128;
+            const int glo = kGlobal ? p.mask.global_key - tile * 128 : 0;
+            const int ghi = kGlobal ? p.seqlen_kv - tile * 128 : 0;
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
               float a0, a1;
               f2_unpack(x2[c], a0, a1);
-              x2[c] = f2_pack(2 * c >= lo && 2 * c < lim ? a0 : -INFINITY,
-                              2 * c + 1 >= lo && 2 * c + 1 < lim ? a1 : -INFINITY);
+              const bool v0 = (2 * c >= lo && 2 * c < lim) || (2 * c >= glo && 2 * c < ghi);
+              const bool v1 = (2 * c + 1 >= lo && 2 * c + 1 < lim) || (2 * c + 1 >= glo && 2 * c + 1 < ghi);
+              x2[c] = f2_pack(v0 ? a0 : -INFINITY, v1 ? a1 : -INFINITY);
             }
           }
           // row maximum as a tree (short dependency chains)
@@ -478,7 +469,7 @@ cudaError_t launch_knorm(const uint16_t* k, uint16_t* kn, int64_t rows, int head
   return cudaGetLastError();
 }
 
-template <int D, bool kRope>
+template <int D, bool kRope, bool kGlobal>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, int n_units, cudaStream_t stream) {
   using L = FwdLayout<D>;
@@ -487,11 +478,12 @@ static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((configured >> dev) & 1u)) {
-    e = cudaFuncSetAttribute(bca_fwd_kernel<D, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    e = cudaFuncSetAttribute(bca_fwd_kernel<D, kRope, kGlobal>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kAlloc);
     if (e != cudaSuccess) return e;
     if (dev < 64) configured |= uint64_t(1) << dev;
   }
-  bca_fwd_kernel<D, kRope><<<n_units, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  bca_fwd_kernel<D, kRope, kGlobal><<<n_units, kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -499,11 +491,19 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int head_dim, int n_units, cudaStream_t stream) {
   if (n_units <= 0) return cudaSuccess;
   const bool rope = p.rope_q != nullptr;
-  if (head_dim == 128)
-    return rope ? launch_fwd_d<128, true>(tq, tk, tv, p, n_units, stream)
-                : launch_fwd_d<128, false>(tq, tk, tv, p, n_units, stream);
-  return rope ? launch_fwd_d<64, true>(tq, tk, tv, p, n_units, stream)
-              : launch_fwd_d<64, false>(tq, tk, tv, p, n_units, stream);
+  const bool global = p.mask.global_key < p.seqlen_kv;
+  if (head_dim == 128) {
+    if (global)
+      return rope ? launch_fwd_d<128, true, true>(tq, tk, tv, p, n_units, stream)
+                  : launch_fwd_d<128, false, true>(tq, tk, tv, p, n_units, stream);
+    return rope ? launch_fwd_d<128, true, false>(tq, tk, tv, p, n_units, stream)
+                : launch_fwd_d<128, false, false>(tq, tk, tv, p, n_units, stream);
+  }
+  if (global)
+    return rope ? launch_fwd_d<64, true, true>(tq, tk, tv, p, n_units, stream)
+                : launch_fwd_d<64, false, true>(tq, tk, tv, p, n_units, stream);
+  return rope ? launch_fwd_d<64, true, false>(tq, tk, tv, p, n_units, stream)
+              : launch_fwd_d<64, false, false>(tq, tk, tv, p, n_units, stream);
 }
 
 size_t fwd_smem_bytes(int head_dim) {

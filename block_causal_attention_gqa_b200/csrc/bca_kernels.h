@@ -5,17 +5,29 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <vector>
 
 #include "../../include/magi_bca.h"
 
 namespace magi {
 
+// Which keys each query row sees, as the kernels read it (built on the host
+// from the chunk offsets, the KV range, the packed samples and the global
+// block; see MaskSpec in bca_sched.h).  A query row of chunk c sees the keys
+// [q_lo[c], q_hi[c]) and the global keys [global_key, seqlen_kv).
+struct MaskArgs {
+  const int32_t* q_offsets;   // device copy of the query chunk offsets [n_q_chunks + 1]
+  const int32_t* q_lo;        // device [n_q_chunks]: first visible key by the block-causal rule
+  const int32_t* q_hi;        // device [n_q_chunks]: end of those keys
+  int n_q_chunks;
+  int n_normal_q;             // chunks [0, n_normal_q) are not global (lo, hi non-decreasing there)
+  int global_q_row;           // rows from here on see every key (seqlen_q: none)
+  int global_key;             // keys from here on are seen by every row (seqlen_kv: none)
+};
+
 struct FwdParams {
   const int32_t* units;       // device, 12 int32 per unit (see magi_bca_fwd_schedule)
-  const int32_t* q_offsets;   // device copy of the query chunk offsets
-  const int32_t* kv_offsets;  // device copy of the kv chunk offsets
-  int n_q_chunks, n_kv_chunks;
-  int kv_range;               // 0 = no limit, else chunks visible back from the row's own
+  MaskArgs mask;
   const float* rope_q;        // rotary angles of the query tokens [Sq, D/2] or nullptr
   const float* gamma_q;
   const float* gamma_k;
@@ -36,11 +48,8 @@ struct BwdParams {
   const float* lse;           // [B, Hq, Sq] natural log
   const float* gamma_q;
   const float* gamma_k;
-  const int32_t* units;       // device schedule, 8 int32 per unit
-  const int32_t* q_offsets;   // device copies of the chunk offsets
-  const int32_t* kv_offsets;
-  int n_q_chunks, n_kv_chunks;
-  int kv_range;               // 0 = no limit, else chunks visible back from the row's own
+  const int32_t* units;       // device schedule, 12 int32 per unit (see magi_bca_bwd_schedule)
+  MaskArgs mask;
   const float* rope_q;        // rotary angles [Sq, D/2] / [Skv, D/2], or nullptr
   const float* rope_k;
   float* drope_q;             // their gradients (summed over batch and heads), or nullptr
@@ -97,6 +106,12 @@ size_t fwd_smem_bytes(int head_dim);
 // Records the diagnostic timing events (magi_bca_profile_events) on `stream`:
 // which = 0 before a main-kernel launch, 1 after it.  No-op when unset.
 void profile_mark(int which, cudaStream_t stream);
+
+// The mask part of a device schedule blob: query offsets, then lo, then hi
+// (3 n_q_chunks + 1 int32), and the MaskArgs that point into it at `dev`.
+struct MaskSpec;
+void append_mask_blob(std::vector<int32_t>& blob, const int32_t* q_offsets, const MaskSpec& m, int n_q_chunks);
+MaskArgs mask_args_at(const int32_t* dev, const MaskSpec& m, int n_q_chunks);
 
 // Shared host helpers (bca_api.cu).
 int make_tensor_map_bf16(CUtensorMap* m, const void* base, int B, int S, int H, int D);

@@ -87,8 +87,8 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   st = validate_offsets(q_chunk_offsets, kv_chunk_offsets, d);
   if (st != MAGI_BCA_OK) return st;
 
-  // Layout inside the array: [workspace][schedule units][q offsets][kv offsets]
-  // and, for the deterministic backward, [dq-pass units].
+  // Layout inside the array: [workspace][schedule units][mask blob: query
+  // offsets, lo, hi] and, for the deterministic backward, [dq-pass units].
   const BwdWorkspace ws = bwd_workspace_layout(d.batch, d.seqlen_q, d.seqlen_kv, d.heads_q, d.heads_kv, d.head_dim);
   int sms = 148;
   {
@@ -97,8 +97,8 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   }
   std::vector<int32_t> blob = build_bwd_schedule(q_chunk_offsets, kv_chunk_offsets, d, sms);
   const int n_units = static_cast<int>(blob.size() / kUnitInts);
-  blob.insert(blob.end(), q_chunk_offsets, q_chunk_offsets + d.n_q_chunks + 1);
-  blob.insert(blob.end(), kv_chunk_offsets, kv_chunk_offsets + d.n_kv_chunks + 1);
+  const MaskSpec mask = build_mask_spec(q_chunk_offsets, kv_chunk_offsets, d);
+  append_mask_blob(blob, q_chunk_offsets, mask, d.n_q_chunks);
   const size_t dq_units_off = blob.size();
   int n_dq_units = 0;
   if (d.deterministic) {
@@ -142,11 +142,7 @@ extern "C" int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16*
   p.gamma_q = gamma_q;
   p.gamma_k = gamma_k;
   p.units = sched;
-  p.q_offsets = sched + (size_t)n_units * kUnitInts;
-  p.kv_offsets = p.q_offsets + d.n_q_chunks + 1;
-  p.n_q_chunks = d.n_q_chunks;
-  p.n_kv_chunks = d.n_kv_chunks;
-  p.kv_range = d.kv_range;
+  p.mask = mask_args_at(sched + (size_t)n_units * kUnitInts, mask, d.n_q_chunks);
   p.rope_q = p.rope_k = nullptr;
   p.drope_q = p.drope_k = nullptr;
   p.deterministic = d.deterministic;

@@ -40,10 +40,18 @@
  *                      key/value chunk (chunk-wise text conditioning, MAGI-1 §7).
  *
  * Ownership: every tensor pointer is caller-owned device memory; the chunk
- * offsets are host memory read during the call.  The library keeps one
- * schedule cache (per device and shape; mutex-guarded) and allocates device
- * memory only when a new shape is first seen, so the first call for a shape
- * must come before any CUDA-graph capture of later calls.
+ * offsets are host memory read during the call.  The library's own device
+ * memory is bounded: a schedule cache (per device, shape and mask; at most 64
+ * entries per device, least recently used evicted; mutex-guarded) and, for the
+ * forward, one normalised-key buffer per stream, grown to the largest key
+ * length seen on it.  It allocates with cudaMallocAsync on the caller's stream
+ * and uploads schedules with cudaMemcpyAsync from pinned staging, and frees in
+ * stream order, so no call waits for the device.  Allocation happens only
+ * when a new shape (or a longer key sequence on a stream) is first seen: make
+ * that first call before any CUDA-graph capture of later calls; on a capturing
+ * stream a call that would need new memory returns MAGI_BCA_UNSUPPORTED.
+ * Schedules and buffers used under capture are kept until
+ * magi_bca_release_caches(), since a graph holds their addresses.
  *
  * Errors: every entry point returns MAGI_BCA_OK (0) or a negative status.
  * No exception crosses the ABI and no call synchronises the host with the
@@ -70,7 +78,7 @@ enum {
   MAGI_BCA_INVALID_ARG = -1,        /* null pointer, non-positive size, bad dims struct */
   MAGI_BCA_UNSUPPORTED = -2,        /* head_dim not 64/128, heads_q % heads_kv != 0, device not sm_100,
                                      * magi_bca_bwd_noalloc on a capturing stream */
-  MAGI_BCA_BAD_OFFSETS = -3,        /* chunk offsets violate the rules above */
+  MAGI_BCA_BAD_OFFSETS = -3,        /* chunk or sample offsets violate the rules above */
   MAGI_BCA_WORKSPACE_TOO_SMALL = -4,
   MAGI_BCA_CUDA_ERROR = -5,         /* a CUDA runtime call failed (launch, copy, ...) */
   MAGI_BCA_DEVICE_TIMEOUT = -6      /* a bounded device-side wait gave up */
@@ -97,6 +105,17 @@ typedef struct {
                           * reduced in a fixed order).  Costs about 7/5 of the tensor work of 0.
                           * 0 = fastest (fp32 reductions whose order depends on timing).  The
                           * forward is always deterministic and ignores it.  Must be 0 or 1. */
+  int32_t n_samples;     /* packed samples (MAGI-1 §4.1.2, Figure 15 (f), "varlen block-causal"): 0 or 1 =
+                          * the whole sequence is one sample; > 1 = sample_chunk_offsets lists the samples
+                          * packed one after another, and a query sees only keys of its own sample (the
+                          * sample of its matched kv chunk). */
+  int32_t n_global_chunks; /* global block (MAGI-1 §4.1.2, Figure 15 (g); App. B.1, Figure 23, a last
+                          * global block): the last n_global_chunks kv chunks.  Every query sees their
+                          * keys, and the query chunks matched to them see every key, whatever the
+                          * sample or the KV range.  0 = none; at most n_kv_chunks. */
+  const int32_t* sample_chunk_offsets; /* host int32 [n_samples + 1], read during the call: cumulative kv-chunk
+                          * counts of the samples, 0 = s[0] < s[1] < ... < s[n_samples] = n_kv_chunks.
+                          * Ignored (may be NULL) when n_samples <= 1. */
 } magi_bca_dims;
 
 /* Forward.  Writes out (bf16) and lse (fp32; may be NULL when the caller
@@ -171,6 +190,17 @@ int magi_bca_bwd_noalloc(const magi_bca_bf16* q, const magi_bca_bf16* k, const m
                          float* dgamma_q, float* dgamma_k,
                          const magi_bca_dims* dims, void* stream);
 
+/* Frees every schedule and buffer the library holds (the paper has no
+ * counterpart; memory management of this library).  Synchronises each device
+ * that holds any (the one call that does), so no launched kernel is still
+ * reading them; CUDA graphs captured earlier that used them must not be
+ * replayed afterwards.  Returns MAGI_BCA_OK or MAGI_BCA_CUDA_ERROR. */
+int magi_bca_release_caches(void);
+
+/* Bytes of device memory the library holds in its caches (schedules and
+ * normalised-key buffers, all devices); host-only, no synchronisation. */
+size_t magi_bca_cache_bytes(void);
+
 /* Static text for a status code. */
 const char* magi_bca_status_string(int status);
 
@@ -229,12 +259,15 @@ int magi_bca_selftest_wait_timeout(void* stream);
  * unit loads into shared memory serves both.  For every unit the scheduler
  * emits 12 int32 values:
  *   {batch, kv_head, head_0, m0_0, head_1, m0_1, n_full, n_tiles,
- *    t_begin, t_full_begin, 0, 0}
+ *    t_begin, t_full_begin, g_begin, g_end}
  * where (head_s, m0_s) is sub-tile s's query head and first query row
  * (head_1 = -1 when the unit has one sub-tile); kv tiles [t_begin, n_tiles)
- * are visited (t_begin > 0 only under a KV range) and tiles below
- * t_full_begin or from n_full on need the per-row mask.  Units are listed in
- * launch order: longest first.  The deterministic backward's query-major dq
+ * are visited (t_begin > 0 under a KV range or packed samples) and tiles below
+ * t_full_begin or from n_full on need the per-row mask; then, with a global
+ * block, the tiles [g_begin, g_end) of its keys that the first range does not
+ * hold (g_begin = g_end = 0 otherwise; masked only where they straddle the
+ * block's start or the sequence's end).  Units are listed in launch order:
+ * longest first.  The deterministic backward's query-major dq
  * pass runs the same units, one CTA per sub-tile.
  * Returns the number of units (even if larger than `capacity`, in which case
  * only `capacity` units are written), or a negative status. */
@@ -247,12 +280,18 @@ int64_t magi_bca_fwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_
  * the tile, numbered qt * G + g with G = heads_q / heads_kv.  Each tile's steps
  * are cut into near-equal pieces whose length is chosen by simulating how
  * `num_sms` SMs would run them (with dims->deterministic = 1 every tile is
- * one unit).  Per unit 8 int32:
+ * one unit).  Per unit 12 int32:
  *   {batch, kv_head, n0 (first key), step_begin, step_end,
- *    diag_end, diag_hi_begin, 0}
- * where query tiles below diag_end or from diag_hi_begin on (KV range) need
- * the mask, in launch order (longest first).  Returns the number of units
- * (writing at most `capacity`), or a negative status. */
+ *    diag_end, diag_hi_begin, split, jump, diag_global, 0, 0}
+ * A unit runs steps v in [step_begin, step_end); step v is the absolute step
+ * v (query tile v / G) below `split` and v + jump from `split` on, so with a
+ * global block a kv tile's steps can be two runs of query tiles: the rows that
+ * see its keys by the block-causal rule, then the global block's query rows
+ * (split = INT32_MAX, jump = 0 when there is one run).  Query tiles of the
+ * first run below diag_end or from diag_hi_begin on (KV range, packed samples)
+ * need the mask; in the second run only query tile diag_global does (-1:
+ * none).  Units are in launch order (longest first).  Returns the number of
+ * units (writing at most `capacity`), or a negative status. */
 int64_t magi_bca_bwd_schedule(const int32_t* q_chunk_offsets, const int32_t* kv_chunk_offsets,
                               const magi_bca_dims* dims, int32_t num_sms, int32_t* units, int64_t capacity);
 

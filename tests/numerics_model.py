@@ -34,7 +34,8 @@ def _rot(x, t):
     return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
 
 
-def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6, kv_range=0, rope_q=None, rope_k=None):
+def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6, kv_range=0, rope_q=None, rope_k=None, samples=None,
+                  n_global=0):
     q = inp["q"].double()
     k = inp["k"].double()
     v = inp["v"].double()
@@ -52,7 +53,8 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6, kv_range=0, rope_q=None,
     tk = None if rope_k is None else torch.as_tensor(rope_k).double()
     q_raw, k_raw = q, k
     q, k = _rot(q, tq), _rot(k, tk)          # a rotation keeps the RMS of the raw row
-    mask = torch.tensor(orc.block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range))
+    mask = torch.tensor(orc.block_causal_mask(q_offsets, kv_offsets, kv_range=kv_range, samples=samples,
+                                              n_global=n_global))
     kr, vr = k.repeat_interleave(g, 2), v.repeat_interleave(g, 2)
     kh = _bf(kr * rk.repeat_interleave(g, 2))
     qh = _bf(q * rq * (gq * gk * sc * l2e))
@@ -72,9 +74,9 @@ def model_fwd_bwd(inp, q_offsets, kv_offsets, eps=1e-6, kv_range=0, rope_q=None,
     q_op = qh / (gk * sc * l2e)                      # what the folded operand represents
     dkt = sc * torch.einsum("bhij,bihd->bjhd", ds, q_op).view(B, -1, Hkv, g, D).sum(3)
     dqt = sc * torch.einsum("bhij,bjhd->bihd", ds, kh * gk)
-    dq, _ = orc.rms_norm_backward(q.numpy(), gq.numpy(), dqt.numpy(), eps)
-    dk, _ = orc.rms_norm_backward(k.numpy(), gk.numpy(), dkt.numpy(), eps)
+    dq, dgq = orc.rms_norm_backward(q.numpy(), gq.numpy(), dqt.numpy(), eps)
+    dk, dgk = orc.rms_norm_backward(k.numpy(), gk.numpy(), dkt.numpy(), eps)
     dq, _ = orc.rope_backward(q_raw.numpy(), rope_q, dq)
     dk, _ = orc.rope_backward(k_raw.numpy(), rope_k, dk)
     return dict(out=out_bf.numpy(), lse=(lse2 / l2e).squeeze(-1).numpy(), dq=_bf(torch.tensor(dq)).numpy(),
-                dk=_bf(torch.tensor(dk)).numpy(), dv=_bf(dv).numpy())
+                dk=_bf(torch.tensor(dk)).numpy(), dv=_bf(dv).numpy(), dgamma_q=dgq, dgamma_k=dgk)

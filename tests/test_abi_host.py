@@ -144,59 +144,84 @@ def row_ends(qo, ko, Sq):
     return ends
 
 
-def row_intervals(qo, ko, kv_range=0):
-    """Per query row the visible keys [begin, end): its matched kv chunk's end,
-    and (KV range R) the start of the chunk R - 1 before it.  Checked against
-    the oracle's token-level mask on small shapes below."""
+def row_intervals(qo, ko, kv_range=0, samples=None, n_global=0):
+    """Per query row the visible keys [begin, end) by the block-causal rule: its
+    matched kv chunk's end, and the start of the chunk R - 1 before it (KV
+    range R) or of its sample, whichever is later; rows of the global block's
+    query chunks see [0, Skv).  Also returns the first global key g0 (every row
+    sees [g0, Skv)).  Checked against the oracle's token-level mask below."""
     nq, nkv = len(qo) - 1, len(ko) - 1
     Sq = int(qo[-1])
+    first_global = nkv - n_global
+    sample_first = np.zeros(nkv, np.int64)
+    if samples is not None:
+        for i in range(len(samples) - 1):
+            sample_first[samples[i]:samples[i + 1]] = samples[i]
     begin = np.zeros(Sq, np.int64)
     end = np.empty(Sq, np.int64)
     for c in range(nq):
         own = nkv - nq + c
-        end[qo[c]:qo[c + 1]] = ko[own + 1]
+        if own >= first_global:
+            begin[qo[c]:qo[c + 1]] = 0
+            end[qo[c]:qo[c + 1]] = ko[-1]
+            continue
+        first = sample_first[own]
         if kv_range > 0:
-            begin[qo[c]:qo[c + 1]] = ko[max(own - kv_range + 1, 0)]
-    return begin, end
+            first = max(first, own - kv_range + 1)
+        end[qo[c]:qo[c + 1]] = ko[own + 1]
+        begin[qo[c]:qo[c + 1]] = ko[first]
+    return begin, end, int(ko[first_global])
 
 
 class TileMask:
-    """any()/all() of the visibility of a (query rows, keys) block from row intervals."""
+    """any()/all() of the visibility of a (query rows, keys) block: a row sees
+    [begin, end) and the global keys [g0, Skv)."""
 
-    def __init__(self, qo, ko, kv_range=0):
-        self.begin, self.end = row_intervals(qo, ko, kv_range)
+    def __init__(self, qo, ko, kv_range=0, samples=None, n_global=0):
+        self.begin, self.end, self.g0 = row_intervals(qo, ko, kv_range, samples, n_global)
         self.Sq, self.Skv = int(qo[-1]), int(ko[-1])
+
+    def _any(self, b, e, k0, k1):
+        return ((b < k1) & (e > k0)) | (self.g0 < k1)
+
+    def _all(self, b, e, k0, k1):
+        # [k0, k1) inside [b, e) | [g0, Skv) (k1 <= Skv)
+        return ((b <= k0) & (e >= k1)) | (self.g0 <= k0) | ((b <= k0) & (e >= self.g0))
 
     def any(self, r0, r1, k0, k1):
         b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
-        return bool(((b < min(k1, self.Skv)) & (e > k0)).any())
+        return bool(self._any(b, e, k0, min(k1, self.Skv)).any())
 
     def all(self, r0, r1, k0, k1):
         b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
-        return bool(((b <= k0) & (e >= min(k1, self.Skv))).all())
+        return bool(self._all(b, e, k0, min(k1, self.Skv)).all())
 
     def any_tiles(self, r0, r1, n_tiles):
         """any() for key tiles 0..n_tiles-1 at once (128-key tiles)."""
         b, e = self.begin[r0:min(r1, self.Sq)], self.end[r0:min(r1, self.Sq)]
         k0 = np.arange(n_tiles) * 128
         k1 = np.minimum(k0 + 128, self.Skv)
-        return ((b[:, None] < k1[None, :]) & (e[:, None] > k0[None, :])).any(axis=0)
+        return self._any(b[:, None], e[:, None], k0[None, :], k1[None, :]).any(axis=0)
 
     def any_row_tiles(self, n_qt, k0, k1):
         """any() for query tiles 0..n_qt-1 at once against keys [k0, k1)."""
-        k1 = min(k1, self.Skv)
-        hit = (self.begin < k1) & (self.end > k0)
+        hit = self._any(self.begin, self.end, k0, min(k1, self.Skv))
         pad = np.zeros(n_qt * 128, bool)
         pad[:self.Sq] = hit
         return pad.reshape(n_qt, 128).any(axis=1)
 
     def all_row_tiles(self, n_qt, k0, k1):
         """all() for query tiles 0..n_qt-1 at once against keys [k0, k1) (rows past Sq ignored)."""
-        k1 = min(k1, self.Skv)
-        ok = (self.begin <= k0) & (self.end >= k1)
+        ok = self._all(self.begin, self.end, k0, min(k1, self.Skv))
         pad = np.ones(n_qt * 128, bool)
         pad[:self.Sq] = ok
         return pad.reshape(n_qt, 128).all(axis=1)
+
+
+def interval_mask(qo, ko, kv_range=0, samples=None, n_global=0):
+    b, e, g0 = row_intervals(qo, ko, kv_range, samples, n_global)
+    keys = np.arange(int(ko[-1]))
+    return ((keys[None, :] >= b[:, None]) & (keys[None, :] < e[:, None])) | (keys[None, :] >= g0)
 
 
 @pytest.mark.parametrize("q_lens,kv_lens,R", [([2, 3, 1], [2, 3, 1], 0), ([2, 3, 1], [2, 3, 1], 2),
@@ -204,39 +229,58 @@ class TileMask:
 def test_row_intervals_match_the_oracle_mask(q_lens, kv_lens, R):
     from oracle import bca_oracle as orc
     qo, ko = _offs(q_lens), _offs(kv_lens)
-    M = orc.block_causal_mask(qo, ko, kv_range=R)
-    b, e = row_intervals(qo, ko, R)
-    keys = np.arange(int(ko[-1]))
-    assert np.array_equal(M, (keys[None, :] >= b[:, None]) & (keys[None, :] < e[:, None]))
+    assert np.array_equal(orc.block_causal_mask(qo, ko, kv_range=R), interval_mask(qo, ko, R))
 
 
-def check_schedule(q_lens, kv_lens, B, Hq, Hkv, D=128, kv_range=0):
+@pytest.mark.parametrize("q_lens,kv_lens,R,samples,G", [
+    ([2, 1, 2, 1, 2], [2, 1, 2, 1, 2], 0, [0, 2, 3, 5], 0),
+    ([2, 1, 2, 1, 2], [2, 1, 2, 1, 2], 0, [0, 2, 3, 5], 1),
+    ([2, 1], [2, 1, 2, 1], 0, [0, 2, 4], 0),
+    ([1] * 5, [1] * 5, 2, [0, 3, 5], 1),
+    ([3, 4, 2, 5], [3, 4, 2, 5], 0, None, 2),
+    ([2, 3], [4, 2, 3], 0, [0, 1, 3], 2),
+])
+def test_row_intervals_with_samples_and_global_block_match_the_oracle_mask(q_lens, kv_lens, R, samples, G):
+    from oracle import bca_oracle as orc
+    qo, ko = _offs(q_lens), _offs(kv_lens)
+    want = orc.block_causal_mask(qo, ko, kv_range=R, samples=samples, n_global=G)
+    assert np.array_equal(want, interval_mask(qo, ko, R, samples, G))
+
+
+def check_schedule(q_lens, kv_lens, B, Hq, Hkv, D=128, kv_range=0, samples=None, n_global=0):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
-    units = bca.magi_bca_fwd_schedule(qo, ko, B, Hq, Hkv, D, kv_range=kv_range)
+    units = bca.magi_bca_fwd_schedule(qo, ko, B, Hq, Hkv, D, kv_range=kv_range, samples=samples,
+                                      n_global=n_global)
     assert units.shape[1] == 12
-    M = TileMask(qo, ko, kv_range)
+    M = TileMask(qo, ko, kv_range, samples, n_global)
     n_kt = -(-Skv // 128)
     g = Hq // Hkv
     seen = np.zeros((B, Hq, (Sq + 127) // 128), np.int64)
     costs = []
     checked = set()   # visibility depends only on the query tile, not on batch or head
-    for b, hk, h0, m00, h1, m01, n_full, n_tiles, t_begin, t_full_begin, z0, z1 in units:
-        assert z0 == 0 and z1 == 0
+    for b, hk, h0, m00, h1, m01, n_full, n_tiles, t_begin, t_full_begin, g_begin, g_end in units:
+        assert 0 <= g_begin <= g_end <= n_kt and (g_begin == g_end == 0 or g_begin >= n_tiles)
         subs = [(h0, m00)] + ([(h1, m01)] if h1 >= 0 else [])
         for h, m0 in subs:
             assert h // g == hk and m0 % 128 == 0
             seen[b, h, m0 // 128] += 1
-            if (m0, n_full, n_tiles, t_begin, t_full_begin) in checked:
+            key = (m0, n_full, n_tiles, t_begin, t_full_begin, g_begin, g_end)
+            if key in checked:
                 continue
-            checked.add((m0, n_full, n_tiles, t_begin, t_full_begin))
+            checked.add(key)
             tiles_seen = list(np.nonzero(M.any_tiles(m0, m0 + 128, n_kt))[0])
             # exactly the tiles with some visible (row, key) pair are visited
-            assert tiles_seen == list(range(t_begin, n_tiles)), (tiles_seen, t_begin, n_tiles)
+            visited = list(range(t_begin, n_tiles)) + list(range(g_begin, g_end))
+            assert tiles_seen == visited, (tiles_seen, t_begin, n_tiles, g_begin, g_end)
             # tiles the kernel leaves unmasked are fully visible to every row
             for t in range(max(t_begin, t_full_begin), min(n_full, n_tiles)):
                 assert M.all(m0, m0 + 128, t * 128, t * 128 + 128), t
-        costs.append((n_tiles - t_begin) * len(subs))
+            g0 = M.g0
+            for t in range(g_begin, g_end):
+                if not (t * 128 < g0 or t * 128 + 128 > Skv):
+                    assert M.all(m0, m0 + 128, t * 128, t * 128 + 128), t
+        costs.append((n_tiles - t_begin + g_end - g_begin) * len(subs))
     # every (batch, head, query tile) exactly once
     assert (seen == 1).all()
     # longest first
@@ -295,29 +339,34 @@ def test_workload_shapes():
     assert (w.batch, w.seqlen_q, w.seqlen_kv) == (2, 23040, 92160)
 
 
-def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=0, deterministic=False):
+def check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=148, kv_range=0, deterministic=False, samples=None,
+                       n_global=0):
     qo, ko = _offs(q_lens), _offs(kv_lens)
     Sq, Skv = int(qo[-1]), int(ko[-1])
     G = Hq // Hkv
     units = bca.magi_bca_bwd_schedule(qo, ko, B, Hq, Hkv, 128, num_sms, kv_range=kv_range,
-                                      deterministic=deterministic)
-    M = TileMask(qo, ko, kv_range)
+                                      deterministic=deterministic, samples=samples, n_global=n_global)
+    assert units.shape[1] == 12
+    M = TileMask(qo, ko, kv_range, samples, n_global)
     n_qt, n_kt = -(-Sq // 128), -(-Skv // 128)
     cover = np.zeros((B, Hkv, n_kt, n_qt, G), np.int64)
     lengths = []
     tile_any, tile_all = {}, {}
-    for b, hk, n0, s0, s1, diag_end, diag_hi_begin, z in units:
-        assert z == 0
-        assert n0 % 128 == 0 and 0 <= s0 < s1 <= n_qt * G
+    for b, hk, n0, s0, s1, diag_end, diag_hi_begin, split, jump, diag_global, z0, z1 in units:
+        assert z0 == 0 and z1 == 0 and jump >= 0
+        assert n0 % 128 == 0 and s0 < s1
         if n0 not in tile_any:
             tile_any[n0] = M.any_row_tiles(n_qt, n0, n0 + 128)
             tile_all[n0] = M.all_row_tiles(n_qt, n0, n0 + 128)
-        steps = np.arange(s0, s1)
+        v = np.arange(s0, s1, dtype=np.int64)
+        first = v < split
+        steps = np.where(first, v, v + jump)
+        assert (steps >= 0).all() and (steps < n_qt * G).all()
         t, g = steps // G, steps % G
         np.add.at(cover, (b, hk, n0 // 128, t, g), 1)
         assert tile_any[n0][t].all()                         # some row of each tile sees some key
-        plain = ~((t < diag_end) | (t >= diag_hi_begin))     # left unmasked: fully visible
-        assert tile_all[n0][t[plain]].all(), (n0, diag_end, diag_hi_begin)
+        masked = np.where(first, (t < diag_end) | (t >= diag_hi_begin), t == diag_global)
+        assert tile_all[n0][t[~masked]].all(), (n0, diag_end, diag_hi_begin, diag_global)   # unmasked: all visible
         lengths.append(s1 - s0)
     # every (kv tile, query tile, head) with a visible pair: exactly once
     for kt in range(n_kt):
@@ -375,9 +424,12 @@ def test_deterministic_bwd_schedule_has_one_unit_per_kv_tile(q_lens, kv_lens, B,
 
 
 def test_dims_struct_layout():
-    """magi_bca_dims: ten 4-byte fields, then kv_range and deterministic."""
-    assert ctypes.sizeof(bca.Dims) == 48
+    """magi_bca_dims: ten 4-byte fields, then kv_range, deterministic, n_samples,
+    n_global_chunks, and the host pointer to the sample offsets."""
+    assert ctypes.sizeof(bca.Dims) == 64
     assert bca.Dims.kv_range.offset == 40 and bca.Dims.deterministic.offset == 44
+    assert bca.Dims.n_samples.offset == 48 and bca.Dims.n_global_chunks.offset == 52
+    assert bca.Dims.sample_chunk_offsets.offset == 56
     assert bca.make_dims(1, 8, 8, 2, 1, 64, 1, 1, deterministic=True).deterministic == 1
 
 
@@ -466,10 +518,7 @@ def test_schedules_on_random_layouts(q_lens, kv_lens, B, Hq, Hkv, R):
     covers each visible (kv tile, query tile, head) once, pieced and whole."""
     from oracle import bca_oracle as orc
     qo, ko = _offs(q_lens), _offs(kv_lens)
-    b, e = row_intervals(qo, ko, R)
-    keys = np.arange(int(ko[-1]))
-    assert np.array_equal(orc.block_causal_mask(qo, ko, kv_range=R),
-                          (keys[None, :] >= b[:, None]) & (keys[None, :] < e[:, None]))
+    assert np.array_equal(orc.block_causal_mask(qo, ko, kv_range=R), interval_mask(qo, ko, R))
     check_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R)
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R)
     check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, kv_range=R, deterministic=True)
@@ -493,3 +542,63 @@ def test_maximum_sizes():
     d2 = bca.make_dims(1, S2, S2, 16, 2, 128, 1, 1)
     ws = bca.magi_bca_bwd_workspace_size(d2)
     assert ws >= S2 * 16 * 128 * (2 + 4)   # at least Q^ (bf16) and the fp32 dq accumulator
+
+
+def random_packed_layouts(seed, n):
+    """Seeded random packed layouts: 1-4 samples of 1-4 chunks of 1-600 tokens,
+    the training layout or (one time in three) the streaming one (the query
+    side the last 1..n_kv chunks), a KV range of 0-3, a global block of 0-2
+    trailing kv chunks, batch 1-2 and a GQA ratio of 1-4."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        sample_chunks = [int(rng.integers(1, 5)) for _ in range(int(rng.integers(1, 5)))]
+        n_kv = sum(sample_chunks)
+        kv = [int(x) for x in rng.integers(1, 601, n_kv)]
+        n_q = n_kv if rng.random() < 2 / 3 else int(rng.integers(1, n_kv + 1))
+        samples = [int(x) for x in np.concatenate([[0], np.cumsum(sample_chunks)])]
+        hkv = int(rng.integers(1, 3))
+        out.append((kv[n_kv - n_q:], kv, int(rng.integers(1, 3)), hkv * int(rng.integers(1, 5)), hkv,
+                    int(rng.integers(0, 4)), samples, int(rng.integers(0, min(2, n_kv) + 1))))
+    return out
+
+
+@pytest.mark.parametrize("q_lens,kv_lens,B,Hq,Hkv,R,samples,G", random_packed_layouts(2025, 24))
+def test_schedules_on_random_packed_layouts_with_global_blocks(q_lens, kv_lens, B, Hq, Hkv, R, samples, G):
+    """Packed samples and a last global block (MAGI-1 §4.1.2, Figure 15 (f), (g)):
+    the interval form of the mask equals the oracle's token mask, the forward
+    visits exactly the kv tiles with a visible pair (both ranges) and masks every
+    tile it does not see whole, and the backward covers each visible (kv tile,
+    query tile, head) once, pieced and whole."""
+    from oracle import bca_oracle as orc
+    qo, ko = _offs(q_lens), _offs(kv_lens)
+    assert np.array_equal(orc.block_causal_mask(qo, ko, kv_range=R, samples=samples, n_global=G),
+                          interval_mask(qo, ko, R, samples, G))
+    kw = dict(kv_range=R, samples=samples, n_global=G)
+    check_schedule(q_lens, kv_lens, B, Hq, Hkv, **kw)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, **kw)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, deterministic=True, **kw)
+    check_bwd_schedule(q_lens, kv_lens, B, Hq, Hkv, num_sms=7, **kw)
+
+
+@pytest.mark.parametrize("case,expect", [("samples_not_covering", BAD_OFFSETS), ("samples_empty", BAD_OFFSETS),
+                                         ("samples_null", INVALID_ARG), ("global_too_many", BAD_OFFSETS),
+                                         ("global_negative", INVALID_ARG), ("samples_negative", INVALID_ARG)])
+def test_bad_samples_and_global_blocks_are_rejected_on_the_host(case, expect):
+    qo = ko = _offs([10, 20, 5])
+    kw = {}
+    if case == "samples_not_covering":
+        kw = dict(samples=[0, 1, 2])
+    elif case == "samples_empty":
+        kw = dict(samples=[0, 1, 1, 3])
+    elif case == "global_too_many":
+        kw = dict(n_global=4)
+    elif case == "global_negative":
+        kw = dict(n_global=-1)
+    d = bca.make_dims(1, 35, 35, 4, 2, 128, 3, 3, **kw)
+    if case == "samples_null":
+        d.n_samples = 2
+        d.sample_chunk_offsets = None
+    elif case == "samples_negative":
+        d.n_samples = -1
+    assert call_fwd(d, qo, ko) == expect

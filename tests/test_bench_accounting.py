@@ -12,7 +12,7 @@ from oracle import bca_oracle as orc
 
 
 def pairs_from_mask(w):
-    return int(orc.block_causal_mask(w.q_offsets, w.kv_offsets, kv_range=w.kv_range).sum())
+    return int(orc.block_causal_mask(w.q_offsets, w.kv_offsets, **w.mask_kw).sum())
 
 
 @pytest.mark.parametrize("w", [
@@ -23,6 +23,11 @@ def pairs_from_mask(w):
     workloads.custom("window", 1, [300, 200, 150, 250, 100], None, 8, 2, 128, seed=0, kv_range=2),
     workloads.custom("xattn", 1, [777], [64], 4, 1, 128, seed=0),
     workloads.custom("chunkwise_text", 1, [300, 200, 250], [77, 120, 64], 4, 2, 64, seed=0, kv_range=1),
+    workloads.custom("packed", 1, [100, 333, 250, 67, 400, 190], None, 4, 2, 128, seed=0, samples=[0, 2, 3, 6]),
+    workloads.custom("packed_global_r2", 1, [100, 333, 250, 67, 400, 190], None, 4, 2, 128, seed=0,
+                     samples=[0, 2, 3, 6], n_global=1, kv_range=2),
+    workloads.custom("packed_stream_global", 2, [150, 250], [300, 200, 150, 250], 8, 2, 64, seed=0,
+                     samples=[0, 1, 4], n_global=1),
 ], ids=lambda w: w.name)
 def test_forward_flops_count_the_visible_pairs(w):
     want = 4.0 * w.head_dim * w.batch * w.heads_q * pairs_from_mask(w)

@@ -12,13 +12,14 @@ import torch
 import block_causal_attention_gqa_b200 as bca
 import workloads
 from oracle import bca_oracle as orc
-from tests._helpers import assert_close, grad_bound, rel_l2, to_np
+from tests._helpers import assert_close, dgamma_bound, grad_bound, rel_l2, to_np
 from tests.test_fwd_parity import SMALL
 
 pytestmark = pytest.mark.gpu
 
 DET_SMALL = ["train4k", "tiny", "ragged_d128", "ragged_d64_gqa3", "stream_small", "token_causal", "many_chunks",
-             "gqa8_long_rows", "window_r2_ragged", "window_stream_r3_d64", "xattn_video_text", "xattn_chunkwise"]
+             "gqa8_long_rows", "window_r2_ragged", "window_stream_r3_d64", "xattn_video_text", "xattn_chunkwise",
+             "packed_global_ragged", "packed_global_r2_d64", "packed_stream_global"]
 
 
 def to_dev(inp):
@@ -33,23 +34,23 @@ def to_dev(inp):
 def det_bwd(w, t, out, lse, rope=False, workspace=None):
     if rope:
         return bca.magi_bca_bwd_rope(t["q"], t["k"], t["v"], out, t["dout"], lse, w.q_offsets, w.kv_offsets,
-                                     t["gamma_q"], t["gamma_k"], t["rope_q"], t["rope_k"], kv_range=w.kv_range,
+                                     t["gamma_q"], t["gamma_k"], t["rope_q"], t["rope_k"], **w.mask_kw,
                                      workspace=workspace, deterministic=True)
     return bca.magi_bca_bwd(t["q"], t["k"], t["v"], out, t["dout"], lse, w.q_offsets, w.kv_offsets, t["gamma_q"],
-                            t["gamma_k"], kv_range=w.kv_range, workspace=workspace, deterministic=True)
+                            t["gamma_k"], **w.mask_kw, workspace=workspace, deterministic=True)
 
 
 def fwd(w, t, rope=False):
     if rope:
         return bca.magi_bca_fwd_rope(t["q"], t["k"], t["v"], w.q_offsets, w.kv_offsets, t["gamma_q"], t["gamma_k"],
-                                     t["rope_q"], t["rope_k"], kv_range=w.kv_range)
+                                     t["rope_q"], t["rope_k"], **w.mask_kw)
     return bca.magi_bca_fwd(t["q"], t["k"], t["v"], w.q_offsets, w.kv_offsets, t["gamma_q"], t["gamma_k"],
-                            kv_range=w.kv_range)
+                            **w.mask_kw)
 
 
 def workspace_filled(w, byte):
     dims = bca.make_dims(w.batch, w.seqlen_q, w.seqlen_kv, w.heads_q, w.heads_kv, w.head_dim,
-                         len(w.q_chunks), len(w.kv_chunks), kv_range=w.kv_range, deterministic=True)
+                         len(w.q_chunks), len(w.kv_chunks), **w.mask_kw, deterministic=True)
     return torch.full((bca.magi_bca_bwd_workspace_size(dims),), byte, device="cuda", dtype=torch.uint8)
 
 
@@ -63,7 +64,7 @@ def test_deterministic_backward_all_rows(name):
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
     ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                       inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
+                       inp["gamma_q"], inp["gamma_k"], **w.mask_kw)
     bound = grad_bound(name)
     for nm, got in (("dq", dq), ("dk", dk), ("dv", dv)):
         e, r = assert_close(f"{name} {nm}", to_np(got), ref[nm], max_abs=bound)
@@ -71,10 +72,11 @@ def test_deterministic_backward_all_rows(name):
     for nm, got in (("dgamma_q", dgq), ("dgamma_k", dgk)):
         r = rel_l2(to_np(got), ref[nm])
         print(f"{name} {nm}: rel L2 {r:.2e}")
-        assert r <= 5e-3, f"{name} {nm}: rel L2 {r:.3e}"
+        assert r <= dgamma_bound(name), f"{name} {nm}: rel L2 {r:.3e}"
 
 
-@pytest.mark.parametrize("name", ["train4k", "ragged_d64_gqa3", "window_r2_ragged", "xattn_chunkwise"])
+@pytest.mark.parametrize("name", ["train4k", "ragged_d64_gqa3", "window_r2_ragged", "xattn_chunkwise",
+                                  "packed_global_ragged"])
 def test_deterministic_backward_is_bitwise_reproducible(name):
     w = SMALL[name]
     t = to_dev(workloads.make_inputs(w, with_grad_out=True))
@@ -113,7 +115,7 @@ def test_deterministic_noalloc_matches_the_workspace_entry_bitwise():
     dgq = torch.empty(w.head_dim, device="cuda")
     dgk = torch.empty(w.head_dim, device="cuda")
     b = bca.magi_bca_bwd_noalloc(t["q"], t["k"], t["v"], out, t["dout"], lse, w.q_offsets, w.kv_offsets,
-                                 t["gamma_q"], t["gamma_k"], dq, dk, dv, dgq, dgk, kv_range=w.kv_range,
+                                 t["gamma_q"], t["gamma_k"], dq, dk, dv, dgq, dgk, **w.mask_kw,
                                  deterministic=True)
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
@@ -143,7 +145,7 @@ def test_deterministic_rope_backward(name):
     for nm, a, b in zip(names, g1, g2):
         assert torch.equal(a, b), f"{name} {nm}: two deterministic calls differ"
     ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
-                       inp["gamma_k"], kv_range=w.kv_range, rope_q=inp["rope_q"], rope_k=inp["rope_k"])
+                       inp["gamma_k"], **w.mask_kw, rope_q=inp["rope_q"], rope_k=inp["rope_k"])
     for nm, got in zip(names[:3], g1[:3]):
         e, r = assert_close(f"{name} {nm}", to_np(got), ref[nm], max_abs=grad_bound(w.name))
         print(f"{name} {nm}: max abs {e:.2e} rel L2 {r:.2e}")

@@ -20,7 +20,7 @@ def run_gpu(inp, w, lse=True):
     dev = "cuda"
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
     out, l = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, inp["gamma_q"].to(dev),
-                              inp["gamma_k"].to(dev), want_lse=lse, kv_range=w.kv_range)
+                              inp["gamma_k"].to(dev), want_lse=lse, **w.mask_kw)
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
     return out, l
@@ -52,6 +52,17 @@ SMALL = {
     "xattn_short_q_d64": workloads.custom("xattn_short_q_d64", 1, [77], [1000], 4, 2, 64, seed=27),
     "xattn_chunkwise": workloads.custom("xattn_chunkwise", 1, [300, 200, 250], [77, 120, 64], 8, 2, 128,
                                         seed=28, kv_range=1),
+    # packed samples (MAGI-1 §4.1.2, Figure 15 (f)) and a last global block (Figure 15 (g))
+    "packed_ragged": workloads.custom("packed_ragged", 2, [100, 333, 250, 67, 400, 190], None, 4, 2, 128, seed=51,
+                                      samples=[0, 2, 3, 6]),
+    "packed_global_ragged": workloads.custom("packed_global_ragged", 2, [100, 333, 250, 67, 400, 190], None, 4, 2,
+                                             128, seed=52, samples=[0, 2, 3, 6], n_global=1),
+    "packed_global_r2_d64": workloads.custom("packed_global_r2_d64", 1, [256, 256, 256, 130, 126, 256, 256], None,
+                                             8, 2, 64, seed=53, samples=[0, 3, 5, 7], n_global=1, kv_range=2),
+    "packed_stream_global": workloads.custom("packed_stream_global", 2, [150, 250], [300, 200, 150, 250], 8, 2, 128,
+                                             seed=54, samples=[0, 1, 4], n_global=1),
+    "packed_global_gqa8": workloads.custom("packed_global_gqa8", 1, [640, 320, 640], None, 16, 2, 128, seed=55,
+                                           samples=[0, 1, 3], n_global=1),
 }
 
 
@@ -61,14 +72,14 @@ def test_forward_all_rows(name):
     inp = workloads.make_inputs(w, with_grad_out=False)
     out, lse = run_gpu(inp, w)
     o_ref, l_ref = orc.forward(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
-                               inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
+                               inp["gamma_q"], inp["gamma_k"], **w.mask_kw)
     e, r = assert_close(f"{name} out", to_np(out), o_ref)
     el, rl = assert_lse_close(f"{name} lse", to_np(lse), l_ref)
     print(f"{name}: out max abs {e:.2e} rel L2 {r:.2e}; lse max abs {el:.2e} rel L2 {rl:.2e}")
     if "q_f32" in inp:
         # information only: error against the unrounded fp32 inputs
         o32, _ = orc.forward(inp["q_f32"], inp["k_f32"], inp["v_f32"], w.q_offsets, w.kv_offsets,
-                             inp["gamma_q"], inp["gamma_k"], kv_range=w.kv_range)
+                             inp["gamma_q"], inp["gamma_k"], **w.mask_kw)
         print(f"{name}: rel L2 vs unrounded fp32 inputs {rel_l2(to_np(out), o32):.3e}")
 
 
@@ -97,7 +108,7 @@ def test_forward_is_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-LARGE = ["model46k", "stream4of16", "long262k", "window262k", "xattn46k"]
+LARGE = ["model46k", "stream4of16", "long262k", "window262k", "xattn46k", "packed46k"]
 
 
 @pytest.mark.parametrize("name", LARGE)
@@ -113,7 +124,7 @@ def test_forward_full_size_sampled_rows(name):
     for b in range(w.batch):
         rows = workloads.sample_rows(w.seqlen_q, w.q_offsets, per_batch, seed=100 + b)
         o_ref, l_ref = orc.forward_rows(inp["q"], inp["k"], inp["v"], w.q_offsets, w.kv_offsets,
-                                        inp["gamma_q"], inp["gamma_k"], rows, batches=[b], kv_range=w.kv_range)
+                                        inp["gamma_q"], inp["gamma_k"], rows, batches=[b], **w.mask_kw)
         idx = torch.as_tensor(rows)
         e, r = assert_close(f"{name} out b{b}", to_np(out_c[b:b + 1, idx]), o_ref)
         el, rl = assert_lse_close(f"{name} lse b{b}", to_np(lse_c[b:b + 1][:, :, idx]), l_ref)

@@ -21,6 +21,8 @@ CASES = {
     "rope_window_r2": (workloads.custom("rope_window_r2", 1, [300, 200, 150, 250], None, 8, 2, 128, seed=34,
                                         rope=True, kv_range=2), "qk"),
     "rope_train4k": (workloads.custom("rope_train4k", 1, [1024] * 4, None, 16, 4, 128, seed=35, rope=True), "qk"),
+    "rope_packed_global": (workloads.custom("rope_packed_global", 1, [300, 200, 150, 250], None, 8, 2, 128, seed=37,
+                                            rope=True, samples=[0, 2, 4], n_global=1), "qk"),
 }
 
 
@@ -40,13 +42,13 @@ def test_rope_forward_and_backward_all_rows(name):
     gq, gk = inp["gamma_q"].to(dev), inp["gamma_k"].to(dev)
     rqd = rq.to(dev) if rq is not None else None
     rkd = rk.to(dev) if rk is not None else None
-    out, lse = bca.magi_bca_fwd_rope(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, rqd, rkd, kv_range=w.kv_range)
+    out, lse = bca.magi_bca_fwd_rope(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, rqd, rkd, **w.mask_kw)
     dq, dk, dv, dgq, dgk, drq, drk = bca.magi_bca_bwd_rope(q, k, v, out, do, lse, w.q_offsets, w.kv_offsets, gq, gk,
-                                                           rqd, rkd, kv_range=w.kv_range)
+                                                           rqd, rkd, **w.mask_kw)
     torch.cuda.synchronize()
     assert bca.magi_bca_last_device_status() == 0
     ref = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets, inp["gamma_q"],
-                       inp["gamma_k"], kv_range=w.kv_range, rope_q=rq, rope_k=rk)
+                       inp["gamma_k"], **w.mask_kw, rope_q=rq, rope_k=rk)
     assert_close(f"{name} out", to_np(out), ref["out"])
     assert_lse_close(f"{name} lse", to_np(lse), ref["lse"])
     for nm, got in (("dq", dq), ("dk", dk), ("dv", dv)):

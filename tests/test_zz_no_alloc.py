@@ -20,26 +20,29 @@ from tests._helpers import assert_close, grad_bound, rel_l2, to_np
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["train4k", "ragged"])
+@pytest.mark.parametrize("name", ["train4k", "ragged", "packed_global"])
 def test_noalloc_backward_matches_regular_backward_twice(name):
     if name == "train4k":
         w = workloads.workload("train4k")
-    else:
+    elif name == "ragged":
         w = workloads.custom("ragged_d128", 2, [100, 333, 1000, 67], None, 4, 2, 128, seed=11)
+    else:
+        w = workloads.custom("packed_global_ragged", 2, [100, 333, 250, 67, 400, 190], None, 4, 2, 128, seed=52,
+                             samples=[0, 2, 3, 6], n_global=1)
     inp = workloads.make_inputs(w, with_grad_out=True)
     dev = "cuda"
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
     gq, gk = inp["gamma_q"].to(dev), inp["gamma_k"].to(dev)
     dout = inp["dout"].to(dev)
-    out, lse = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk)
-    ref = bca.magi_bca_bwd(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk)
+    out, lse = bca.magi_bca_fwd(q, k, v, w.q_offsets, w.kv_offsets, gq, gk, **w.mask_kw)
+    ref = bca.magi_bca_bwd(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk, **w.mask_kw)
     torch.cuda.synchronize()
     want = orc.backward(inp["q"], inp["k"], inp["v"], inp["dout"], w.q_offsets, w.kv_offsets,
-                        inp["gamma_q"], inp["gamma_k"])
+                        inp["gamma_q"], inp["gamma_k"], **w.mask_kw)
     for call in range(2):
         got = (torch.full_like(q, 3.0), torch.full_like(k, 3.0), torch.full_like(v, 3.0),
                torch.full((w.head_dim,), 3.0, device=dev), torch.full((w.head_dim,), 3.0, device=dev))
-        bca.magi_bca_bwd_noalloc(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk, *got)
+        bca.magi_bca_bwd_noalloc(q, k, v, out, dout, lse, w.q_offsets, w.kv_offsets, gq, gk, *got, **w.mask_kw)
         torch.cuda.synchronize()
         assert bca.magi_bca_last_device_status() == 0
         for nm, a, b in zip(("dq", "dk", "dv"), got[:3], ref[:3]):

@@ -51,6 +51,8 @@ class Workload:
     kv_range: int = 0            # KV range in chunks (0 = every earlier chunk); MAGI-1 §2.4.4, Fig. 12
     rope: bool = False           # rotary angles for q and k (3D positions, see rope_angles)
     deterministic: bool = False  # backward with every sum in a fixed order (same bits on every call)
+    samples: Optional[tuple] = None  # packed samples: cumulative kv-chunk counts (None: one sample)
+    n_global: int = 0            # the last n_global kv chunks form a global block
     shard_rank: int = 0          # with shard_world > 1: this workload is kv heads [r*Hkv, (r+1)*Hkv) (and
     shard_world: int = 1         # their query groups) of a problem with shard_world times the heads
 
@@ -61,6 +63,13 @@ class Workload:
     @property
     def seqlen_kv(self) -> int:
         return int(sum(self.kv_chunks))
+
+    @property
+    def mask_kw(self) -> dict:
+        """The mask options as keyword arguments (the binding's entry points and
+        the oracle take the same names)."""
+        return dict(kv_range=self.kv_range, samples=None if self.samples is None else list(self.samples),
+                    n_global=self.n_global)
 
     @property
     def q_offsets(self) -> np.ndarray:
@@ -108,6 +117,11 @@ WORKLOADS = {
     # RoPE; angles from the 6 x 24 x 40 latent grid of each chunk, see rope_angles).
     "model46k_rope": Workload("model46k_rope", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760),
                               24, 8, 128, seed=7, backward=True, rope=True),
+    # packed training sequence of model46k's size (MAGI-1 §4.1.2, Figure 15 (g)): three samples of
+    # 3, 1 and 3 chunks of 5760 tokens packed one after another, and a last chunk that forms a global
+    # block (every query sees it, its queries see everything), GQA 24/8
+    "packed46k": Workload("packed46k", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760), 24, 8, 128,
+                          seed=8, backward=True, samples=(0, 3, 4, 7, 8), n_global=1),
     # model46k through the deterministic backward (dq from a query-major pass, one unit
     # per kv tile, fixed-order dgamma): the reproducible-training setting
     "model46k_det": Workload("model46k_det", 1, uniform_offsets(8, 5760), uniform_offsets(8, 5760),
@@ -117,7 +131,7 @@ WORKLOADS = {
 }
 
 ORDER = ["tiny", "train4k", "model46k", "stream4of16", "long262k", "window262k", "xattn46k", "model46k_rope",
-         "model46k_det", "train4k_det", "long65k"]
+         "model46k_det", "train4k_det", "long65k", "packed46k"]
 
 
 def workload(name_or_index) -> Workload:
@@ -147,10 +161,13 @@ def shard_heads(w: Workload, world: int, rank: int) -> Workload:
 def custom(name: str, batch: int, q_chunks: Sequence[int], kv_chunks: Optional[Sequence[int]],
            heads_q: int, heads_kv: int, head_dim: int, seed: int, backward: bool = True,
            gamma: str = "perturbed", token_scale: bool = False, kv_range: int = 0,
-           rope: bool = False) -> Workload:
+           rope: bool = False, samples: Optional[Sequence[int]] = None, n_global: int = 0,
+           deterministic: bool = False) -> Workload:
     kv = tuple(kv_chunks) if kv_chunks is not None else tuple(q_chunks)
     return Workload(name, batch, tuple(q_chunks), kv, heads_q, heads_kv, head_dim, seed,
-                    backward, gamma=gamma, token_scale=token_scale, kv_range=kv_range, rope=rope)
+                    backward, gamma=gamma, token_scale=token_scale, kv_range=kv_range, rope=rope,
+                    deterministic=deterministic, samples=None if samples is None else tuple(samples),
+                    n_global=n_global)
 
 
 def rope_angles(positions: np.ndarray, head_dim: int, grid=(6, 24, 40), base: float = 10000.0) -> np.ndarray:

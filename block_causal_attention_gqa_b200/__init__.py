@@ -26,7 +26,9 @@ __all__ = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_fwd_rope", "magi_bca_bwd_ro
            "library_path", "EXPORTED_SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libmagi_bca.so")
+# MAGI_BCA_LIBRARY selects another build of the library (e.g. the bounds-checked
+# libmagi_bca_debug.so from `build.py --debug`); the default is the in-tree build.
+library_path = os.environ.get("MAGI_BCA_LIBRARY") or os.path.join(_HERE, "libmagi_bca.so")
 
 EXPORTED_SYMBOLS = ["magi_bca_fwd", "magi_bca_bwd", "magi_bca_bwd_workspace_size", "magi_bca_status_string",
                     "magi_bca_last_device_status", "magi_bca_fwd_schedule", "magi_bca_version",

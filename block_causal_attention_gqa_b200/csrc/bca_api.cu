@@ -397,6 +397,7 @@ const char* magi_bca_status_string(int status) {
     case MAGI_BCA_WORKSPACE_TOO_SMALL: return "workspace too small";
     case MAGI_BCA_CUDA_ERROR: return "CUDA runtime error";
     case MAGI_BCA_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MAGI_BCA_DEVICE_CHECK: return "device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -477,9 +478,11 @@ int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   p.gamma_k = gamma_k;
   p.out = out;
   p.lse = lse;
+  p.batch = d.batch;
   p.seqlen_q = d.seqlen_q;
   p.seqlen_kv = d.seqlen_kv;
   p.heads_q = d.heads_q;
+  p.heads_kv = d.heads_kv;
   p.scale_log2 = resolve_scale(d) * 1.4426950408889634f;
   p.eps = d.rms_eps;
   p.status = ds->status;
@@ -653,7 +656,8 @@ int magi_bca_last_device_status(void) {
   if (cudaMemcpyFromSymbol(&host, g_device_status, sizeof(int)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MAGI_BCA_CUDA_ERROR;
-  return host == 0 ? MAGI_BCA_OK : MAGI_BCA_DEVICE_TIMEOUT;
+  if (host == 0) return MAGI_BCA_OK;
+  return host >= 3000 && host < 3100 ? MAGI_BCA_DEVICE_CHECK : MAGI_BCA_DEVICE_TIMEOUT;
 }
 
 }  // extern "C"

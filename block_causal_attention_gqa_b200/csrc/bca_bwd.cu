@@ -261,6 +261,9 @@ bca_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int32_t* u = p.units + (size_t)blockIdx.x * kUnitInts;
+  if constexpr (kDebugChecks) {
+    if (!bwd_unit_in_range(u, p.batch, p.heads_q, p.heads_kv, p.seqlen_q, p.seqlen_kv, p.status)) return;
+  }
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
   // this kv tile's steps t = 0 .. n_steps-1; absolute step s = bs.abs_step(t)
   // is (query tile s / group, head s % group of the kv head's group), and

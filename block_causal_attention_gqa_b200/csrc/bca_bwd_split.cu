@@ -81,6 +81,9 @@ bca_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int32_t* u = p.units + (size_t)blockIdx.x * kUnitInts;
+  if constexpr (kDebugChecks) {
+    if (!bwd_unit_in_range(u, p.batch, p.heads_q, p.heads_kv, p.seqlen_q, p.seqlen_kv, p.status)) return;
+  }
   const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
   const BwdSteps bs = bwd_steps(u);   // steps t -> absolute steps, and which need the mask
   const int group = p.heads_q / p.heads_kv;
@@ -390,7 +393,10 @@ bca_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_consta
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const BwdParams p, const int smem_alloc) {
   using L = DqLayout<D>;
-  const int32_t* u = p.dq_units + (size_t)(blockIdx.x >> 1) * 12;
+  const int32_t* u = p.dq_units + (size_t)(blockIdx.x >> 1) * kFwdUnitInts;
+  if constexpr (kDebugChecks) {
+    if (!fwd_unit_in_range(u, p.batch, p.heads_q, p.heads_kv, p.seqlen_q, p.seqlen_kv, p.status)) return;
+  }
   const int sub = blockIdx.x & 1;
   const int h = __ldg(u + (sub ? 4 : 2));
   if (h < 0) return;  // the unit has one sub-tile: this CTA has no work

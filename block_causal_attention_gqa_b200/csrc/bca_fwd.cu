@@ -104,7 +104,10 @@ bca_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int32_t* u = p.units + (size_t)blockIdx.x * 12;
+  const int32_t* u = p.units + (size_t)blockIdx.x * kFwdUnitInts;
+  if constexpr (kDebugChecks) {
+    if (!fwd_unit_in_range(u, p.batch, p.heads_q, p.heads_kv, p.seqlen_q, p.seqlen_kv, p.status)) return;
+  }
   const int b = __ldg(u + 0), hk = __ldg(u + 1);
   const int head0 = __ldg(u + 2), head1 = __ldg(u + 4);
   const int m00 = __ldg(u + 3), m01 = __ldg(u + 5);

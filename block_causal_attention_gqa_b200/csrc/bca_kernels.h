@@ -33,10 +33,10 @@ struct FwdParams {
   const float* gamma_k;
   uint16_t* out;              // [B, Sq, Hq, D] bf16
   float* lse;                 // [B, Hq, Sq] or nullptr
-  int seqlen_q, seqlen_kv, heads_q;
+  int batch, seqlen_q, seqlen_kv, heads_q, heads_kv;
   float scale_log2;           // softmax_scale * log2(e)
   float eps;
-  int* status;                // device status word (bounded waits)
+  int* status;                // device status word (bounded waits, debug checks)
 };
 
 struct BwdParams {

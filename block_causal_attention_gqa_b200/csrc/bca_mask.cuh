@@ -112,4 +112,52 @@ __device__ __forceinline__ BwdSteps bwd_steps(const int32_t* u) {
   return s;
 }
 
+// ------------------------------------------------------------ debug build
+// Built with -DMAGI_BCA_DEBUG (build.py --debug), every attention kernel first
+// checks its work unit against the problem's sizes; a unit out of range (a
+// scheduler defect) records kErrDbgUnit in the device status word and the CTA
+// returns before any memory access, barrier or TMEM allocation.  The host reads
+// the code as MAGI_BCA_DEVICE_CHECK.  The product build compiles the checks out.
+#ifdef MAGI_BCA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+constexpr int kErrDbgUnit = 3001;
+
+__device__ __forceinline__ bool debug_fail(int* status) {
+  atomicCAS(status, 0, kErrDbgUnit);
+  return false;
+}
+
+// A forward (query-major) unit: batch, kv head, its query heads and rows, and
+// both kv tile ranges inside the problem.
+__device__ __forceinline__ bool fwd_unit_in_range(const int32_t* u, int batch, int heads_q, int heads_kv,
+                                                  int seqlen_q, int seqlen_kv, int* status) {
+  const int group = heads_q / heads_kv;
+  const int n_kt = (seqlen_kv + 127) / 128;
+  const int b = __ldg(u + 0), hk = __ldg(u + 1), h0 = __ldg(u + 2), m0 = __ldg(u + 3), h1 = __ldg(u + 4),
+            m1 = __ldg(u + 5);
+  const FwdTiles f = fwd_tiles(u);
+  bool ok = b >= 0 && b < batch && hk >= 0 && hk < heads_kv;
+  ok = ok && h0 >= hk * group && h0 < (hk + 1) * group && m0 >= 0 && m0 < seqlen_q && m0 % 128 == 0;
+  ok = ok && (h1 == -1 || (h1 >= hk * group && h1 < (hk + 1) * group && m1 >= 0 && m1 < seqlen_q && m1 % 128 == 0));
+  ok = ok && f.t_begin >= 0 && f.t_begin <= f.n_tiles && f.n_tiles <= n_kt;
+  ok = ok && ((f.g_begin == 0 && f.g_end == 0) || (f.n_tiles <= f.g_begin && f.g_begin <= f.g_end && f.g_end <= n_kt));
+  return ok || debug_fail(status);
+}
+
+// A backward (kv-major) unit: batch, kv head, kv tile and every step it runs.
+__device__ __forceinline__ bool bwd_unit_in_range(const int32_t* u, int batch, int heads_q, int heads_kv,
+                                                  int seqlen_q, int seqlen_kv, int* status) {
+  const int group = heads_q / heads_kv;
+  const int n_steps_all = (seqlen_q + 127) / 128 * group;
+  const int b = __ldg(u + 0), hk = __ldg(u + 1), n0 = __ldg(u + 2);
+  const BwdSteps bs = bwd_steps(u);
+  bool ok = b >= 0 && b < batch && hk >= 0 && hk < heads_kv && n0 >= 0 && n0 < seqlen_kv && n0 % 128 == 0;
+  ok = ok && bs.v_begin < bs.v_end && bs.jump >= 0;
+  ok = ok && bs.abs_step(0) >= 0 && bs.abs_step(bs.count() - 1) < n_steps_all;
+  return ok || debug_fail(status);
+}
+
 }  // namespace magi

@@ -81,7 +81,9 @@ enum {
   MAGI_BCA_BAD_OFFSETS = -3,        /* chunk or sample offsets violate the rules above */
   MAGI_BCA_WORKSPACE_TOO_SMALL = -4,
   MAGI_BCA_CUDA_ERROR = -5,         /* a CUDA runtime call failed (launch, copy, ...) */
-  MAGI_BCA_DEVICE_TIMEOUT = -6      /* a bounded device-side wait gave up */
+  MAGI_BCA_DEVICE_TIMEOUT = -6,     /* a bounded device-side wait gave up */
+  MAGI_BCA_DEVICE_CHECK = -7        /* a device-side bounds check failed (library built with
+                                     * -DMAGI_BCA_DEBUG: a work unit outside the problem) */
 };
 
 typedef struct {
@@ -226,8 +228,9 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
                       const magi_bca_dims* dims, void* stream);
 
 /* Reads (and clears) the device status word that bounded waits write when
- * they give up.  Synchronises with the device; returns MAGI_BCA_OK or
- * MAGI_BCA_DEVICE_TIMEOUT (or MAGI_BCA_CUDA_ERROR if the read itself fails).
+ * they give up (and, in a -DMAGI_BCA_DEBUG build, the kernels' bounds checks).
+ * Synchronises with the device; returns MAGI_BCA_OK, MAGI_BCA_DEVICE_TIMEOUT or
+ * MAGI_BCA_DEVICE_CHECK (or MAGI_BCA_CUDA_ERROR if the read itself fails).
  * Meant for tests and diagnostics, not for the hot path. */
 int magi_bca_last_device_status(void);
 

@@ -14,7 +14,7 @@ import workloads
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "magi_bca.h")
 
-OK, INVALID_ARG, UNSUPPORTED, BAD_OFFSETS, WS_SMALL, CUDA_ERROR, TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+OK, INVALID_ARG, UNSUPPORTED, BAD_OFFSETS, WS_SMALL, CUDA_ERROR, TIMEOUT, CHECK = 0, -1, -2, -3, -4, -5, -6, -7
 
 
 def declared_functions():
@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in (OK, INVALID_ARG, UNSUPPORTED, BAD_OFFSETS, WS_SMALL, CUDA_ERROR, TIMEOUT):
+    for code in (OK, INVALID_ARG, UNSUPPORTED, BAD_OFFSETS, WS_SMALL, CUDA_ERROR, TIMEOUT, CHECK):
         assert bca.magi_bca_status_string(code) != "unknown status"
     assert bca.magi_bca_status_string(12345) == "unknown status"
 

@@ -163,7 +163,7 @@ class ClockSampler:
 def kernel_source_sha():
     h = hashlib.sha256()
     for f in ("bca_fwd.cu", "bca_bwd.cu", "bca_bwd_split.cu", "bca_bwd_common.cuh", "sm100.cuh", "bca_norm.cuh",
-              "bca_kernels.h"):
+              "bca_kernels.h", "bca_mask.cuh"):
         p = os.path.join(ROOT, "block_causal_attention_gqa_b200", "csrc", f)
         if os.path.exists(p):
             h.update(open(p, "rb").read())

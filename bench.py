@@ -170,20 +170,26 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel, workload_name):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+def ncu_traffic_entry(kernel, workload_name):
+    """The committed ncu DRAM-traffic record of (kernel, workload), if it was
+    taken on the current kernel sources (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p))
-        e = d.get(kernel, {}).get(workload_name)
-        if e and e.get("kernel_source_sha") == kernel_source_sha():
-            return float(e["dram_bytes_per_launch"])
+        e = json.load(open(p)).get(kernel, {}).get(workload_name)
     except Exception:
         return None
+    if e and e.get("kernel_source_sha") == kernel_source_sha():
+        return e
     return None
+
+
+def ncu_traffic(kernel, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    e = ncu_traffic_entry(kernel, workload_name)
+    return float(e["dram_bytes_per_launch"]) if e else None
 
 
 # ------------------------------------------------------------------ distributed
@@ -459,6 +465,8 @@ def run_ours(args, w, world, rank, local, light=False, pass_=None, steps=None, w
                 "frac_of_sustained": round(achieved / sustained, 4),
                 "frac_of_datasheet_2250": round(achieved / DATASHEET_BF16_TFLOPS, 4),
                 "traffic": ncu_traffic(dom, w.name),
+                "traffic_source": (ncu_traffic_entry(dom, w.name) or {}).get(
+                    "source", "no ncu record at the current kernel sources"),
                 "avg_launch_ms": round(dom_ms, 4),
                 "algorithmic_bytes_per_launch": alg_bytes}
     # HBM rate of the dominant kernel: ncu's DRAM bytes per launch (and, for the

@@ -68,3 +68,35 @@ def test_forward_bytes():
     kv = 2 * 46080 * 8 * 128 * 2
     assert bench.fwd_bytes(w) == q + kv + q + 24 * 46080 * 4
     assert abs(bench.fwd_bytes(w) / 1e9 - 0.759) < 1e-3
+
+
+def test_backward_main_bytes():
+    """The backward main kernel's algorithmic bytes: Q^, dO and the 16-byte
+    {-lse, -Delta} rows read once, K^ and V read once, and the fp32 dq, dV and
+    G_k accumulators read and written once."""
+    w = workloads.workload("model46k")
+    rows_q, rows_k, D = 46080 * 24, 46080 * 8, 128
+    pad = -(-46080 // 128) * 128
+    want = (2 * rows_q * D * 2 + 24 * pad * 16 + 2 * rows_k * D * 2
+            + 2 * (rows_q * D * 4) + 2 * 2 * (rows_k * D * 4))
+    assert bench.bwd_main_bytes(w) == want
+
+
+def test_traffic_records_are_complete():
+    """Every DRAM-traffic record that bench.py may quote names its kernel
+    sources, the ncu command and where the figure comes from; a figure scaled
+    from a smaller capture says so."""
+    import json
+    import os
+    d = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles", "ncu_traffic.json")))
+    assert d
+    for kernel, per_w in d.items():
+        assert kernel in ("bca_fwd_kernel", "bca_bwd_main_kernel")
+        for name, e in per_w.items():
+            assert name in workloads.WORKLOADS, name
+            assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
+            assert len(e["kernel_source_sha"]) == 16 and e["command"].startswith("ncu ")
+            assert "--clock-control none" in e["command"]
+            assert e["source"]
+            if "long65k" in e["command"] and name != "long65k":
+                assert "scaled" in e["source"]

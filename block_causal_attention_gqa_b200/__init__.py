@@ -207,6 +207,14 @@ def _check_f32(name, t, shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _check_same_device(device, named):
+    """Every tensor of a call must live on the device the call runs on: the
+    kernels dereference each pointer there."""
+    for name, t in named:
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+
+
 def _stream_handle(stream, device):
     import torch
     if stream is None:
@@ -219,7 +227,7 @@ def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse,
     import torch
     _check_bf16("q", q)
     B, Sq, Hq, D = q.shape
-    _check_bf16("k", k)
+    _check_bf16("k", k)                     # a CUDA bf16 tensor before its shape is read
     Skv, Hkv = k.shape[1], k.shape[2]
     _check_bf16("k", k, (B, Skv, Hkv, D))
     _check_bf16("v", v, (B, Skv, Hkv, D))
@@ -233,6 +241,8 @@ def _fwd(q, k, v, q_chunk_offsets, kv_chunk_offsets, gamma_q, gamma_k, out, lse,
         lse = torch.empty(B, Hq, Sq, device=q.device, dtype=torch.float32)
     if lse is not None:
         _check_f32("lse", lse, (B, Hq, Sq))
+    _check_same_device(q.device, (("k", k), ("v", v), ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("out", out),
+                                  ("lse", lse)) + ((("rope_q", rope[0]), ("rope_k", rope[1])) if rope else ()))
     dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
                      samples=samples, n_global=n_global)
     ptr = lambda t: t.data_ptr() if t is not None else None
@@ -308,9 +318,18 @@ def _bwd(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offsets, gamma_q, ga
     if want_dgamma:
         dgamma_q = torch.empty(D, device=q.device, dtype=torch.float32) if dgamma_q is None else dgamma_q
         dgamma_k = torch.empty(D, device=q.device, dtype=torch.float32) if dgamma_k is None else dgamma_k
+    for nm, t in (("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
+        if t is not None:
+            _check_f32(nm, t, (D,))
     ws_bytes = magi_bca_bwd_workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), device=q.device, dtype=torch.uint8)
+    elif not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    _check_same_device(q.device, (("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse),
+                                  ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("dq", dq), ("dk", dk), ("dv", dv),
+                                  ("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k), ("workspace", workspace))
+                       + tuple(zip(("rope_q", "rope_k", "drope_q", "drope_k"), rope or ())))
     ptr = lambda t: t.data_ptr() if t is not None else None
     common = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
               _i32p(qo), _i32p(ko), gamma_q.data_ptr(), gamma_k.data_ptr())
@@ -391,6 +410,9 @@ def magi_bca_bwd_noalloc(q, k, v, out, dout, lse, q_chunk_offsets, kv_chunk_offs
     for nm, t in (("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
         if t is not None:
             _check_f32(nm, t, (D,))
+    _check_same_device(q.device, (("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse),
+                                  ("gamma_q", gamma_q), ("gamma_k", gamma_k), ("dq", dq), ("dk", dk), ("dv", dv),
+                                  ("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)))
     qo, ko = _offsets(q_chunk_offsets), _offsets(kv_chunk_offsets)
     dims = make_dims(B, Sq, Skv, Hq, Hkv, D, len(qo) - 1, len(ko) - 1, softmax_scale, rms_eps, kv_range,
                      deterministic, samples=samples, n_global=n_global)

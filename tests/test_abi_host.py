@@ -490,6 +490,17 @@ def test_no_cpu_fallback_host_tensors_are_refused(entry):
         calls[entry]()
 
 
+def test_tensors_on_another_device_are_refused():
+    """A call runs on q's device; a tensor elsewhere (another GPU, the host)
+    is refused before any pointer reaches a kernel."""
+    import torch
+    here = torch.device("cuda", 0)
+    t0 = torch.zeros(4)
+    with pytest.raises(ValueError, match="gamma_k is on cpu"):
+        bca._check_same_device(here, (("gamma_k", t0),))
+    bca._check_same_device(torch.device("cpu"), (("k", t0), ("lse", None)))
+
+
 def random_layouts(seed, n):
     """Seeded random chunk layouts: 1-6 kv chunks of 1-700 tokens (rarely tile
     aligned), the query side the last 1..n_kv of them (training layout when all)

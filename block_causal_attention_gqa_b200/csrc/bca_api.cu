@@ -100,13 +100,21 @@ struct ScheduleEntry {
   uint64_t last_use = 0;   // LRU clock
   int refs = 0;            // calls between lookup and launch
   bool pinned = false;     // used under stream capture: kept until release
-  std::vector<cudaStream_t> streams;  // every stream that has used it
+  // Events recorded on the caller's stream after each call's launches, so an
+  // eviction can wait for the reads without touching the callers' streams
+  // (which may have been destroyed since).  Completed ones are dropped as new
+  // ones are added; `untracked` is set if an event could not be recorded.
+  std::vector<cudaEvent_t> uses;
+  bool untracked = false;
 };
 
 struct KnormBuffer {
   void* ptr = nullptr;
   size_t bytes = 0;
   bool pinned = false;     // used under stream capture
+  // recorded after each forward's launches: growing the buffer frees the old
+  // one only after it, even if the stream handle now names a new stream
+  cudaEvent_t last_use = nullptr;
 };
 
 // Pinned staging of a schedule upload, freed once its copy has completed.
@@ -141,22 +149,18 @@ void reap_staging() {
   }
 }
 
-// Frees `ptr` in the order of `stream` after everything already enqueued on
-// `users` (caller holds g_mutex, device current).
-void free_after(void* ptr, const std::vector<cudaStream_t>& users, cudaStream_t stream) {
-  bool waited = true;
-  for (cudaStream_t u : users) {
-    if (u == stream) continue;
-    cudaEvent_t ev;
-    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
-      waited = false;
-      continue;
-    }
-    if (cudaEventRecord(ev, u) != cudaSuccess || cudaStreamWaitEvent(stream, ev, 0) != cudaSuccess) waited = false;
+// Frees a schedule's device memory in the order of `stream`, after the calls
+// that read it (their events), and destroys those events (caller holds
+// g_mutex, device current).
+void free_schedule(ScheduleEntry& e, cudaStream_t stream) {
+  bool waited = !e.untracked;
+  for (cudaEvent_t ev : e.uses) {
+    if (cudaStreamWaitEvent(stream, ev, 0) != cudaSuccess) waited = false;
     cudaEventDestroy(ev);
   }
-  if (!waited) cudaDeviceSynchronize();   // a user stream is gone: the slow, safe way
-  cudaFreeAsync(ptr, stream);
+  e.uses.clear();
+  if (!waited) cudaDeviceSynchronize();   // a use is not covered by an event: the slow, safe way
+  cudaFreeAsync(e.dev, stream);
 }
 
 int knorm_buffer(int dev, cudaStream_t stream, size_t bytes, void** out) {
@@ -173,11 +177,18 @@ int knorm_buffer(int dev, cudaStream_t stream, size_t bytes, void** out) {
                   "the first forward call for a key length must come before stream capture");
     return MAGI_BCA_UNSUPPORTED;
   }
-  // grow: the old buffer is only used on this stream, so a stream-ordered free is safe
+  // grow: the old buffer is freed in this stream's order after its last use
+  cudaEvent_t last_use = kb.last_use;
   if (kb.ptr != nullptr) {
-    if (kb.pinned) g_retired.push_back(kb.ptr); else cudaFreeAsync(kb.ptr, stream);
+    if (kb.pinned) {
+      g_retired.push_back(kb.ptr);
+    } else {
+      if (last_use != nullptr && cudaStreamWaitEvent(stream, last_use, 0) != cudaSuccess) cudaDeviceSynchronize();
+      cudaFreeAsync(kb.ptr, stream);
+    }
   }
   kb = KnormBuffer();
+  kb.last_use = last_use;
   void* ptr = nullptr;
   const cudaError_t e = cudaMallocAsync(&ptr, bytes, stream);
   if (e != cudaSuccess) return cuda_fail("cudaMallocAsync (normalised-key buffer)", e);
@@ -186,6 +197,29 @@ int knorm_buffer(int dev, cudaStream_t stream, size_t bytes, void** out) {
   *out = ptr;
   return MAGI_BCA_OK;
 }
+
+// Records the end of a forward's use of its key buffer (not under capture: a
+// buffer used there is pinned and never freed before release).
+void knorm_mark_use(int dev, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  auto it = g_knorm_bufs.find(std::make_pair(dev, reinterpret_cast<uintptr_t>(stream)));
+  if (it == g_knorm_bufs.end() || capturing(stream)) return;
+  KnormBuffer& kb = it->second;
+  if (kb.last_use == nullptr && cudaEventCreateWithFlags(&kb.last_use, cudaEventDisableTiming) != cudaSuccess) {
+    kb.last_use = nullptr;
+    return;
+  }
+  cudaEventRecord(kb.last_use, stream);
+}
+
+struct KnormUse {
+  int dev = 0;
+  cudaStream_t stream = nullptr;
+  bool held = false;
+  ~KnormUse() {
+    if (held) knorm_mark_use(dev, stream);
+  }
+};
 
 // Checks the current device once (sm_100 family) and resolves the status word.
 int device_state(int* device_out, DeviceState** st_out) {
@@ -246,7 +280,7 @@ int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, c
             (victim == g_schedules.end() || v->second.last_use < victim->second.last_use))
           victim = v;
       if (victim == g_schedules.end()) break;   // everything is in use or pinned
-      free_after(victim->second.dev, victim->second.streams, stream);
+      free_schedule(victim->second, stream);
       g_schedules.erase(victim);
       --count;
     }
@@ -281,7 +315,6 @@ int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, c
   e.last_use = ++g_clock;
   e.refs += 1;
   e.pinned = e.pinned || cap;
-  if (std::find(e.streams.begin(), e.streams.end(), stream) == e.streams.end()) e.streams.push_back(stream);
   out->dev = e.dev;
   out->n_units = e.n_units;
   out->mask = e.mask;
@@ -289,19 +322,45 @@ int get_schedule(int dev, int kind, const magi_bca_dims& d, const int32_t* qo, c
   return MAGI_BCA_OK;
 }
 
-// Ends the reference get_schedule took (after the launches that use it).
-void release_schedule(const std::vector<int32_t>& key) {
+// Ends the reference get_schedule took, after the launches that use it, and
+// records on `stream` the event an eviction will wait for.  Under stream
+// capture the entry is pinned (never evicted), so nothing is recorded.
+void release_schedule(const std::vector<int32_t>& key, cudaStream_t stream) {
   std::lock_guard<std::mutex> lock(g_mutex);
   auto it = g_schedules.find(key);
-  if (it != g_schedules.end() && it->second.refs > 0) it->second.refs -= 1;
+  if (it == g_schedules.end()) return;
+  ScheduleEntry& e = it->second;
+  if (e.refs > 0) e.refs -= 1;
+  if (capturing(stream)) return;
+  for (size_t i = 0; i < e.uses.size();) {
+    if (cudaEventQuery(e.uses[i]) == cudaSuccess) {
+      cudaEventDestroy(e.uses[i]);
+      e.uses[i] = e.uses.back();
+      e.uses.pop_back();
+    } else {
+      ++i;
+    }
+  }
+  cudaEvent_t ev;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+    e.untracked = true;
+    return;
+  }
+  if (cudaEventRecord(ev, stream) != cudaSuccess) {
+    cudaEventDestroy(ev);
+    e.untracked = true;
+    return;
+  }
+  e.uses.push_back(ev);
 }
 
 // Holds a schedule reference for the scope of an entry point.
 struct ScheduleRef {
   std::vector<int32_t> key;
+  cudaStream_t stream = nullptr;
   bool held = false;
   ~ScheduleRef() {
-    if (held) release_schedule(key);
+    if (held) release_schedule(key, stream);
   }
 };
 
@@ -458,10 +517,15 @@ int magi_bca_fwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, cs, &sched, &ref.key);
   if (st != MAGI_BCA_OK) return st;
   ref.held = true;
+  ref.stream = cs;
   const int64_t kv_rows = (int64_t)d.batch * d.seqlen_kv * d.heads_kv;
   void* kn = nullptr;
   st = knorm_buffer(dev, cs, (size_t)kv_rows * d.head_dim * 2, &kn);
   if (st != MAGI_BCA_OK) return st;
+  KnormUse kuse;
+  kuse.dev = dev;
+  kuse.stream = cs;
+  kuse.held = true;
   cudaError_t ke = launch_knorm(k, static_cast<uint16_t*>(kn), kv_rows, d.head_dim, d.rms_eps, cs, rope_k,
                                 d.heads_kv, d.seqlen_kv);
   if (ke != cudaSuccess) return cuda_fail("key normalisation launch", ke);
@@ -537,10 +601,12 @@ int magi_bca_bwd_rope(const magi_bca_bf16* q, const magi_bca_bf16* k, const magi
   st = get_schedule(dev, 1, d, q_chunk_offsets, kv_chunk_offsets, cs, &sched, &ref.key);
   if (st != MAGI_BCA_OK) return st;
   ref.held = true;
+  ref.stream = cs;
   if (d.deterministic) {   // the dq pass runs the forward's query-major units
     st = get_schedule(dev, 0, d, q_chunk_offsets, kv_chunk_offsets, cs, &dq_sched, &dq_ref.key);
     if (st != MAGI_BCA_OK) return st;
     dq_ref.held = true;
+    dq_ref.stream = cs;
   }
   uint8_t* w = static_cast<uint8_t*>(workspace);
   BwdParams p;
@@ -611,11 +677,17 @@ int magi_bca_release_caches(void) {
   devs.erase(std::unique(devs.begin(), devs.end()), devs.end());
   for (int dv : devs) {
     if (cudaSetDevice(dv) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
-    for (auto& kv : g_schedules)
-      if (kv.second.device == dv && cudaFree(kv.second.dev) != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
-    for (auto& kv : g_knorm_bufs)
-      if (kv.first.first == dv && kv.second.ptr != nullptr && cudaFree(kv.second.ptr) != cudaSuccess)
-        status = MAGI_BCA_CUDA_ERROR;
+    for (auto& kv : g_schedules) {
+      if (kv.second.device != dv) continue;
+      for (cudaEvent_t ev : kv.second.uses) cudaEventDestroy(ev);
+      kv.second.uses.clear();
+      if (cudaFree(kv.second.dev) != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
+    }
+    for (auto& kv : g_knorm_bufs) {
+      if (kv.first.first != dv) continue;
+      if (kv.second.last_use != nullptr) cudaEventDestroy(kv.second.last_use);
+      if (kv.second.ptr != nullptr && cudaFree(kv.second.ptr) != cudaSuccess) status = MAGI_BCA_CUDA_ERROR;
+    }
     if (dv == prev) {
       for (void* ptr : g_retired) cudaFree(ptr);
       g_retired.clear();
